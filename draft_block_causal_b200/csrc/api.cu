@@ -1,0 +1,223 @@
+// api.cu -- the C ABI of libdomino: argument checks, workspace layout and launch sequencing.
+// Every entry point validates on the host, then enqueues kernels on the caller's stream; it
+// never synchronises and never allocates.
+#include "domino.h"
+#include "internal.h"
+#include "persistent.h"
+
+#include <atomic>
+
+namespace domino {
+
+namespace {
+
+std::atomic<uint64_t> g_spin_limit{0};
+
+inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// K dimension in 16-byte vectors: a multiple of 32 vectors, or a power of two up to 32.
+inline bool vec_layout_ok(int K, int dtype) {
+  int nv = K / (dtype == DOMINO_DTYPE_F32 ? 4 : 8);
+  if (nv < 1) return false;
+  if (nv % 32 == 0) return true;
+  return nv <= 32 && (nv & (nv - 1)) == 0;
+}
+
+int check_shape(const domino_shape_t* s) {
+  if (!s) return DOMINO_ERR_INVALID_ARGUMENT;
+  if (s->dtype != DOMINO_DTYPE_F32 && s->dtype != DOMINO_DTYPE_BF16) return DOMINO_ERR_INVALID_ARGUMENT;
+  if (s->B < 1 || s->L < 1 || s->L > DOMINO_MAX_L || s->d < 8 || s->Hs < 8 || s->r < 8 || s->V < 8)
+    return DOMINO_ERR_INVALID_ARGUMENT;
+  if (s->d % 8 || s->Hs % 8 || s->r % 8 || s->V % 8) return DOMINO_ERR_INVALID_ARGUMENT;
+  if ((int64_t)s->B * s->L > (1 << 19)) return DOMINO_ERR_UNSUPPORTED;
+  if (s->r > 1024) return DOMINO_ERR_UNSUPPORTED;
+  if (!vec_layout_ok(s->d, s->dtype) || !vec_layout_ok(s->Hs, s->dtype) || !vec_layout_ok(s->r, s->dtype))
+    return DOMINO_ERR_UNSUPPORTED;
+  return DOMINO_OK;
+}
+
+int check_weights(const domino_weights_t* w) {
+  if (!w) return DOMINO_ERR_INVALID_ARGUMENT;
+  const void* p[] = {w->embed, w->W_ih, w->W_hh, w->b_ih, w->b_hh, w->W1, w->W2};
+  for (const void* q : p)
+    if (!q || !aligned16(q)) return DOMINO_ERR_INVALID_ARGUMENT;
+  return DOMINO_OK;
+}
+
+Shape to_shape(const domino_shape_t* s) { return Shape{s->B, s->L, s->d, s->Hs, s->r, s->V, s->dtype}; }
+
+inline int cuda_rc(cudaError_t e) { return e == cudaSuccess ? DOMINO_OK : DOMINO_ERR_CUDA; }
+
+}  // namespace
+
+Workspace layout_workspace(const Shape& s, void* base) {
+  Workspace w{};
+  char* p = static_cast<char*>(base);
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    size_t o = off;
+    off = align256(off + bytes);
+    return p ? p + o : nullptr;
+  };
+  const size_t BL = (size_t)s.B * s.L;
+  w.status = reinterpret_cast<int32_t*>(take(sizeof(int32_t)));
+  w.sync = reinterpret_cast<uint32_t*>(take(kSyncWords * sizeof(uint32_t)));
+  w.keys = reinterpret_cast<uint64_t*>(take(BL * sizeof(uint64_t)));
+  w.acc_keys = reinterpret_cast<uint64_t*>(take(BL * sizeof(uint64_t)));
+  w.P = reinterpret_cast<float*>(take(BL * s.r * sizeof(float)));
+  w.u = reinterpret_cast<float*>(take(BL * s.r * sizeof(float)));
+  w.S = reinterpret_cast<float*>(take(2 * (size_t)s.B * s.Hs * sizeof(float)));
+  w.states = reinterpret_cast<float*>(take(BL * s.Hs * sizeof(float)));
+  w.a_acc = reinterpret_cast<float*>(take(BL * s.r * sizeof(float)));
+  w.bytes = off;
+  return w;
+}
+
+size_t accept_workspace_bytes(int B, int L) {
+  // the accept path uses the status word and acc_keys of the general layout
+  Shape s{B, L, 8, 8, 8, 8, DOMINO_DTYPE_F32};
+  Workspace w = layout_workspace(s, nullptr);
+  return w.bytes;
+}
+
+uint64_t spin_limit() {
+  uint64_t v = g_spin_limit.load(std::memory_order_relaxed);
+  return v ? v : kDefaultSpinLimit;
+}
+
+}  // namespace domino
+
+using namespace domino;
+
+extern "C" {
+
+int32_t domino_abi_version(void) { return DOMINO_ABI_VERSION; }
+
+int domino_debug_set_spin_limit(uint64_t limit) {
+  g_spin_limit.store(limit, std::memory_order_relaxed);
+  return DOMINO_OK;
+}
+
+const char* domino_status_string(int code) {
+  switch (code) {
+    case DOMINO_OK: return "ok";
+    case DOMINO_ERR_INVALID_ARGUMENT: return "invalid argument (null pointer, bad shape or misalignment)";
+    case DOMINO_ERR_UNSUPPORTED: return "unsupported shape, layout or device";
+    case DOMINO_ERR_CUDA: return "CUDA launch or query failed";
+    case DOMINO_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case DOMINO_STATUS_DEVICE_TIMEOUT: return "device: a bounded wait gave up (outputs invalid)";
+    case DOMINO_STATUS_BAD_TOKEN: return "device: teacher-forcing token outside [0, V)";
+    default: return "unknown code";
+  }
+}
+
+size_t domino_workspace_bytes(const domino_shape_t* shape) {
+  if (check_shape(shape) != DOMINO_OK) return 0;
+  return layout_workspace(to_shape(shape), nullptr).bytes;
+}
+
+size_t domino_accept_workspace_bytes(int32_t B, int32_t L) {
+  if (B < 1 || L < 1 || L > DOMINO_MAX_L) return 0;
+  return accept_workspace_bytes(B, L);
+}
+
+int domino_draft_greedy(const domino_shape_t* shape, const domino_weights_t* w, const void* base_logits,
+                        const void* hidden, const float* S0, int32_t* tokens_out, float* logits_out,
+                        float* states_out, void* workspace, size_t workspace_bytes, int32_t* status_dev,
+                        domino_stream_t stream) {
+  int rc = check_shape(shape);
+  if (rc != DOMINO_OK) return rc;
+  if ((rc = check_weights(w)) != DOMINO_OK) return rc;
+  if (!base_logits || !hidden || !S0 || !tokens_out) return DOMINO_ERR_INVALID_ARGUMENT;
+  if (!aligned16(base_logits) || !aligned16(hidden) || !aligned16(S0) || !aligned16(tokens_out) ||
+      (logits_out && !aligned16(logits_out)) || (states_out && !aligned16(states_out)))
+    return DOMINO_ERR_INVALID_ARGUMENT;
+  const Shape s = to_shape(shape);
+  const Workspace need = layout_workspace(s, nullptr);
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || workspace_bytes < need.bytes)
+    return DOMINO_ERR_WORKSPACE;
+  const Workspace ws = layout_workspace(s, workspace);
+  int32_t* st = status_dev ? status_dev : ws.status;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+
+  if (use_persistent_greedy(s)) return cuda_rc(launch_persistent_greedy(s, *w, base_logits, hidden, S0, tokens_out,
+                                                                         logits_out, states_out, ws, st,
+                                                                         spin_limit(), cs));
+
+  const size_t BL = (size_t)s.B * s.L;
+  cudaError_t e = cudaMemsetAsync(ws.keys, 0, BL * sizeof(uint64_t), cs);
+  if (e == cudaSuccess) e = launch_hproj(s, w->W1, hidden, (int)BL, ws.P, cs);
+  if (e == cudaSuccess && states_out) e = launch_copy_rows(S0, s.Hs, states_out, (size_t)s.L * s.Hs, s.B, s.Hs, cs);
+  const float* S_cur = S0;
+  for (int i = 0; i < s.L && e == cudaSuccess; ++i) {
+    e = launch_u(s, w->W1, ws.P, s.L, i, S_cur, s.Hs, s.B, ws.u, cs);
+    if (e == cudaSuccess)
+      e = launch_w2(s, w->W2, ws.u, s.B, base_logits, s.L, i, ws.keys + (size_t)i * s.B, logits_out, cs);
+    if (e == cudaSuccess && i < s.L - 1) {
+      float* S_next = ws.S + (size_t)(i & 1) * s.B * s.Hs;
+      e = launch_gru(s, w->embed, w->W_ih, w->W_hh, w->b_ih, w->b_hh, ws.keys + (size_t)i * s.B, nullptr, 0, 0,
+                     S_cur, s.Hs, S_next, s.Hs, states_out ? states_out + (size_t)(i + 1) * s.Hs : nullptr,
+                     (size_t)s.L * s.Hs, s.B, st, cs);
+      S_cur = S_next;
+    }
+  }
+  if (e == cudaSuccess) e = launch_tokens_from_keys(ws.keys, s.B, s.L, tokens_out, cs);
+  return cuda_rc(e);
+}
+
+int domino_teacher_forced(const domino_shape_t* shape, const domino_weights_t* w, const void* base_logits,
+                          const void* hidden, const float* S0, const int32_t* tokens, float* logits_out,
+                          float* states_out, void* workspace, size_t workspace_bytes, int32_t* status_dev,
+                          domino_stream_t stream) {
+  int rc = check_shape(shape);
+  if (rc != DOMINO_OK) return rc;
+  if ((rc = check_weights(w)) != DOMINO_OK) return rc;
+  if (!base_logits || !hidden || !S0 || !tokens || !logits_out) return DOMINO_ERR_INVALID_ARGUMENT;
+  if (!aligned16(base_logits) || !aligned16(hidden) || !aligned16(S0) || !aligned16(tokens) ||
+      !aligned16(logits_out) || (states_out && !aligned16(states_out)))
+    return DOMINO_ERR_INVALID_ARGUMENT;
+  const Shape s = to_shape(shape);
+  const Workspace need = layout_workspace(s, nullptr);
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || workspace_bytes < need.bytes)
+    return DOMINO_ERR_WORKSPACE;
+  const Workspace ws = layout_workspace(s, workspace);
+  int32_t* st = status_dev ? status_dev : ws.status;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+
+  const size_t BL = (size_t)s.B * s.L;
+  float* SB = states_out ? states_out : ws.states;  // [B][L][Hs]
+  const size_t row = (size_t)s.L * s.Hs;
+  cudaError_t e = launch_hproj(s, w->W1, hidden, (int)BL, ws.P, cs);
+  if (e == cudaSuccess) e = launch_copy_rows(S0, s.Hs, SB, row, s.B, s.Hs, cs);
+  for (int i = 0; i + 1 < s.L && e == cudaSuccess; ++i)
+    e = launch_gru(s, w->embed, w->W_ih, w->W_hh, w->b_ih, w->b_hh, nullptr, tokens, s.L, i, SB + (size_t)i * s.Hs,
+                   row, SB + (size_t)(i + 1) * s.Hs, row, nullptr, 0, s.B, st, cs);
+  if (e == cudaSuccess) e = launch_u(s, w->W1, ws.P, 1, 0, SB, s.Hs, (int)BL, ws.u, cs);
+  if (e == cudaSuccess) e = launch_w2(s, w->W2, ws.u, (int)BL, base_logits, 1, 0, nullptr, logits_out, cs);
+  return cuda_rc(e);
+}
+
+int domino_accept_len(int32_t B, int32_t L, int32_t V, const int32_t* draft_tokens, const float* target_logits,
+                      int32_t* accept_out, void* workspace, size_t workspace_bytes, int32_t* status_dev,
+                      domino_stream_t stream) {
+  (void)status_dev;
+  if (B < 1 || L < 1 || L > DOMINO_MAX_L || V < 8 || V % 8) return DOMINO_ERR_INVALID_ARGUMENT;
+  if ((int64_t)B * L > (1 << 19)) return DOMINO_ERR_UNSUPPORTED;
+  if (!draft_tokens || !target_logits || !accept_out) return DOMINO_ERR_INVALID_ARGUMENT;
+  if (!aligned16(target_logits)) return DOMINO_ERR_INVALID_ARGUMENT;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) ||
+      workspace_bytes < accept_workspace_bytes(B, L))
+    return DOMINO_ERR_WORKSPACE;
+  Shape s{B, L, 8, 8, 8, 8, DOMINO_DTYPE_F32};
+  const Workspace ws = layout_workspace(s, workspace);
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  const size_t BL = (size_t)B * L;
+  cudaError_t e = cudaMemsetAsync(ws.acc_keys, 0, BL * sizeof(uint64_t), cs);
+  if (e == cudaSuccess) e = launch_row_argmax(target_logits, (int)BL, V, ws.acc_keys, cs);
+  if (e == cudaSuccess) e = launch_accept_count(draft_tokens, ws.acc_keys, B, L, accept_out, cs);
+  return cuda_rc(e);
+}
+
+}  // extern "C"

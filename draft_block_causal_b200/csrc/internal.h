@@ -1,0 +1,49 @@
+// internal.h -- host-side declarations shared by the libdomino translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace domino {
+
+struct Shape {
+  int B, L, d, Hs, r, V, dtype;
+};
+
+// Scratch layout inside the caller's workspace.  Every region starts on a 256-byte boundary.
+struct Workspace {
+  int32_t* status;     // fallback status word when the caller passes no status pointer
+  uint32_t* sync;      // barrier counters of the persistent kernels (kSyncWords words)
+  uint64_t* keys;      // [L][B]   greedy argmax keys per position
+  uint64_t* acc_keys;  // [B*L]    target-logit argmax keys (accept length)
+  float* P;            // [B*L][r] W1 . H for every position
+  float* u;            // [B*L][r] SiLU activations
+  float* S;            // [2][B][Hs] greedy state ping-pong
+  float* states;       // [B][L][Hs] teacher-forced states when the caller keeps none
+  float* a_acc;        // [L][B][r] pre-activation accumulators of the fused greedy kernel
+  size_t bytes;
+};
+constexpr int kSyncWords = 64;
+
+Workspace layout_workspace(const Shape& s, void* base);
+size_t accept_workspace_bytes(int B, int L);
+
+// ---- step kernels (one launch per phase; any storage type, any batch) ----
+cudaError_t launch_hproj(const Shape& s, const void* W1, const void* hidden, int N, float* P, cudaStream_t st);
+cudaError_t launch_u(const Shape& s, const void* W1, const float* P, int p_mul, int p_add, const float* S,
+                     size_t s_stride, int M, float* u, cudaStream_t st);
+cudaError_t launch_w2(const Shape& s, const void* W2, const float* u, int M, const void* Lb, int l_mul,
+                      int l_add, uint64_t* keys, float* logits, cudaStream_t st);
+cudaError_t launch_gru(const Shape& s, const void* embed, const void* W_ih, const void* W_hh, const void* b_ih,
+                       const void* b_hh, const uint64_t* tok_keys, const int32_t* tokens, int tok_mul, int tok_add,
+                       const float* Sin, size_t sin_stride, float* Sout, size_t sout_stride, float* Sout2,
+                       size_t sout2_stride, int M, int32_t* status, cudaStream_t st);
+cudaError_t launch_tokens_from_keys(const uint64_t* keys, int B, int L, int32_t* tokens, cudaStream_t st);
+cudaError_t launch_copy_rows(const float* src, size_t src_stride, float* dst, size_t dst_stride, int rows, int n,
+                             cudaStream_t st);
+cudaError_t launch_row_argmax(const float* T, int rows, int V, uint64_t* keys, cudaStream_t st);
+cudaError_t launch_accept_count(const int32_t* draft, const uint64_t* keys, int B, int L, int32_t* out,
+                                cudaStream_t st);
+
+}  // namespace domino

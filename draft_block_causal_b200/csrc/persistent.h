@@ -1,0 +1,21 @@
+// persistent.h -- the fused, persistent greedy-drafting kernel (small batch).
+#pragma once
+
+#include "domino.h"
+#include "internal.h"
+
+namespace domino {
+
+// Default iteration limit of bounded device-wide waits (about a second of polling).
+constexpr uint64_t kDefaultSpinLimit = 1ull << 22;
+uint64_t spin_limit();
+
+// True when the fused persistent kernel handles this shape (else the step kernels do).
+bool use_persistent_greedy(const Shape& s);
+
+cudaError_t launch_persistent_greedy(const Shape& s, const domino_weights_t& w, const void* base_logits,
+                                     const void* hidden, const float* S0, int32_t* tokens_out, float* logits_out,
+                                     float* states_out, const Workspace& ws, int32_t* status, uint64_t spin_limit,
+                                     cudaStream_t st);
+
+}  // namespace domino

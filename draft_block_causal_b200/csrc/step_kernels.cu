@@ -1,0 +1,391 @@
+// step_kernels.cu -- one-launch-per-phase kernels of the Domino head (any storage type, any
+// batch).  They compute, phase by phase, the equations of the Domino review page, section 二:
+//   P = W1[:, :d] . H                 (H-projection, all positions)
+//   u = SiLU(P + W1[:, d:] . S)        (low-rank activation)
+//   z = L_base + W2 . u, argmax        (logit-space residual, fused vocabulary argmax)
+//   S' = GRUCell(embed[t], S)          (causal encoder update)
+// and the accept-length check.  A warp owns one output row of the weight matrix and applies it
+// to a tile of up to kTileM right-hand vectors, so each weight row is read once per tile.
+#include "common.cuh"
+#include "internal.h"
+
+namespace domino {
+
+namespace {
+
+constexpr int kWarps = 8;
+constexpr int kThreads = kWarps * 32;
+constexpr int kTileM = 8;
+
+// fp32 vector of N elements at p (16-byte aligned), N in {4, 8}.
+template <int N> __device__ __forceinline__ void load_f32(const float* p, float (&f)[N]) {
+  const float4* q = reinterpret_cast<const float4*>(p);
+#pragma unroll
+  for (int i = 0; i < N / 4; ++i) {
+    float4 v = __ldg(q + i);
+    f[4 * i] = v.x; f[4 * i + 1] = v.y; f[4 * i + 2] = v.z; f[4 * i + 3] = v.w;
+  }
+}
+
+// P[n][k] = sum_c W1[k][c] H[n][c]
+template <typename T>
+__global__ void __launch_bounds__(kThreads) k_hproj(const T* __restrict__ W1, int ldw, const T* __restrict__ H,
+                                                    int N, int d, int r, float* __restrict__ P) {
+  constexpr int E = Vec<T>::N;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int k = blockIdx.x * kWarps + warp;
+  if (k >= r) return;
+  const int n0 = blockIdx.y * kTileM;
+  float acc[kTileM];
+#pragma unroll
+  for (int m = 0; m < kTileM; ++m) acc[m] = 0.f;
+  const T* wrow = W1 + (size_t)k * ldw;
+  for (int q = lane; q < d / E; q += 32) {
+    float w[E];
+    widen(ldg16(wrow + q * E), w);
+#pragma unroll
+    for (int m = 0; m < kTileM; ++m) {
+      if (n0 + m < N) {
+        float h[E];
+        widen(ldg16(H + (size_t)(n0 + m) * d + q * E), h);
+#pragma unroll
+        for (int e = 0; e < E; ++e) acc[m] = fmaf(w[e], h[e], acc[m]);
+      }
+    }
+  }
+#pragma unroll
+  for (int m = 0; m < kTileM; ++m) {
+    float s = warp_sum(acc[m]);
+    if (lane == 0 && n0 + m < N) P[(size_t)(n0 + m) * r + k] = s;
+  }
+}
+
+// u[m][k] = SiLU(P[m*p_mul + p_add][k] + sum_j W1[k][d+j] S[m][j])
+template <typename T>
+__global__ void __launch_bounds__(kThreads) k_u(const T* __restrict__ W1, int ldw, int d, int Hs, int r,
+                                                const float* __restrict__ P, int p_mul, int p_add,
+                                                const float* __restrict__ S, size_t s_stride, int M,
+                                                float* __restrict__ u) {
+  constexpr int E = Vec<T>::N;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int k = blockIdx.x * kWarps + warp;
+  if (k >= r) return;
+  const int m0 = blockIdx.y * kTileM;
+  float acc[kTileM];
+#pragma unroll
+  for (int m = 0; m < kTileM; ++m) acc[m] = 0.f;
+  const T* wrow = W1 + (size_t)k * ldw + d;
+  for (int q = lane; q < Hs / E; q += 32) {
+    float w[E];
+    widen(ldg16(wrow + q * E), w);
+#pragma unroll
+    for (int m = 0; m < kTileM; ++m) {
+      if (m0 + m < M) {
+        float h[E];
+        load_f32<E>(S + (size_t)(m0 + m) * s_stride + q * E, h);
+#pragma unroll
+        for (int e = 0; e < E; ++e) acc[m] = fmaf(w[e], h[e], acc[m]);
+      }
+    }
+  }
+#pragma unroll
+  for (int m = 0; m < kTileM; ++m) {
+    float s = warp_sum(acc[m]);
+    if (lane == 0 && m0 + m < M) {
+      float a = P[(size_t)((m0 + m) * p_mul + p_add) * r + k] + s;
+      u[(size_t)(m0 + m) * r + k] = siluf_(a);
+    }
+  }
+}
+
+// z[m][v] = Lb[row(m)][v] + sum_k W2[v][k] u[m][k],  row(m) = m*l_mul + l_add.
+// keys != null: keys[m] = max(keys[m], argmax_key(z, v)).  logits != null: logits[row(m)][v] = z.
+template <typename T>
+__global__ void __launch_bounds__(kThreads) k_w2(const T* __restrict__ W2, int r, int V, const float* __restrict__ u,
+                                                 int M, const T* __restrict__ Lb, int l_mul, int l_add,
+                                                 uint64_t* __restrict__ keys, float* __restrict__ logits) {
+  constexpr int E = Vec<T>::N;
+  extern __shared__ float u_s[];  // [kTileM][r]
+  __shared__ uint64_t best_s[kWarps][kTileM];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int m0 = blockIdx.y * kTileM;
+  const int mt = min(kTileM, M - m0);
+  for (int i = threadIdx.x; i < kTileM * r; i += kThreads) {
+    int m = i / r;
+    u_s[i] = (m < mt) ? u[(size_t)(m0 + m) * r + (i % r)] : 0.f;
+  }
+  __syncthreads();
+  uint64_t best[kTileM];
+#pragma unroll
+  for (int m = 0; m < kTileM; ++m) best[m] = 0ull;
+  for (int v = blockIdx.x * kWarps + warp; v < V; v += gridDim.x * kWarps) {
+    float acc[kTileM];
+#pragma unroll
+    for (int m = 0; m < kTileM; ++m) acc[m] = 0.f;
+    const T* wrow = W2 + (size_t)v * r;
+    for (int q = lane; q < r / E; q += 32) {
+      float w[E];
+      widen(ldg16(wrow + q * E), w);
+#pragma unroll
+      for (int m = 0; m < kTileM; ++m) {
+#pragma unroll
+        for (int e = 0; e < E; ++e) acc[m] = fmaf(w[e], u_s[m * r + q * E + e], acc[m]);
+      }
+    }
+#pragma unroll
+    for (int m = 0; m < kTileM; ++m) {
+      float s = warp_sum(acc[m]);
+      if (lane == 0 && m < mt) {
+        size_t row = (size_t)(m0 + m) * l_mul + l_add;
+        float z = to_f32(Lb[row * V + v]) + s;
+        if (logits) logits[row * V + v] = z;
+        best[m] = umax64(best[m], argmax_key(z, v));
+      }
+    }
+  }
+  if (keys) {
+    if (lane == 0) {
+#pragma unroll
+      for (int m = 0; m < kTileM; ++m) best_s[warp][m] = best[m];
+    }
+    __syncthreads();
+    if (threadIdx.x < mt) {
+      uint64_t b = 0ull;
+      for (int w = 0; w < kWarps; ++w) b = umax64(b, best_s[w][threadIdx.x]);
+      atomicMax(reinterpret_cast<unsigned long long*>(keys + m0 + threadIdx.x), (unsigned long long)b);
+    }
+  }
+}
+
+// GRU update, PyTorch GRUCell form, for every row m < M and unit j < Hs:
+//   t = tok_keys ? index(tok_keys[m]) : tokens[m*tok_mul + tok_add];  x = embed[t];  h = Sin[m]
+//   r = sig(gi_r + gh_r), z = sig(gi_z + gh_z), n = tanh(gi_n + r * gh_n), h' = (1-z) n + z h[j]
+template <typename T>
+__global__ void __launch_bounds__(kThreads) k_gru(const T* __restrict__ embed, const T* __restrict__ W_ih,
+                                                  const T* __restrict__ W_hh, const T* __restrict__ b_ih,
+                                                  const T* __restrict__ b_hh, int d, int Hs, int V,
+                                                  const uint64_t* __restrict__ tok_keys,
+                                                  const int32_t* __restrict__ tokens, int tok_mul, int tok_add,
+                                                  const float* __restrict__ Sin, size_t sin_stride,
+                                                  float* __restrict__ Sout, size_t sout_stride,
+                                                  float* __restrict__ Sout2, size_t sout2_stride, int M,
+                                                  int32_t* __restrict__ status) {
+  constexpr int E = Vec<T>::N;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int j = blockIdx.x * kWarps + warp;
+  if (j >= Hs) return;
+  const int m0 = blockIdx.y * kTileM;
+  const T* xrow[kTileM];
+  bool ok[kTileM];
+#pragma unroll
+  for (int m = 0; m < kTileM; ++m) {
+    int t = 0;
+    ok[m] = false;
+    if (m0 + m < M) {
+      t = tok_keys ? key_index(tok_keys[m0 + m]) : tokens[(size_t)(m0 + m) * tok_mul + tok_add];
+      ok[m] = (t >= 0 && t < V);
+      if (!ok[m] && lane == 0 && j == 0) set_status(status, 2 /* DOMINO_STATUS_BAD_TOKEN */);
+    }
+    xrow[m] = embed + (size_t)(ok[m] ? t : 0) * d;
+  }
+  float gi[3][kTileM], gh[3][kTileM];
+#pragma unroll
+  for (int g = 0; g < 3; ++g)
+#pragma unroll
+    for (int m = 0; m < kTileM; ++m) gi[g][m] = gh[g][m] = 0.f;
+  for (int q = lane; q < d / E; q += 32) {
+    float w[3][E];
+#pragma unroll
+    for (int g = 0; g < 3; ++g) widen(ldg16(W_ih + ((size_t)g * Hs + j) * d + q * E), w[g]);
+#pragma unroll
+    for (int m = 0; m < kTileM; ++m) {
+      if (ok[m]) {
+        float x[E];
+        widen(ldg16(xrow[m] + q * E), x);
+#pragma unroll
+        for (int g = 0; g < 3; ++g)
+#pragma unroll
+          for (int e = 0; e < E; ++e) gi[g][m] = fmaf(w[g][e], x[e], gi[g][m]);
+      }
+    }
+  }
+  for (int q = lane; q < Hs / E; q += 32) {
+    float w[3][E];
+#pragma unroll
+    for (int g = 0; g < 3; ++g) widen(ldg16(W_hh + ((size_t)g * Hs + j) * Hs + q * E), w[g]);
+#pragma unroll
+    for (int m = 0; m < kTileM; ++m) {
+      if (m0 + m < M) {
+        float h[E];
+        load_f32<E>(Sin + (size_t)(m0 + m) * sin_stride + q * E, h);
+#pragma unroll
+        for (int g = 0; g < 3; ++g)
+#pragma unroll
+          for (int e = 0; e < E; ++e) gh[g][m] = fmaf(w[g][e], h[e], gh[g][m]);
+      }
+    }
+  }
+  float bi[3], bh[3];
+#pragma unroll
+  for (int g = 0; g < 3; ++g) {
+    bi[g] = to_f32(b_ih[(size_t)g * Hs + j]);
+    bh[g] = to_f32(b_hh[(size_t)g * Hs + j]);
+  }
+#pragma unroll
+  for (int m = 0; m < kTileM; ++m) {
+    float si[3], sh[3];
+#pragma unroll
+    for (int g = 0; g < 3; ++g) {
+      si[g] = warp_sum(gi[g][m]) + bi[g];
+      sh[g] = warp_sum(gh[g][m]) + bh[g];
+    }
+    if (lane == 0 && m0 + m < M) {
+      float h = Sin[(size_t)(m0 + m) * sin_stride + j];
+      float rg = sigmoidf_(si[0] + sh[0]);
+      float zg = sigmoidf_(si[1] + sh[1]);
+      float ng = tanhf(si[2] + rg * sh[2]);
+      float hn = (1.f - zg) * ng + zg * h;
+      Sout[(size_t)(m0 + m) * sout_stride + j] = hn;
+      if (Sout2) Sout2[(size_t)(m0 + m) * sout2_stride + j] = hn;
+    }
+  }
+}
+
+__global__ void k_tokens_from_keys(const uint64_t* __restrict__ keys, int B, int L, int32_t* __restrict__ tokens) {
+  int n = blockIdx.x * blockDim.x + threadIdx.x;
+  if (n >= B * L) return;
+  int b = n / L, i = n % L;
+  tokens[n] = key_index(keys[(size_t)i * B + b]);
+}
+
+__global__ void k_copy_rows(const float* __restrict__ src, size_t src_stride, float* __restrict__ dst,
+                            size_t dst_stride, int rows, int n) {
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < rows * n; i += gridDim.x * blockDim.x) {
+    int m = i / n, c = i % n;
+    dst[(size_t)m * dst_stride + c] = src[(size_t)m * src_stride + c];
+  }
+}
+
+// keys[n] = max over the row of argmax_key(T[n][v], v); blockIdx.y = row, blockIdx.x = chunk.
+constexpr int kArgChunk = 8192;
+__global__ void __launch_bounds__(256) k_row_argmax(const float* __restrict__ T, int V, uint64_t* __restrict__ keys) {
+  __shared__ uint64_t red[8];
+  const int n = blockIdx.y;
+  const int v0 = blockIdx.x * kArgChunk;
+  const int v1 = min(V, v0 + kArgChunk);
+  const float* row = T + (size_t)n * V;
+  uint64_t best = 0ull;
+  for (int v = v0 + 4 * threadIdx.x; v < v1; v += 4 * blockDim.x) {
+    float4 q = __ldcs(reinterpret_cast<const float4*>(row + v));
+    best = umax64(best, argmax_key(q.x, v));
+    best = umax64(best, argmax_key(q.y, v + 1));
+    best = umax64(best, argmax_key(q.z, v + 2));
+    best = umax64(best, argmax_key(q.w, v + 3));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) best = umax64(best, __shfl_xor_sync(0xffffffffu, best, o));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = best;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    for (int w = 1; w < (int)(blockDim.x >> 5); ++w) best = umax64(best, red[w]);
+    atomicMax(reinterpret_cast<unsigned long long*>(keys + n), (unsigned long long)best);
+  }
+}
+
+__global__ void k_accept_count(const int32_t* __restrict__ draft, const uint64_t* __restrict__ keys, int B, int L,
+                               int32_t* __restrict__ out) {
+  int b = blockIdx.x * blockDim.x + threadIdx.x;
+  if (b >= B) return;
+  int k = 0;
+  for (int j = 0; j < L; ++j) {
+    if (draft[(size_t)b * L + j] != key_index(keys[(size_t)b * L + j])) break;
+    k = j + 1;
+  }
+  out[b] = k;
+}
+
+inline unsigned cdiv(size_t a, size_t b) { return (unsigned)((a + b - 1) / b); }
+
+}  // namespace
+
+cudaError_t launch_hproj(const Shape& s, const void* W1, const void* hidden, int N, float* P, cudaStream_t st) {
+  dim3 grid(cdiv(s.r, kWarps), cdiv(N, kTileM));
+  if (s.dtype == 0)
+    k_hproj<float><<<grid, kThreads, 0, st>>>((const float*)W1, s.d + s.Hs, (const float*)hidden, N, s.d, s.r, P);
+  else
+    k_hproj<bf16><<<grid, kThreads, 0, st>>>((const bf16*)W1, s.d + s.Hs, (const bf16*)hidden, N, s.d, s.r, P);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_u(const Shape& s, const void* W1, const float* P, int p_mul, int p_add, const float* S,
+                     size_t s_stride, int M, float* u, cudaStream_t st) {
+  dim3 grid(cdiv(s.r, kWarps), cdiv(M, kTileM));
+  if (s.dtype == 0)
+    k_u<float><<<grid, kThreads, 0, st>>>((const float*)W1, s.d + s.Hs, s.d, s.Hs, s.r, P, p_mul, p_add, S,
+                                          s_stride, M, u);
+  else
+    k_u<bf16><<<grid, kThreads, 0, st>>>((const bf16*)W1, s.d + s.Hs, s.d, s.Hs, s.r, P, p_mul, p_add, S,
+                                         s_stride, M, u);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_w2(const Shape& s, const void* W2, const float* u, int M, const void* Lb, int l_mul, int l_add,
+                      uint64_t* keys, float* logits, cudaStream_t st) {
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  unsigned gx = (unsigned)min((size_t)sms * 4, (size_t)cdiv(s.V, kWarps));
+  dim3 grid(gx, cdiv(M, kTileM));
+  size_t smem = (size_t)kTileM * s.r * sizeof(float);
+  if (s.dtype == 0)
+    k_w2<float><<<grid, kThreads, smem, st>>>((const float*)W2, s.r, s.V, u, M, (const float*)Lb, l_mul, l_add,
+                                              keys, logits);
+  else
+    k_w2<bf16><<<grid, kThreads, smem, st>>>((const bf16*)W2, s.r, s.V, u, M, (const bf16*)Lb, l_mul, l_add, keys,
+                                             logits);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gru(const Shape& s, const void* embed, const void* W_ih, const void* W_hh, const void* b_ih,
+                       const void* b_hh, const uint64_t* tok_keys, const int32_t* tokens, int tok_mul, int tok_add,
+                       const float* Sin, size_t sin_stride, float* Sout, size_t sout_stride, float* Sout2,
+                       size_t sout2_stride, int M, int32_t* status, cudaStream_t st) {
+  dim3 grid(cdiv(s.Hs, kWarps), cdiv(M, kTileM));
+  if (s.dtype == 0)
+    k_gru<float><<<grid, kThreads, 0, st>>>((const float*)embed, (const float*)W_ih, (const float*)W_hh,
+                                            (const float*)b_ih, (const float*)b_hh, s.d, s.Hs, s.V, tok_keys, tokens,
+                                            tok_mul, tok_add, Sin, sin_stride, Sout, sout_stride, Sout2,
+                                            sout2_stride, M, status);
+  else
+    k_gru<bf16><<<grid, kThreads, 0, st>>>((const bf16*)embed, (const bf16*)W_ih, (const bf16*)W_hh,
+                                           (const bf16*)b_ih, (const bf16*)b_hh, s.d, s.Hs, s.V, tok_keys, tokens,
+                                           tok_mul, tok_add, Sin, sin_stride, Sout, sout_stride, Sout2, sout2_stride,
+                                           M, status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_tokens_from_keys(const uint64_t* keys, int B, int L, int32_t* tokens, cudaStream_t st) {
+  k_tokens_from_keys<<<cdiv((size_t)B * L, 256), 256, 0, st>>>(keys, B, L, tokens);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_copy_rows(const float* src, size_t src_stride, float* dst, size_t dst_stride, int rows, int n,
+                             cudaStream_t st) {
+  unsigned g = min(cdiv((size_t)rows * n, 256), 4096u);
+  k_copy_rows<<<g, 256, 0, st>>>(src, src_stride, dst, dst_stride, rows, n);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_row_argmax(const float* T, int rows, int V, uint64_t* keys, cudaStream_t st) {
+  dim3 grid(cdiv(V, kArgChunk), rows);
+  k_row_argmax<<<grid, 256, 0, st>>>(T, V, keys);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_accept_count(const int32_t* draft, const uint64_t* keys, int B, int L, int32_t* out,
+                                cudaStream_t st) {
+  k_accept_count<<<cdiv(B, 128), 128, 0, st>>>(draft, keys, B, L, out);
+  return cudaGetLastError();
+}
+
+}  // namespace domino

@@ -1,0 +1,160 @@
+/*
+ * domino.h -- C ABI of libdomino, the B200 (sm_100a) implementation of the Domino head.
+ *
+ * The Domino head (Domino review page, paper.oopus.info, section 二 "Domino Head") turns the
+ * parallel backbone's outputs for one draft block -- hidden states H[i] and base logits
+ * L_base[i] at every position i -- into corrected logits
+ *
+ *     L_final[i] = L_base[i] + W2 . SiLU(W1 . [H[i] ; S_{i-1}])
+ *
+ * where S_{i-1} is the state of a GRU causal encoder (hidden size Hs, 1024 on the pages) that has
+ * read the embeddings of the tokens drafted before position i.  W1 is rank r (256 on the pages)
+ * and W2 maps r -> V over the whole vocabulary; the LM head is not recomputed.
+ *
+ * Conventions shared by every entry point
+ *   - Every pointer is caller-owned device memory (cudaMalloc / PyTorch), row-major, contiguous
+ *     and 16-byte aligned, unless stated otherwise.  The library allocates nothing: scratch
+ *     memory is the caller's workspace.
+ *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy default stream) and
+ *     never synchronises the host.  Calls that share a workspace must be ordered on the GPU.
+ *   - Host-side checks happen before any launch: on a negative return code nothing was enqueued.
+ *   - Device-side problems (a bounded wait that gave up, a token outside [0, V)) are reported by
+ *     writing a positive DOMINO_STATUS_* code to *status_dev with an atomic compare-and-swap from
+ *     0, so the first problem wins.  The library never clears *status_dev: zero it before the
+ *     call and read it after your own synchronisation.  status_dev may be NULL, in which case
+ *     the code lands in a word inside the workspace.
+ *   - Storage type (`dtype`): DOMINO_DTYPE_BF16 means embed, W_ih, W_hh, b_ih, b_hh, W1, W2,
+ *     base_logits and hidden are bf16; DOMINO_DTYPE_F32 means they are fp32.  S0, states,
+ *     logits and target logits are always fp32; tokens are int32.  Arithmetic accumulates in
+ *     fp32 in every mode.
+ *   - Shapes: 1 <= B, 1 <= L <= DOMINO_MAX_L; d, Hs and r must each be a multiple of 8 and, in
+ *     16-byte vectors, either a multiple of 32 vectors or a power of two up to 32 vectors; V must
+ *     be a multiple of 8.
+ */
+#ifndef DOMINO_H_
+#define DOMINO_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define DOMINO_API __attribute__((visibility("default")))
+#else
+#define DOMINO_API
+#endif
+
+#define DOMINO_ABI_VERSION 1
+#define DOMINO_MAX_L 64
+
+/* Storage type of the weights, embedding table, base logits and hidden states. */
+#define DOMINO_DTYPE_F32 0
+#define DOMINO_DTYPE_BF16 1
+
+/* Host return codes. */
+#define DOMINO_OK 0
+#define DOMINO_ERR_INVALID_ARGUMENT (-1) /* null required pointer, bad shape, misalignment      */
+#define DOMINO_ERR_UNSUPPORTED (-2)      /* valid but not handled (dims layout, device, grid)   */
+#define DOMINO_ERR_CUDA (-3)             /* a CUDA launch or query failed                       */
+#define DOMINO_ERR_WORKSPACE (-4)        /* workspace missing, misaligned (256 B) or too small  */
+
+/* Device status codes written to *status_dev. */
+#define DOMINO_STATUS_OK 0
+#define DOMINO_STATUS_DEVICE_TIMEOUT 1 /* a bounded device-wide wait gave up; outputs invalid */
+#define DOMINO_STATUS_BAD_TOKEN 2      /* a teacher-forcing token was outside [0, V)          */
+
+/* cudaStream_t, kept opaque so this header needs no CUDA include. */
+typedef void* domino_stream_t;
+
+/* Problem shape.  B rows, L positions per draft block, embedding / hidden width d, GRU hidden
+ * size Hs, correction rank r, vocabulary V, storage type dtype (DOMINO_DTYPE_*). */
+typedef struct {
+  int32_t B, L, d, Hs, r, V, dtype;
+} domino_shape_t;
+
+/* Head weights (device pointers, storage type = shape.dtype):
+ *   embed [V, d]      token embedding table, shared with the backbone
+ *   W_ih  [3Hs, d]    GRU input weights, gate blocks in the order (r | z | n)
+ *   W_hh  [3Hs, Hs]   GRU recurrent weights, same gate order
+ *   b_ih  [3Hs], b_hh [3Hs]
+ *   W1    [r, d+Hs]   columns 0..d-1 multiply H[i], columns d..d+Hs-1 multiply S_{i-1}
+ *   W2    [V, r]
+ * The GRU cell is the PyTorch nn.GRUCell form:
+ *   r = sig(W_ir x + b_ir + W_hr h + b_hr), z = sig(W_iz x + b_iz + W_hz h + b_hz),
+ *   n = tanh(W_in x + b_in + r * (W_hn h + b_hn)), h' = (1 - z) * n + z * h.            */
+typedef struct {
+  const void *embed, *W_ih, *W_hh, *b_ih, *b_hh, *W1, *W2;
+} domino_weights_t;
+
+/* Workspace bytes needed by domino_draft_greedy, domino_teacher_forced and domino_accept_len
+ * for `shape` (the largest of the three), or 0 if the shape is invalid.  The workspace must be
+ * device memory aligned to 256 bytes; its contents need no initialisation. */
+DOMINO_API size_t domino_workspace_bytes(const domino_shape_t* shape);
+
+/* Greedy drafting of one block per row (review page section 二: GRU causal encoder + low-rank
+ * logit-space correction; news.sig.ai article: the greedy decoding setting).
+ *
+ * For every row b and position i = 0..L-1, with S_{-1} = S0[b]:
+ *   z_i = L_base[b,i] + W2 . SiLU(W1 . [H[b,i] ; S_{i-1}])
+ *   t_i = argmax_v z_i[v]            (lowest index on ties; decided on fp32 z)
+ *   S_i = GRU(embed[t_i], S_{i-1})   for i < L-1 (the state after the last position is unused)
+ * Inputs:  base_logits [B, L, V], hidden [B, L, d] (storage type), S0 [B, Hs] fp32.
+ * Outputs: tokens_out [B, L] int32 (required);
+ *          logits_out [B, L, V] fp32 = z_i, or NULL to skip (the greedy path then never writes
+ *          logits: the argmax is fused into the W2 product);
+ *          states_out [B, L, Hs] fp32 = the state each position consumed (states_out[b,0] = S0),
+ *          or NULL.
+ * Returns DOMINO_OK or a negative DOMINO_ERR_* code (nothing launched). */
+DOMINO_API int domino_draft_greedy(const domino_shape_t* shape, const domino_weights_t* weights,
+                        const void* base_logits, const void* hidden, const float* S0,
+                        int32_t* tokens_out, float* logits_out, float* states_out,
+                        void* workspace, size_t workspace_bytes, int32_t* status_dev,
+                        domino_stream_t stream);
+
+/* Teacher-forced causal encoding (review page section 二, "Teacher Forcing": the GRU reads the
+ * given tokens instead of its own predictions).  Same equations as greedy drafting with
+ * t_i := tokens[b, i]; no argmax is taken.
+ * Inputs:  as domino_draft_greedy plus tokens [B, L] int32 (each in [0, V); an out-of-range
+ *          token sets DOMINO_STATUS_BAD_TOKEN and its row's later outputs are unspecified).
+ * Outputs: logits_out [B, L, V] fp32 (required); states_out [B, L, Hs] fp32 or NULL.
+ * Returns DOMINO_OK or a negative DOMINO_ERR_* code. */
+DOMINO_API int domino_teacher_forced(const domino_shape_t* shape, const domino_weights_t* weights,
+                          const void* base_logits, const void* hidden, const float* S0,
+                          const int32_t* tokens, float* logits_out, float* states_out,
+                          void* workspace, size_t workspace_bytes, int32_t* status_dev,
+                          domino_stream_t stream);
+
+/* Greedy accept length (the accept-length metric of the review page, section 四; the target
+ * verifies the whole block in one pass and keeps the longest agreeing prefix, sections 一 and
+ * the researchpapers.dev summary):
+ *   accept_out[b] = number of leading positions j (0 <= j < L) with
+ *                   draft_tokens[b, j] == argmax_v target_logits[b, j, v]  (lowest index on ties)
+ * No bonus token is counted.  draft_tokens [B, L] int32, target_logits [B, L, V] fp32,
+ * accept_out [B] int32.  Needs domino_accept_workspace_bytes(B, L) bytes of workspace (a
+ * workspace sized by domino_workspace_bytes for the same B and L also suffices).
+ * Returns DOMINO_OK or a negative DOMINO_ERR_* code. */
+DOMINO_API size_t domino_accept_workspace_bytes(int32_t B, int32_t L);
+DOMINO_API int domino_accept_len(int32_t B, int32_t L, int32_t V, const int32_t* draft_tokens,
+                      const float* target_logits, int32_t* accept_out, void* workspace,
+                      size_t workspace_bytes, int32_t* status_dev, domino_stream_t stream);
+
+/* Human-readable text for a DOMINO_ERR_* or DOMINO_STATUS_* code (static storage). */
+DOMINO_API const char* domino_status_string(int code);
+
+/* DOMINO_ABI_VERSION of the loaded library. */
+DOMINO_API int32_t domino_abi_version(void);
+
+/* Test hook: iteration limit of the library's bounded device-wide waits (0 restores the
+ * default, about one second).  A tiny limit makes waits give up early, which exercises the
+ * DOMINO_STATUS_DEVICE_TIMEOUT path without faulting or hanging the GPU.  Process-wide; takes
+ * effect at the next launch.  Returns DOMINO_OK. */
+DOMINO_API int domino_debug_set_spin_limit(uint64_t limit);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DOMINO_H_ */

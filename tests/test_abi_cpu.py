@@ -1,0 +1,110 @@
+"""The C-ABI library on a machine without a GPU: it loads, exports every symbol that
+include/domino.h declares, and its host-side logic (workspace sizing, argument checks, status
+strings) answers without touching the device."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+from draft_block_causal_b200 import domino
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    names = set()
+    for f in os.listdir(os.path.join(ROOT, "include")):
+        if f.endswith(".h"):
+            txt = open(os.path.join(ROOT, "include", f)).read()
+            names |= set(re.findall(r"DOMINO_API\s+[\w\s\*]+?\b(domino_\w+)\s*\(", txt))
+    return names
+
+
+@pytest.fixture(scope="module")
+def L():
+    from draft_block_causal_b200 import build
+    build.build()
+    return domino.lib()
+
+
+def test_every_declared_symbol_is_exported(L):
+    declared = _declared()
+    assert set(domino.EXPORTS) <= declared
+    out = subprocess.run(["nm", "-D", "--defined-only", domino.LIB_PATH], capture_output=True, text=True).stdout
+    exported = set(re.findall(r"\bT (domino_\w+)", out))
+    assert declared <= exported, declared - exported
+    for n in declared:
+        assert hasattr(L, n)
+
+
+def test_abi_version_and_status_strings(L):
+    assert domino.abi_version() == 1
+    for code in (0, -1, -2, -3, -4, 1, 2):
+        s = domino.status_string(code)
+        assert s and s != "unknown code"
+    assert domino.status_string(12345) == "unknown code"
+
+
+def _shape(**kw):
+    base = dict(B=1, L=16, d=4096, Hs=1024, r=256, V=151936, dtype=1)
+    base.update(kw)
+    return domino.Shape(*(base[k] for k in ("B", "L", "d", "Hs", "r", "V", "dtype")))
+
+
+def test_workspace_bytes_host_logic(L):
+    n1 = L.domino_workspace_bytes(ctypes.byref(_shape()))
+    n32 = L.domino_workspace_bytes(ctypes.byref(_shape(B=32)))
+    assert n1 > 0 and n32 > n1 and n1 % 256 == 0
+    # invalid shapes give 0
+    for bad in (dict(B=0), dict(L=0), dict(L=65), dict(d=12), dict(V=1001), dict(dtype=7), dict(r=2048)):
+        assert L.domino_workspace_bytes(ctypes.byref(_shape(**bad))) == 0, bad
+    # a d whose 16-byte vector count is neither a multiple of 32 nor a power of two up to 32
+    assert L.domino_workspace_bytes(ctypes.byref(_shape(d=8 * 40))) == 0
+    assert L.domino_workspace_bytes(ctypes.byref(_shape(d=2560))) > 0  # 320 vectors = 10 x 32
+    assert L.domino_accept_workspace_bytes(32, 16) > 0
+    assert L.domino_accept_workspace_bytes(0, 16) == 0
+
+
+def test_invalid_arguments_are_rejected_before_any_launch(L):
+    sh = _shape()
+    fake = ctypes.c_void_p(0x10000)  # 16-byte aligned, never dereferenced
+    w = domino.Weights(*([0x10000] * 7))
+    ws_bytes = L.domino_workspace_bytes(ctypes.byref(sh))
+    # null shape / weights
+    assert L.domino_draft_greedy(None, ctypes.byref(w), fake, fake, fake, fake, None, None, fake, ws_bytes, None,
+                                 None) == domino.ERR_INVALID_ARGUMENT
+    assert L.domino_draft_greedy(ctypes.byref(sh), None, fake, fake, fake, fake, None, None, fake, ws_bytes, None,
+                                 None) == domino.ERR_INVALID_ARGUMENT
+    # null required outputs / inputs
+    assert L.domino_draft_greedy(ctypes.byref(sh), ctypes.byref(w), fake, fake, fake, None, None, None, fake,
+                                 ws_bytes, None, None) == domino.ERR_INVALID_ARGUMENT
+    assert L.domino_teacher_forced(ctypes.byref(sh), ctypes.byref(w), fake, fake, fake, fake, None, None, fake,
+                                   ws_bytes, None, None) == domino.ERR_INVALID_ARGUMENT
+    # misaligned pointer
+    mis = ctypes.c_void_p(0x10004)
+    assert L.domino_draft_greedy(ctypes.byref(sh), ctypes.byref(w), mis, fake, fake, fake, None, None, fake,
+                                 ws_bytes, None, None) == domino.ERR_INVALID_ARGUMENT
+    w_mis = domino.Weights(*([0x10000] * 6 + [0x10008]))
+    assert L.domino_draft_greedy(ctypes.byref(sh), ctypes.byref(w_mis), fake, fake, fake, fake, None, None, fake,
+                                 ws_bytes, None, None) == domino.ERR_INVALID_ARGUMENT
+    # workspace missing, misaligned or too small
+    assert L.domino_draft_greedy(ctypes.byref(sh), ctypes.byref(w), fake, fake, fake, fake, None, None, None,
+                                 ws_bytes, None, None) == domino.ERR_WORKSPACE
+    assert L.domino_draft_greedy(ctypes.byref(sh), ctypes.byref(w), fake, fake, fake, fake, None, None,
+                                 ctypes.c_void_p(0x10010), ws_bytes, None, None) == domino.ERR_WORKSPACE
+    assert L.domino_draft_greedy(ctypes.byref(sh), ctypes.byref(w), fake, fake, fake, fake, None, None, fake,
+                                 ws_bytes - 256, None, None) == domino.ERR_WORKSPACE
+    # bad shapes
+    for bad in (dict(B=0), dict(L=100), dict(V=999), dict(dtype=3)):
+        assert L.domino_draft_greedy(ctypes.byref(_shape(**bad)), ctypes.byref(w), fake, fake, fake, fake, None,
+                                     None, fake, ws_bytes, None, None) == domino.ERR_INVALID_ARGUMENT
+    # accept length
+    i32 = ctypes.c_int32
+    assert L.domino_accept_len(i32(0), i32(16), i32(151936), fake, fake, fake, fake, 1 << 20, None,
+                               None) == domino.ERR_INVALID_ARGUMENT
+    assert L.domino_accept_len(i32(1), i32(16), i32(151936), None, fake, fake, fake, 1 << 20, None,
+                               None) == domino.ERR_INVALID_ARGUMENT
+    assert L.domino_accept_len(i32(1), i32(16), i32(151936), fake, fake, fake, fake, 16, None,
+                               None) == domino.ERR_WORKSPACE

@@ -1,0 +1,86 @@
+"""GPU boundary behaviour of the C ABI: device status codes, optional outputs, stream ordering,
+and the bounded-wait error path (driven from the host by a tiny spin limit -- nothing is made
+to fault or hang)."""
+import time
+
+import numpy as np
+import pytest
+import torch
+
+from draft_block_causal_b200 import domino, synth
+
+pytestmark = pytest.mark.gpu
+
+if torch.cuda.is_available():
+    from tests import gpu_common as G
+else:
+    G = None
+
+
+def _small(B=2, L=6, dtype=1, seed=200):
+    wl = dict(B=B, L=L, d=128, Hs=64, r=32, V=2000, dtype=dtype, weight_seed=seed, input_seed=seed + 1,
+              s0_std=0.2, peak=2.0, name="small")
+    return synth.make_workload(wl, with_tokens=True)
+
+
+def test_bad_teacher_forcing_token_sets_status():
+    data = _small()
+    w, lb, h, S0 = G.device_inputs(data)
+    y = torch.from_numpy(data["tokens"]).cuda()
+    y[1, 2] = 5000  # V = 2000
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    domino.teacher_forced(w, lb, h, S0, y, status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == domino.STATUS_BAD_TOKEN
+    # row 0 is unaffected and still matches the oracle
+    y0 = torch.from_numpy(data["tokens"]).cuda()
+    status.zero_()
+    lg, _ = domino.teacher_forced(w, lb, h, S0, y0, status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+
+
+def test_optional_outputs_and_no_status_pointer():
+    data = _small()
+    w, lb, h, S0 = G.device_inputs(data)
+    t1, l1, s1 = domino.draft_greedy(w, lb, h, S0)  # no logits, no states, status in workspace
+    t2, l2, s2 = domino.draft_greedy(w, lb, h, S0, logits_out=True, states_out=True)
+    torch.cuda.synchronize()
+    assert l1 is None and s1 is None and l2 is not None and s2 is not None
+    assert torch.equal(s2[:, 0], S0)  # the state consumed at position 0 is S0
+
+
+def test_calls_are_asynchronous_and_ordered_on_the_callers_stream():
+    data = _small(B=4, L=8)
+    w, lb, h, S0 = G.device_inputs(data)
+    ref_tok, _, _ = domino.draft_greedy(w, lb, h, S0)
+    torch.cuda.synchronize()
+    s = torch.cuda.Stream()
+    lb2 = torch.zeros_like(lb)
+    with torch.cuda.stream(s):
+        torch.cuda._sleep(200_000_000)  # ~0.1 s of GPU time on this stream
+        lb2.copy_(lb)                   # the inputs only become valid after the sleep
+        t0 = time.perf_counter()
+        tok, _, _ = domino.draft_greedy(w, lb2, h, S0, stream=s)
+        host_s = time.perf_counter() - t0
+    s.synchronize()
+    assert host_s < 0.05, f"call blocked the host for {host_s:.3f} s"
+    assert torch.equal(tok, ref_tok)
+
+
+def test_accept_len_workspace_from_head_sizing():
+    data = _small(B=3, L=5)
+    w, lb, h, S0 = G.device_inputs(data)
+    ws = domino.alloc_workspace(domino.workspace_bytes(w, 3, 5))
+    tok, _, _ = domino.draft_greedy(w, lb, h, S0, workspace=ws)
+    T = torch.randn(3, 5, 2000, device="cuda")
+    acc = domino.accept_len(tok, T, workspace=ws)
+    want = []
+    am = T.argmax(-1).cpu().numpy()
+    tk = tok.cpu().numpy()
+    for b in range(3):
+        k = 0
+        while k < 5 and tk[b, k] == am[b, k]:
+            k += 1
+        want.append(k)
+    assert acc.cpu().numpy().tolist() == want

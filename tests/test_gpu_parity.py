@@ -1,0 +1,106 @@
+"""GPU parity: the CUDA path, called through the C ABI, against the fp64 oracle on the same
+seeded inputs (procedure in gpu_common).  Small cases are checked on every output; the full
+Qwen3-shaped workloads on every output of sampled rows (rows are independent)."""
+import numpy as np
+import pytest
+import torch
+
+from draft_block_causal_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+if torch.cuda.is_available():
+    from tests import gpu_common as G
+else:  # collected but skipped on machines without a GPU
+    G = None
+
+
+def _custom(B, L, d, Hs, r, V, dtype, seed, s0_std=0.2, peak=2.0):
+    wl = dict(B=B, L=L, d=d, Hs=Hs, r=r, V=V, dtype=dtype, weight_seed=seed, input_seed=seed + 1,
+              s0_std=s0_std, peak=peak, name=f"custom-{seed}")
+    return wl
+
+
+SMALL = [
+    synth.workload("tiny-f32-b1"),
+    _custom(3, 5, 256, 128, 64, 4104, 1, 100),            # ragged vocab tail, several rows
+    _custom(5, 7, 64, 32, 16, 1000, 0, 110),              # fp32, odd B and L
+    _custom(2, 16, 512, 256, 256, 20008, 1, 120),         # bf16, full block, r = 256
+    _custom(1, 1, 64, 64, 32, 64, 1, 130),                # a single position: no GRU update
+    _custom(17, 3, 128, 64, 32, 3000, 1, 140),            # B not a multiple of the row tiles
+]
+
+
+@pytest.mark.parametrize("wl", SMALL, ids=lambda w: w["name"] + f"-B{w['B']}")
+def test_greedy_small(wl):
+    data = synth.make_workload(wl)
+    res = G.greedy_parity(data)
+    print(wl["name"], {k: v for k, v in res.items() if k != "tokens"})
+
+
+@pytest.mark.parametrize("wl", SMALL[1:4], ids=lambda w: w["name"] + f"-B{w['B']}")
+def test_teacher_forced_small(wl):
+    data = synth.make_workload(wl, with_tokens=True)
+    res = G.tf_parity(data)
+    print(wl["name"], res)
+
+
+def test_greedy_and_teacher_forced_4b_shapes():
+    wl = synth.workload("qwen3-4b-head-b1")
+    data = synth.make_workload(wl, with_tokens=True)
+    print("greedy", {k: v for k, v in G.greedy_parity(data).items() if k != "tokens"})
+    print("tf", G.tf_parity(data))
+
+
+def test_greedy_and_accept_8b_b1():
+    wl = synth.workload("qwen3-8b-head-b1")
+    data = synth.make_workload(wl, with_target=True)
+    res = G.greedy_parity(data)
+    acc = G.accept_parity(res["tokens"], data["target_logits"])
+    print({k: v for k, v in res.items() if k != "tokens"}, "accept", acc)
+
+
+def test_greedy_tf_accept_8b_b32_sampled_rows():
+    wl = synth.workload("qwen3-8b-head-b32")
+    data = synth.make_workload(wl, with_tokens=True, with_target=True)
+    rows = [0, 13, 31]
+    res = G.greedy_parity(data, rows=rows)
+    print("greedy", {k: v for k, v in res.items() if k != "tokens"})
+    print("tf", G.tf_parity(data, rows=rows))
+    acc = G.accept_parity(res["tokens"], data["target_logits"])
+    print("accept", acc)
+
+
+@pytest.mark.parametrize("B,peak", list(zip(synth.SWEEP_BATCHES, (1.0, 2.0, 4.0, 1.0, 2.0, 4.0))))
+def test_greedy_batch_sweep_sampled_rows(B, peak):
+    wl = synth.workload("qwen3-8b-head-sweep", B=B, peak=peak)
+    data = synth.make_workload(wl)
+    rows = sorted({0, B // 2, B - 1})
+    res = G.greedy_parity(data, rows=rows)
+    print(B, peak, {k: v for k, v in res.items() if k != "tokens"})
+
+
+def test_accept_length_constructed_prefixes():
+    rng = np.random.default_rng(7)
+    B, L, V = 40, 16, 151936
+    T = rng.standard_normal((B, L, V)).astype(np.float32)
+    am = np.argmax(T, axis=-1).astype(np.int32)
+    draft = am.copy()
+    for b in range(B):
+        k = b % (L + 1)
+        if k < L:
+            draft[b, k] = (draft[b, k] + 1) % V
+    # exact ties: the lowest index must win
+    T[3, 0, 10] = T[3, 0, 20] = 100.0
+    draft[3, 0] = 10
+    got = G.accept_parity(draft, T)
+    assert got[0] == 0 and got[16] == 16
+
+
+def test_accept_length_small_vocab_and_single_position():
+    rng = np.random.default_rng(8)
+    for B, L, V in [(1, 1, 8), (3, 4, 24), (65, 16, 1000)]:
+        T = rng.integers(-2, 3, (B, L, V)).astype(np.float32)  # ties everywhere
+        draft = np.argmax(T, axis=-1).astype(np.int32)
+        draft[::2, L // 2] = (draft[::2, L // 2] + 1) % V
+        G.accept_parity(draft, T)

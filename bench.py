@@ -1,0 +1,438 @@
+#!/usr/bin/env python
+"""Benchmark of the Domino-head hot path on B200: greedy drafting of 16-token blocks plus the
+greedy accept-length check, Qwen3-8B-shaped head (d=4096, GRU hidden 1024, rank 256,
+V=151936), bf16 storage, fp32 accumulation, synthetic seeded inputs.
+
+One step = one greedy draft of B rows (H-projection, 16 sequential positions of SiLU
+activation, W2 product with fused argmax and GRU update) followed by the accept-length check of
+the drafted tokens against synthetic target logits, with every input resident in HBM.  L2 is
+flushed (a 256 MiB write) before every timed step, as the target model's verification pass
+would between two drafts; each step is timed alone with CUDA events on the launching stream.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+With N > 1 (launched by torch.distributed.run) every rank drafts its own B rows on its own GPU
+with a full weight replica: rows are independent, so there is no collective on the data path
+("replicas only", weak scaling).  Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from draft_block_causal_b200 import synth  # noqa: E402
+
+METRIC = "Domino-head 16-token draft blocks/s and µs/block at B=1/32/128; % of roofline"
+UNIT = "blocks/s"
+HEADLINE = "qwen3-8b-head-b1"
+FLUSH_BYTES = 256 << 20
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            j = json.load(f)
+        return {"hbm_gbs": float(j["hbm_gbs"]), "bf16_tflops": float(j["bf16_tflops"]),
+                "bf16_tflops_sustained": float(j.get("bf16_tflops_sustained", j["bf16_tflops"])),
+                "source": "measured (MEASURED_PEAKS.json)"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def greedy_bytes(sh: dict) -> int:
+    """Algorithmic bytes of one greedy draft call with no reuse between positions: every
+    position streams W2 and the W1 state block, every GRU update streams W_ih and W_hh, W1's H
+    block is read once, plus per row the base logits, hidden states, embedding rows, S0 and the
+    token output."""
+    B, L, d, Hs, r, V = (sh[k] for k in ("B", "L", "d", "Hs", "r", "V"))
+    e = 2 if sh["dtype"] == synth.BF16 else 4
+    w2 = L * V * r * e
+    w1s = L * r * Hs * e
+    w1h = r * d * e
+    gru = (L - 1) * (3 * Hs * d + 3 * Hs * Hs + 6 * Hs) * e
+    per_row = L * V * e + L * d * e + (L - 1) * d * e + Hs * 4 + L * 4
+    return w2 + w1s + w1h + gru + B * per_row
+
+
+def greedy_flops(sh: dict) -> int:
+    B, L, d, Hs, r, V = (sh[k] for k in ("B", "L", "d", "Hs", "r", "V"))
+    return 2 * B * (L * r * V + (L - 1) * 3 * Hs * (d + Hs) + L * r * (d + Hs))
+
+
+def accept_bytes(B: int, L: int, V: int) -> int:
+    return B * L * V * 4 + B * L * 4 + B * 4
+
+
+class ClockSampler:
+    """SM clock and clock-event (throttle) reasons polled through NVML every ~2 ms while the timed
+    region runs (nvidia-smi's 100 ms floor is longer than the region itself)."""
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
+
+    def __init__(self, cuda_index: int):
+        self.samples = []
+        self.stop_flag = threading.Event()
+        self.thread = None
+        self.nvml = None
+        self.err = None
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            props = torch.cuda.get_device_properties(cuda_index)
+            try:
+                bus = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
+                self.handle = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+            except Exception:
+                self.handle = pynvml.nvmlDeviceGetHandleByIndex(cuda_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.handle, pynvml.NVML_CLOCK_SM)
+            self.nvml = pynvml
+        except Exception as e:  # no NVML: report it rather than guess
+            self.err = f"nvml unavailable: {type(e).__name__}"
+
+    def _poll(self):
+        nv = self.nvml
+        getr = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        while not self.stop_flag.is_set():
+            try:
+                self.samples.append((nv.nvmlDeviceGetClockInfo(self.handle, nv.NVML_CLOCK_SM), int(getr(self.handle))))
+            except Exception:
+                pass
+            time.sleep(0.002)
+
+    def start(self):
+        if self.nvml is None:
+            return
+        self.thread = threading.Thread(target=self._poll, daemon=True)
+        self.thread.start()
+
+    def stop(self) -> dict:
+        if self.nvml is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [self.err]}
+        self.stop_flag.set()
+        self.thread.join(timeout=2)
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["no samples"]}
+        mhz = [m for m, _ in self.samples]
+        reasons = sorted({n for _, r in self.samples for bit, n in self.REASONS.items() if r & bit})
+        return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": self.max_mhz, "reasons": reasons,
+                "samples": len(self.samples), "sm_mhz_min": min(mhz), "source": "nvml, 2 ms polling"}
+
+
+# ----------------------------------------------------------------------------------------------
+# our arm
+# ----------------------------------------------------------------------------------------------
+class Point:
+    """Device-resident inputs of one batch point plus the timed step."""
+
+    def __init__(self, wl: dict, device):
+        import torch
+        from draft_block_causal_b200 import domino
+        self.torch, self.domino = torch, domino
+        self.wl = wl
+        data = synth.make_workload(wl, with_target=True)
+        self.data = data
+        sh = self.sh = data["shape"]
+        dt = sh["dtype"]
+        self.w = domino.to_device_weights(data["weights"], dt, device)
+        self.lb = domino.to_device(data["base_logits"], dt, device)
+        self.h = domino.to_device(data["hidden"], dt, device)
+        self.S0 = torch.from_numpy(data["S0"]).to(device)
+        self.T = torch.from_numpy(data["target_logits"]).to(device)
+        B, L = sh["B"], sh["L"]
+        self.ws = domino.alloc_workspace(domino.workspace_bytes(self.w, B, L), device)
+        self.tok = torch.empty((B, L), dtype=torch.int32, device=device)
+        self.acc = torch.empty((B,), dtype=torch.int32, device=device)
+        self.status = torch.zeros(1, dtype=torch.int32, device=device)
+
+    def greedy(self, stream):
+        self.domino.draft_greedy(self.w, self.lb, self.h, self.S0, tokens_out=self.tok, workspace=self.ws,
+                                 status=self.status, stream=stream)
+
+    def accept(self, stream):
+        self.domino.accept_len(self.tok, self.T, accept_out=self.acc, workspace=self.ws, status=self.status,
+                               stream=stream)
+
+    def tf(self, stream, tokens, logits):
+        self.domino.teacher_forced(self.w, self.lb, self.h, self.S0, tokens, logits_out=logits, workspace=self.ws,
+                                   status=self.status, stream=stream)
+
+
+def time_steps(pt: Point, steps: int, warmup: int, flush, stream, dist=None):
+    """Warm up, then time `steps` steps, each on a freshly flushed L2.  Returns per-step device
+    times (ms) of the whole step and of its greedy-draft call."""
+    torch = pt.torch
+    for _ in range(warmup):
+        flush.zero_()
+        pt.greedy(stream)
+        pt.accept(stream)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+            torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    n0 = pt.domino.launch_count()
+    with torch.cuda.stream(stream):
+        for e0, e1, e2 in evs:
+            flush.zero_()
+            e0.record(stream)
+            pt.greedy(stream)
+            e1.record(stream)
+            pt.accept(stream)
+            e2.record(stream)
+    launches = pt.domino.launch_count() - n0
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    step = [e0.elapsed_time(e2) for e0, _, e2 in evs]
+    greedy = [e0.elapsed_time(e1) for e0, e1, _ in evs]
+    return step, greedy, launches
+
+
+def time_e2e(pt: Point, steps: int, warmup: int, flush, stream):
+    """Same step through the public API from pinned host buffers: each step copies its inputs
+    host->device and reads the tokens and accept lengths back, all inside the timed region."""
+    torch = pt.torch
+    host = {k: v.cpu().pin_memory() for k, v in (("lb", pt.lb), ("h", pt.h), ("S0", pt.S0), ("T", pt.T))}
+    out_tok = torch.empty(pt.tok.shape, dtype=torch.int32).pin_memory()
+    out_acc = torch.empty(pt.acc.shape, dtype=torch.int32).pin_memory()
+    dev = {k: torch.empty_like(getattr(pt, k)) for k in ("lb", "h", "S0", "T")}
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = out_tok.numel() * 4 + out_acc.numel() * 4
+
+    def one():
+        for k in ("lb", "h", "S0", "T"):
+            dev[k].copy_(host[k], non_blocking=True)
+        pt.domino.draft_greedy(pt.w, dev["lb"], dev["h"], dev["S0"], tokens_out=pt.tok, workspace=pt.ws,
+                               status=pt.status, stream=stream)
+        pt.domino.accept_len(pt.tok, dev["T"], accept_out=pt.acc, workspace=pt.ws, status=pt.status,
+                             stream=stream)
+        out_tok.copy_(pt.tok, non_blocking=True)
+        out_acc.copy_(pt.acc, non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        for _ in range(warmup):
+            flush.zero_()
+            one()
+        torch.cuda.synchronize()
+        times = []
+        for _ in range(steps):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            one()
+            e1.record(stream)
+            e1.synchronize()
+            times.append(e0.elapsed_time(e1))
+    return times, h2d, d2h
+
+
+def cpu_baseline(seconds: float) -> dict:
+    """The fp64 oracle, as it stands, on the host cores: greedy draft + accept length of the
+    headline workload (one row), repeated for about `seconds`."""
+    import oracle
+    wl = synth.workload(HEADLINE)
+    data = synth.make_workload(wl, with_target=True)
+    sh = data["shape"]
+    n, t0 = 0, time.perf_counter()
+    while True:
+        g = oracle.head(sh, data["weights"], data["base_logits"], data["hidden"], data["S0"], want_logits=False,
+                        want_states=False)
+        oracle.accept_len(g["tokens"], data["target_logits"])
+        n += 1
+        el = time.perf_counter() - t0
+        if el >= seconds:
+            break
+    return {"value": round(n * sh["B"] / el, 4), "unit": UNIT, "cores": oracle.max_threads(), "kind": "oracle",
+            "sample": f"{n} greedy draft + accept-length calls of the {HEADLINE} workload (B=1, 16 positions), "
+                      f"{el:.1f} s", "ms_per_block": round(1e3 * el / (n * sh["B"]), 3)}
+
+
+def run_ours(args):
+    import torch
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dist = None
+    if world > 1:
+        import torch.distributed as dist_mod
+        dist = dist_mod
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(local)
+    from draft_block_causal_b200 import domino
+    domino.lib()
+    device = torch.device("cuda", local)
+    stream = torch.cuda.Stream(device)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
+    peaks = _peaks()
+
+    # headline point: every rank drafts its own batch (replicas; rows differ per rank)
+    wl = synth.workload(HEADLINE, input_seed=synth.WORKLOADS[HEADLINE]["input_seed"] + 1000 * rank)
+    pt = Point(wl, device)
+    clk = ClockSampler(local)
+    clk.start()
+    step_ms, greedy_ms, launches = time_steps(pt, args.steps, args.warmup, flush, stream, dist)
+    clocks = clk.stop()
+    total_ms = sum(step_ms)
+    if dist is not None:
+        t = torch.tensor([total_ms], device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    torch.cuda.synchronize()
+    assert int(pt.status.item()) == 0, domino.status_string(int(pt.status.item()))
+    sh = pt.sh
+    B = sh["B"]
+    value = B * world * args.steps / (total_ms * 1e-3)
+
+    g_avg = statistics.mean(greedy_ms)
+    gbytes = greedy_bytes(sh)
+    achieved = gbytes / (g_avg * 1e-3) / 1e9
+    plan = domino.greedy_plan(domino.make_shape(pt.w, sh["B"], sh["L"]))
+    roof = {"bound": "hbm", "kernel": plan, "achieved": round(achieved, 1),
+            "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
+            "traffic": None, "algorithmic_bytes": gbytes, "launch_ms": round(g_avg, 4),
+            "peak_source": peaks["source"] + ", hbm_gbs (copy)"}
+
+    result = None
+    if rank == 0:
+        e2e_ms, h2d, d2h = time_e2e(pt, max(3, args.steps // 2), 2, flush, stream)
+        e2e_val = B / (statistics.mean(e2e_ms) * 1e-3)
+        points = {}
+        if not args.no_points:
+            del pt
+            torch.cuda.empty_cache()
+            for pb in (32, 128):
+                pwl = synth.workload("qwen3-8b-head-sweep", B=pb, peak=4.0)
+                p = Point(pwl, device)
+                s_ms, g_ms, _ = time_steps(p, max(3, args.steps // 2), args.warmup, flush, stream)
+                psh = p.sh
+                ga = statistics.mean(g_ms)
+                fl = greedy_flops(psh)
+                points[str(pb)] = {
+                    "blocks_per_s": round(pb * len(s_ms) / (sum(s_ms) * 1e-3), 1),
+                    "us_per_block": round(1e3 * statistics.mean(s_ms) / pb, 3),
+                    "ms_per_step": round(statistics.mean(s_ms), 4),
+                    "greedy_ms": round(ga, 4),
+                    "hbm_frac": round(greedy_bytes(psh) / (ga * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
+                    "tensor_frac": round(fl / (ga * 1e-3) / 1e12 / peaks["bf16_tflops"], 4),
+                    "greedy_tflops": round(fl / (ga * 1e-3) / 1e12, 2),
+                }
+                del p
+                torch.cuda.empty_cache()
+        cpu = None if args.no_cpu_baseline else cpu_baseline(args.cpu_seconds)
+        result = {
+            "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 4), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": f"{HEADLINE}: Qwen3-8B-shaped Domino head, greedy draft + accept length",
+                       "B_per_gpu": B, "block": sh["L"], "d": sh["d"], "gru_hidden": sh["Hs"], "rank": sh["r"],
+                       "vocab": sh["V"], "storage": "bf16 weights/inputs, fp32 accumulate",
+                       "parallelism": f"replicas x{world} (rows independent, no collective)",
+                       "l2": "flushed (256 MiB write) before every timed step"},
+            "us_per_block": round(1e3 * total_ms / args.steps / B, 3),
+            "roofline": roof,
+            "cpu_baseline": cpu,
+            "e2e": {"value": round(e2e_val, 2), "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "ms_per_step": round(statistics.mean(e2e_ms), 4)},
+            "gpu_launches": launches,
+            "clocks": clocks,
+            "points": points,
+        }
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    return result
+
+
+def profile_driver(n: int, batch: int = 1):
+    """A short, fixed sequence of greedy calls for an external profiler (ncu -k ... -s ... -c ...)."""
+    import torch
+    torch.cuda.set_device(0)
+    device = torch.device("cuda", 0)
+    wl = synth.workload(HEADLINE) if batch == 1 else synth.workload("qwen3-8b-head-sweep", B=batch)
+    pt = Point(wl, device)
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
+    for _ in range(n):
+        flush.zero_()
+        pt.greedy(stream)
+    torch.cuda.synchronize()
+    assert int(pt.status.item()) == 0
+
+
+def run_reference(args):
+    """The oracle as the reference arm, on the host cores (rank 0 only)."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return None
+    import oracle
+    wl = synth.workload(HEADLINE)
+    data = synth.make_workload(wl, with_target=True)
+    sh = data["shape"]
+
+    def step():
+        g = oracle.head(sh, data["weights"], data["base_logits"], data["hidden"], data["S0"], want_logits=False,
+                        want_states=False)
+        oracle.accept_len(g["tokens"], data["target_logits"])
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    el = time.perf_counter() - t0
+    value = sh["B"] * args.steps / el
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * el / args.steps, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"{HEADLINE}: Qwen3-8B-shaped Domino head, greedy draft + accept length",
+                   "B_per_gpu": sh["B"], "block": sh["L"], "d": sh["d"], "gru_hidden": sh["Hs"], "rank": sh["r"],
+                   "vocab": sh["V"], "storage": "bf16 weights/inputs widened to fp64"},
+        "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": oracle.max_threads(), "kind": "oracle",
+                         "sample": f"{args.steps} timed steps of one row (B=1), fp64 C oracle"},
+        "e2e": {"value": round(value, 4), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--no-points", action="store_true", help="skip the B=32 and B=128 points")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--profile", type=int, default=0, metavar="N",
+                    help="profiling driver: run N greedy calls of the headline workload (L2 flushed "
+                         "before each) and exit without timing or output")
+    args = ap.parse_args()
+    if args.profile:
+        profile_driver(args.profile)
+        return
+    if args.warmup < 3 and args.impl == "ours":
+        args.warmup = 3
+    res = run_reference(args) if args.impl == "reference" else run_ours(args)
+    if res is not None:
+        print(json.dumps(res), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -12,6 +12,7 @@ namespace domino {
 namespace {
 
 std::atomic<uint64_t> g_spin_limit{0};
+std::atomic<uint64_t> g_launches{0};
 
 inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
@@ -64,13 +65,14 @@ Workspace layout_workspace(const Shape& s, void* base) {
   const size_t BL = (size_t)s.B * s.L;
   w.status = reinterpret_cast<int32_t*>(take(sizeof(int32_t)));
   w.sync = reinterpret_cast<uint32_t*>(take(kSyncWords * sizeof(uint32_t)));
+  // sync, keys and a_acc are adjacent so that one memset clears all three
   w.keys = reinterpret_cast<uint64_t*>(take(BL * sizeof(uint64_t)));
+  w.a_acc = reinterpret_cast<float*>(take(BL * s.r * sizeof(float)));
   w.acc_keys = reinterpret_cast<uint64_t*>(take(BL * sizeof(uint64_t)));
   w.P = reinterpret_cast<float*>(take(BL * s.r * sizeof(float)));
   w.u = reinterpret_cast<float*>(take(BL * s.r * sizeof(float)));
   w.S = reinterpret_cast<float*>(take(2 * (size_t)s.B * s.Hs * sizeof(float)));
   w.states = reinterpret_cast<float*>(take(BL * s.Hs * sizeof(float)));
-  w.a_acc = reinterpret_cast<float*>(take(BL * s.r * sizeof(float)));
   w.bytes = off;
   return w;
 }
@@ -80,6 +82,11 @@ size_t accept_workspace_bytes(int B, int L) {
   Shape s{B, L, 8, 8, 8, 8, DOMINO_DTYPE_F32};
   Workspace w = layout_workspace(s, nullptr);
   return w.bytes;
+}
+
+cudaError_t note_launch(cudaError_t e) {
+  if (e == cudaSuccess) g_launches.fetch_add(1, std::memory_order_relaxed);
+  return e;
 }
 
 uint64_t spin_limit() {
@@ -94,6 +101,15 @@ using namespace domino;
 extern "C" {
 
 int32_t domino_abi_version(void) { return DOMINO_ABI_VERSION; }
+
+uint64_t domino_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+const char* domino_greedy_plan(const domino_shape_t* shape) {
+  if (check_shape(shape) != DOMINO_OK) return "invalid shape";
+  const Shape s = to_shape(shape);
+  if (use_persistent_greedy(s)) return persistent_plan(s);
+  return "per-phase kernels: k_hproj, then per position k_u + k_w2 (fused argmax) + k_gru, then k_tokens";
+}
 
 int domino_debug_set_spin_limit(uint64_t limit) {
   g_spin_limit.store(limit, std::memory_order_relaxed);

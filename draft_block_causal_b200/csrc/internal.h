@@ -27,6 +27,9 @@ struct Workspace {
 constexpr int kSyncWords = 64;
 
 Workspace layout_workspace(const Shape& s, void* base);
+
+// Counts one enqueued kernel when `e` reports success; returns `e`.
+cudaError_t note_launch(cudaError_t e);
 size_t accept_workspace_bytes(int B, int L);
 
 // ---- step kernels (one launch per phase; any storage type, any batch) ----

@@ -1,13 +1,453 @@
-// persistent.cu -- placeholder until the fused greedy kernel lands.
+// persistent.cu -- fused greedy drafting of a whole block in one cooperative launch (small batch,
+// bf16 storage, rank 256).
+//
+// Computes, for every row b and position i (Domino review page, section 二, head equation and
+// the GRU causal encoder beside it; greedy setting of the news.sig.ai article):
+//   z_i = L_base[b,i] + W2 . SiLU(W1 . [H[b,i] ; S_{i-1}]),  t_i = argmax z_i,
+//   S_i = GRUCell(embed[t_i], S_{i-1})
+// with one CTA per SM for the whole block.  The 16 positions are sequential through the argmax,
+// so the kernel walks them in a loop separated by bounded grid-wide barriers:
+//
+//   prologue  a_acc[i] += W1[:, :d] . H[b,i] for every i (rank rows split over CTAs)
+//             a_acc[0] += W1[:, d:] . S0   (each CTA adds the part of its own GRU units)
+//   -- barrier --
+//   step i    u = SiLU(a_acc[i]) in every CTA (r floats per row)
+//             gh = W_hh . S_{i-1} for the CTA's GRU units (independent of the argmax)
+//             z = L_base + W2 . u over the CTA's contiguous vocabulary slice; per-CTA argmax
+//             folded into one u64 key per row with atomicMax (value, then lowest index)
+//   -- barrier --
+//             t_i from the key; gi = W_ih . embed[t_i] for the CTA's units; GRU cell -> S_i
+//             a_acc[i+1] += W1[:, d:] (own columns) . S_i   (float4 atomics)
+//   -- barrier --
+//
+// Weights stream from L2/HBM with 16-byte loads straight into registers.  The W2 rows of a warp
+// are reduced eight at a time with a transpose-reduction (9 shuffles per 8 rows).  Every wait
+// is bounded: a barrier that does not fill within the spin limit writes DEVICE_TIMEOUT to the
+// status word and every CTA returns (no copy or TMEM is ever held across a wait).
+#include "common.cuh"
 #include "persistent.h"
+
+#include <algorithm>
 
 namespace domino {
 
-bool use_persistent_greedy(const Shape&) { return false; }
+namespace {
 
-cudaError_t launch_persistent_greedy(const Shape&, const domino_weights_t&, const void*, const void*, const float*,
-                                     int32_t*, float*, float*, const Workspace&, int32_t*, uint64_t, cudaStream_t) {
-  return cudaErrorNotSupported;
+constexpr int kPThreads = 512;
+constexpr int kPWarps = kPThreads / 32;
+constexpr int kR = 256;       // rank handled by this kernel (one 16-byte vector per lane per row)
+constexpr int kSeg = 256;     // K-segment of a GRU dot product: 32 lanes x 8 bf16
+constexpr int kMaxB = 4;
+
+struct PArgs {
+  const bf16 *embed, *W_ih, *W_hh, *b_ih, *b_hh, *W1, *W2;
+  const bf16 *Lb, *H;
+  const float* S0;
+  int32_t* tokens;
+  float* logits;
+  float* states;
+  uint64_t* keys;   // [L][B]
+  float* a_acc;     // [L][B][r]
+  float* Sbuf;      // [2][B][Hs]
+  unsigned* bar;    // grid barrier counter (zeroed before launch)
+  int32_t* status;
+  int B, L, d, Hs, V, maxu;
+  unsigned long long spin_limit;
+};
+
+__device__ __forceinline__ unsigned ld_acquire(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ int ld_relaxed(const int32_t* p) {
+  int v;
+  asm volatile("ld.relaxed.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Grid-wide barrier over a monotonic counter: the k-th barrier waits for k * gridDim.x arrivals.
+// Returns false (in every thread of the CTA) when the wait gave up or another CTA already did.
+__device__ bool grid_sync(const PArgs& p, unsigned& epoch, int* flag_s) {
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    ++epoch;
+    __threadfence();
+    atomicAdd(p.bar, 1u);
+    const unsigned target = epoch * gridDim.x;
+    bool ok = false;
+    for (unsigned long long it = 0; it < p.spin_limit; ++it) {
+      if (ld_acquire(p.bar) >= target) { ok = true; break; }
+      if ((it & 31) == 31 && ld_relaxed(p.status) == DOMINO_STATUS_DEVICE_TIMEOUT) break;
+    }
+    if (!ok) set_status(p.status, DOMINO_STATUS_DEVICE_TIMEOUT);
+    __threadfence();
+    *flag_s = ok ? 1 : 0;
+  }
+  __syncthreads();
+  const bool ok = *flag_s != 0;
+  __syncthreads();  // nobody rewrites the flag before everyone has read it
+  return ok;
+}
+
+// Sum over the 32 lanes of ROWS per-lane values at once.  On return, lane l holds the full sum of
+// value index (l >> log2(32 / ROWS)).
+template <int ROWS>
+__device__ __forceinline__ float transpose_reduce(float (&v)[ROWS], int lane) {
+#pragma unroll
+  for (int n = ROWS, m = 16; n > 1; n >>= 1, m >>= 1) {
+    const bool up = (lane & m) != 0;
+#pragma unroll
+    for (int k = 0; k < n / 2; ++k) {
+      const float send = up ? v[k] : v[k + n / 2];
+      const float keep = up ? v[k + n / 2] : v[k];
+      v[k] = keep + __shfl_xor_sync(0xffffffffu, send, m);
+    }
+  }
+  float s = v[0];
+#pragma unroll
+  for (int m = (32 / ROWS) >> 1; m > 0; m >>= 1) s += __shfl_xor_sync(0xffffffffu, s, m);
+  return s;
+}
+
+__device__ __forceinline__ void fma8(const uint4& q, const float (&x)[8], float& acc) {
+  float w[8];
+  widen(q, w);
+#pragma unroll
+  for (int e = 0; e < 8; ++e) acc = fmaf(w[e], x[e], acc);
+}
+
+// CTA-wide dot products of `nrows` rows of a bf16 matrix (row length K, a multiple of kSeg) with
+// up to kMaxB input vectors held in shared memory (fp32 [BMAX][K] or bf16 [BMAX][K]), adding the
+// results into acc_s[b * acc_stride + row].  Work items are (row, K-segment) pairs, four per warp
+// iteration, reduced with one transpose-reduction.  row_ptr(row) gives the row's address.
+template <int BMAX, typename In, typename RowPtr>
+__device__ void cta_rows_dot(RowPtr row_ptr, int nrows, int K, const In* in_s, int B, float* acc_s, int acc_stride,
+                             int warp, int lane) {
+  const int nseg = K / kSeg;
+  const int nitems = nrows * nseg;
+  for (int base = warp * 4; base < nitems; base += kPWarps * 4) {
+    uint4 q[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int it = base + k;
+      q[k] = make_uint4(0u, 0u, 0u, 0u);
+      if (it < nitems) q[k] = ldg16(row_ptr(it / nseg) + (it % nseg) * kSeg + lane * 8);
+    }
+    float acc[BMAX][4];
+#pragma unroll
+    for (int b = 0; b < BMAX; ++b)
+#pragma unroll
+      for (int k = 0; k < 4; ++k) acc[b][k] = 0.f;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int it = base + k;
+      if (it < nitems) {
+        const int col = (it % nseg) * kSeg + lane * 8;
+#pragma unroll
+        for (int b = 0; b < BMAX; ++b) {
+          if (b < B) {
+            float x[8];
+            if constexpr (sizeof(In) == 4) {
+              const float4* xp = reinterpret_cast<const float4*>(in_s + (size_t)b * K + col);
+              float4 x0 = xp[0], x1 = xp[1];
+              x[0] = x0.x; x[1] = x0.y; x[2] = x0.z; x[3] = x0.w; x[4] = x1.x; x[5] = x1.y; x[6] = x1.z; x[7] = x1.w;
+            } else {
+              widen(*reinterpret_cast<const uint4*>(in_s + (size_t)b * K + col), x);
+            }
+            fma8(q[k], x, acc[b][k]);
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int b = 0; b < BMAX; ++b) {
+      if (b < B) {
+        const float s = transpose_reduce<4>(acc[b], lane);
+        const int it = base + (lane >> 3);
+        if ((lane & 7) == 0 && it < nitems) atomicAdd(acc_s + b * acc_stride + it / nseg, s);
+      }
+    }
+  }
+}
+
+template <int BMAX, int ROWS>
+__global__ void __launch_bounds__(kPThreads, 1) k_greedy_persistent(PArgs p) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  const int G = gridDim.x, c = blockIdx.x, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int B = p.B, L = p.L, d = p.d, Hs = p.Hs, V = p.V, maxu = p.maxu;
+  const int v0 = (int)((long long)V * c / G), v1 = (int)((long long)V * (c + 1) / G);
+  const int j0 = (int)((long long)Hs * c / G), j1 = (int)((long long)Hs * (c + 1) / G);
+  const int nu = j1 - j0;
+  const int ldw1 = d + Hs;
+
+  // shared memory carve-up (16-byte aligned pieces)
+  float* u_s = reinterpret_cast<float*>(smem);                       // [BMAX][kR]
+  float* S_s = u_s + BMAX * kR;                                      // [BMAX][Hs]  S_{i-1}
+  bf16* x_s = reinterpret_cast<bf16*>(S_s + (size_t)BMAX * Hs);      // [BMAX][d]   embed[t_i]
+  float* w1s_s = reinterpret_cast<float*>(x_s + (size_t)BMAX * d);   // [maxu][kR]  W1[:, d + j0 + jj]
+  float* gh_s = w1s_s + (size_t)maxu * kR;                           // [BMAX][3*maxu]
+  float* gi_s = gh_s + BMAX * 3 * maxu;                              // [BMAX][3*maxu]
+  float* sn_s = gi_s + BMAX * 3 * maxu;                              // [BMAX][maxu]  S_i (own units)
+  uint64_t* best_s = reinterpret_cast<uint64_t*>(sn_s + ((BMAX * maxu + 3) & ~3));  // [kPWarps][BMAX]
+  int* flag_s = reinterpret_cast<int*>(best_s + kPWarps * BMAX);
+  unsigned epoch = 0;
+
+  // ---------------- prologue ----------------
+  for (int k = tid; k < maxu * kR; k += kPThreads) {
+    const int jj = k / kR, kk = k % kR;
+    w1s_s[k] = (jj < nu) ? __bfloat162float(p.W1[(size_t)kk * ldw1 + d + j0 + jj]) : 0.f;
+  }
+  for (int k = tid; k < BMAX * 6 * maxu; k += kPThreads) gh_s[k] = 0.f;  // gh_s and gi_s
+  // a_acc[i][b][k] += W1[k, :d] . H[b, i]   for the rank rows k = c, c + G, ...
+  {
+    const int nk = (kR - c + G - 1) / G;  // rank rows owned by this CTA
+    const int npos = B * L;
+    const int nseg = d / kSeg;
+    for (int item = warp; item < nk * npos; item += kPWarps) {
+      const int k = c + (item / npos) * G, n = item % npos;
+      const bf16* wr = p.W1 + (size_t)k * ldw1;
+      const bf16* hr = p.H + (size_t)n * d;
+      float acc = 0.f;
+      for (int s = 0; s < nseg; ++s) {
+        float x[8];
+        widen(ldg16(hr + s * kSeg + lane * 8), x);
+        fma8(ldg16(wr + s * kSeg + lane * 8), x, acc);
+      }
+      acc = warp_sum(acc);
+      const int b = n / L, i = n % L;
+      if (lane == 0) atomicAdd(p.a_acc + ((size_t)i * B + b) * kR + k, acc);
+    }
+  }
+  __syncthreads();
+  // a_acc[0][b] += W1[:, d + own units] . S0[b, own units];  states_out[b, 0] = S0[b]
+  for (int t = tid; t < BMAX * (kR / 4); t += kPThreads) {
+    const int b = t / (kR / 4), k4 = (t % (kR / 4)) * 4;
+    if (b < B && nu > 0) {
+      float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int jj = 0; jj < nu; ++jj) {
+        const float h = p.S0[(size_t)b * Hs + j0 + jj];
+        const float* w = w1s_s + jj * kR + k4;
+        s.x = fmaf(w[0], h, s.x); s.y = fmaf(w[1], h, s.y); s.z = fmaf(w[2], h, s.z); s.w = fmaf(w[3], h, s.w);
+      }
+      atomicAdd(reinterpret_cast<float4*>(p.a_acc + (size_t)b * kR + k4), s);
+    }
+  }
+  if (p.states)
+    for (int t = tid; t < B * nu; t += kPThreads) {
+      const int b = t / nu, jj = t % nu;
+      p.states[(size_t)b * L * Hs + j0 + jj] = p.S0[(size_t)b * Hs + j0 + jj];
+    }
+  if (!grid_sync(p, epoch, flag_s)) return;
+
+  // ---------------- the block, one position at a time ----------------
+  for (int i = 0; i < L; ++i) {
+    // u = SiLU(a_acc[i]) ; S_{i-1} into shared memory
+    for (int t = tid; t < BMAX * kR; t += kPThreads) {
+      const int b = t / kR;
+      u_s[t] = (b < B) ? siluf_(__ldcg(p.a_acc + ((size_t)i * B + b) * kR + (t % kR))) : 0.f;
+    }
+    if (i < L - 1) {
+      const float* Sprev = (i == 0) ? p.S0 : p.Sbuf + (size_t)((i - 1) & 1) * B * Hs;
+      for (int t = tid; t < B * Hs; t += kPThreads) S_s[t] = __ldcg(Sprev + t);
+    }
+    __syncthreads();
+
+    // gh = W_hh . S_{i-1} for the own units (rows g*Hs + j0 + jj), independent of the argmax
+    if (i < L - 1 && nu > 0) {
+      auto rowp = [&](int row) { return p.W_hh + ((size_t)(row / nu) * Hs + j0 + row % nu) * Hs; };
+      cta_rows_dot<BMAX, float>(rowp, 3 * nu, Hs, S_s, B, gh_s, 3 * maxu, warp, lane);
+    }
+
+    // z = L_base + W2 . u over the vocabulary slice [v0, v1), fused argmax
+    {
+      float uv[BMAX][8];
+#pragma unroll
+      for (int b = 0; b < BMAX; ++b)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) uv[b][e] = u_s[b * kR + lane * 8 + e];
+      uint64_t best[BMAX];
+#pragma unroll
+      for (int b = 0; b < BMAX; ++b) best[b] = 0ull;
+      const int nrows = v1 - v0;
+      const int nch = (nrows + ROWS - 1) / ROWS;
+      const size_t lrow = (size_t)i * V;  // + b * L * V
+      for (int ch = warp; ch < nch; ch += kPWarps) {
+        const int vb = v0 + ch * ROWS;
+        uint4 q[ROWS];
+#pragma unroll
+        for (int k = 0; k < ROWS; ++k)
+          q[k] = (vb + k < v1) ? ldg16(p.W2 + (size_t)(vb + k) * kR + lane * 8) : make_uint4(0u, 0u, 0u, 0u);
+        float acc[BMAX][ROWS];
+#pragma unroll
+        for (int k = 0; k < ROWS; ++k) {
+          float w[8];
+          widen(q[k], w);
+#pragma unroll
+          for (int b = 0; b < BMAX; ++b) {
+            float a = 0.f;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) a = fmaf(w[e], uv[b][e], a);
+            acc[b][k] = a;
+          }
+        }
+        const int v = vb + (lane >> (5 - (ROWS == 8 ? 3 : 2)));
+#pragma unroll
+        for (int b = 0; b < BMAX; ++b) {
+          if (b < B) {
+            const float s = transpose_reduce<ROWS>(acc[b], lane);
+            if ((lane & (32 / ROWS - 1)) == 0 && v < v1) {
+              const size_t at = lrow + (size_t)b * L * V + v;
+              const float z = __bfloat162float(p.Lb[at]) + s;
+              if (p.logits) p.logits[at] = z;
+              best[b] = umax64(best[b], argmax_key(z, v));
+            }
+          }
+        }
+      }
+#pragma unroll
+      for (int b = 0; b < BMAX; ++b) {
+        uint64_t m = best[b];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = umax64(m, __shfl_xor_sync(0xffffffffu, m, o));
+        if (lane == 0) best_s[warp * BMAX + b] = m;
+      }
+      __syncthreads();
+      if (tid < B) {
+        uint64_t m = 0ull;
+        for (int w = 0; w < kPWarps; ++w) m = umax64(m, best_s[w * BMAX + tid]);
+        atomicMax(reinterpret_cast<unsigned long long*>(p.keys + (size_t)i * B + tid), (unsigned long long)m);
+      }
+    }
+    if (!grid_sync(p, epoch, flag_s)) return;
+    if (i == L - 1) break;
+
+    // t_i, x = embed[t_i], gi = W_ih . x for the own units, GRU cell -> S_i
+    for (int t = tid; t < B * (d / 8); t += kPThreads) {
+      const int b = t / (d / 8), q = t % (d / 8);
+      // the key of a finished argmax always names a row in [0, V); the clamp only guards the load
+      const int tok = min(max(key_index(__ldcg(p.keys + (size_t)i * B + b)), 0), V - 1);
+      reinterpret_cast<uint4*>(x_s + (size_t)b * d)[q] = ldg16(p.embed + (size_t)tok * d + q * 8);
+    }
+    __syncthreads();
+    if (nu > 0) {
+      auto rowp = [&](int row) { return p.W_ih + ((size_t)(row / nu) * Hs + j0 + row % nu) * d; };
+      cta_rows_dot<BMAX, bf16>(rowp, 3 * nu, d, x_s, B, gi_s, 3 * maxu, warp, lane);
+    }
+    __syncthreads();
+    float* Snext = p.Sbuf + (size_t)(i & 1) * B * Hs;
+    for (int t = tid; t < B * nu; t += kPThreads) {
+      const int b = t / nu, jj = t % nu, j = j0 + jj;
+      float gi[3], gh[3];
+#pragma unroll
+      for (int g = 0; g < 3; ++g) {
+        gi[g] = gi_s[b * 3 * maxu + g * nu + jj] + __bfloat162float(p.b_ih[(size_t)g * Hs + j]);
+        gh[g] = gh_s[b * 3 * maxu + g * nu + jj] + __bfloat162float(p.b_hh[(size_t)g * Hs + j]);
+        gi_s[b * 3 * maxu + g * nu + jj] = 0.f;
+        gh_s[b * 3 * maxu + g * nu + jj] = 0.f;
+      }
+      const float rg = sigmoidf_(gi[0] + gh[0]);
+      const float zg = sigmoidf_(gi[1] + gh[1]);
+      const float ng = tanhf(gi[2] + rg * gh[2]);
+      const float hn = (1.f - zg) * ng + zg * S_s[b * Hs + j];
+      sn_s[b * maxu + jj] = hn;
+      Snext[(size_t)b * Hs + j] = hn;
+      if (p.states) p.states[((size_t)b * L + i + 1) * Hs + j] = hn;
+    }
+    __syncthreads();
+    // a_acc[i+1][b] += W1[:, d + own units] . S_i[b, own units]
+    for (int t = tid; t < BMAX * (kR / 4); t += kPThreads) {
+      const int b = t / (kR / 4), k4 = (t % (kR / 4)) * 4;
+      if (b < B && nu > 0) {
+        float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int jj = 0; jj < nu; ++jj) {
+          const float h = sn_s[b * maxu + jj];
+          const float* w = w1s_s + jj * kR + k4;
+          s.x = fmaf(w[0], h, s.x); s.y = fmaf(w[1], h, s.y); s.z = fmaf(w[2], h, s.z); s.w = fmaf(w[3], h, s.w);
+        }
+        atomicAdd(reinterpret_cast<float4*>(p.a_acc + ((size_t)(i + 1) * B + b) * kR + k4), s);
+      }
+    }
+    if (!grid_sync(p, epoch, flag_s)) return;
+  }
+  // tokens: every key is final after the last barrier
+  if (c == 0)
+    for (int t = tid; t < B * L; t += kPThreads) {
+      const int b = t / L, i = t % L;
+      p.tokens[t] = key_index(__ldcg(p.keys + (size_t)i * B + b));
+    }
+}
+
+size_t smem_bytes(int bmax, int d, int Hs, int maxu) {
+  size_t f = (size_t)bmax * kR + (size_t)bmax * Hs;
+  size_t bytes = f * 4 + (size_t)bmax * d * 2;
+  bytes += ((size_t)maxu * kR + 6 * (size_t)bmax * maxu + (((size_t)bmax * maxu + 3) & ~(size_t)3)) * 4;
+  bytes += (size_t)kPWarps * bmax * 8 + 16;
+  return bytes;
+}
+
+int g_num_sms = 0;
+
+int num_sms() {
+  if (g_num_sms == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&g_num_sms, cudaDevAttrMultiProcessorCount, dev);
+  }
+  return g_num_sms;
+}
+
+template <int BMAX, int ROWS>
+cudaError_t launch_t(const PArgs& a, int G, size_t smem, cudaStream_t st) {
+  auto kern = k_greedy_persistent<BMAX, ROWS>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  int per_sm = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kPThreads, smem);
+  if (e != cudaSuccess) return e;
+  if (per_sm < 1) return cudaErrorCooperativeLaunchTooLarge;
+  PArgs args = a;
+  void* params[] = {&args};
+  return cudaLaunchCooperativeKernel((const void*)kern, dim3(G), dim3(kPThreads), params, smem, st);
+}
+
+}  // namespace
+
+bool use_persistent_greedy(const Shape& s) {
+  return s.dtype == DOMINO_DTYPE_BF16 && s.r == kR && s.B <= kMaxB && s.d % kSeg == 0 && s.Hs % kSeg == 0 &&
+         s.d <= 16384 && s.Hs <= 8192;
+}
+
+const char* persistent_plan(const Shape& s) {
+  (void)s;
+  return "k_greedy_persistent: one cooperative launch, one CTA per SM, 16 positions with bounded grid barriers";
+}
+
+cudaError_t launch_persistent_greedy(const Shape& s, const domino_weights_t& w, const void* base_logits,
+                                     const void* hidden, const float* S0, int32_t* tokens_out, float* logits_out,
+                                     float* states_out, const Workspace& ws, int32_t* status, uint64_t spin,
+                                     cudaStream_t st) {
+  const int G = num_sms();
+  if (G < 1) return cudaErrorNoDevice;
+  PArgs a{};
+  a.embed = (const bf16*)w.embed; a.W_ih = (const bf16*)w.W_ih; a.W_hh = (const bf16*)w.W_hh;
+  a.b_ih = (const bf16*)w.b_ih; a.b_hh = (const bf16*)w.b_hh; a.W1 = (const bf16*)w.W1; a.W2 = (const bf16*)w.W2;
+  a.Lb = (const bf16*)base_logits; a.H = (const bf16*)hidden; a.S0 = S0;
+  a.tokens = tokens_out; a.logits = logits_out; a.states = states_out;
+  a.keys = ws.keys; a.a_acc = ws.a_acc; a.Sbuf = ws.S; a.bar = ws.sync; a.status = status;
+  a.B = s.B; a.L = s.L; a.d = s.d; a.Hs = s.Hs; a.V = s.V;
+  a.maxu = (s.Hs + G - 1) / G;
+  a.spin_limit = spin;
+  // barrier counter, argmax keys and accumulators are contiguous in the workspace: one memset
+  const size_t zero_bytes = (size_t)((char*)(ws.a_acc + (size_t)s.L * s.B * s.r) - (char*)ws.sync);
+  cudaError_t e = cudaMemsetAsync(ws.sync, 0, zero_bytes, st);
+  if (e != cudaSuccess) return e;
+  const int bmax = s.B <= 1 ? 1 : (s.B <= 2 ? 2 : 4);
+  const size_t smem = smem_bytes(bmax, s.d, s.Hs, a.maxu);
+  if (bmax == 1) e = launch_t<1, 8>(a, G, smem, st);
+  else if (bmax == 2) e = launch_t<2, 8>(a, G, smem, st);
+  else e = launch_t<4, 4>(a, G, smem, st);
+  return note_launch(e);
 }
 
 }  // namespace domino

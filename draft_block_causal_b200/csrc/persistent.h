@@ -12,6 +12,7 @@ uint64_t spin_limit();
 
 // True when the fused persistent kernel handles this shape (else the step kernels do).
 bool use_persistent_greedy(const Shape& s);
+const char* persistent_plan(const Shape& s);
 
 cudaError_t launch_persistent_greedy(const Shape& s, const domino_weights_t& w, const void* base_logits,
                                      const void* hidden, const float* S0, int32_t* tokens_out, float* logits_out,

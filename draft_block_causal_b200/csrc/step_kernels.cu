@@ -98,42 +98,56 @@ __global__ void __launch_bounds__(kThreads) k_u(const T* __restrict__ W1, int ld
   }
 }
 
-// z[m][v] = Lb[row(m)][v] + sum_k W2[v][k] u[m][k],  row(m) = m*l_mul + l_add.
-// keys != null: keys[m] = max(keys[m], argmax_key(z, v)).  logits != null: logits[row(m)][v] = z.
-template <typename T>
+// z[m][v] = Lb[row(m)][v] + sum_k W2[v][k] u[m][k],  row(m) = m*l_mul + l_add, for a tile of MT
+// rows m.  keys != null: keys[m] = max(keys[m], argmax_key(z, v)).  logits != null:
+// logits[row(m)][v] = z.  u sits in shared memory as [m][vector][E + pad] so that the 16-byte
+// reads of 32 lanes (one vector each) hit distinct bank groups.
+template <typename T> struct UPad { static constexpr int v = 0; };
+template <> struct UPad<bf16> { static constexpr int v = 4; };
+
+template <typename T, int MT>
 __global__ void __launch_bounds__(kThreads) k_w2(const T* __restrict__ W2, int r, int V, const float* __restrict__ u,
                                                  int M, const T* __restrict__ Lb, int l_mul, int l_add,
                                                  uint64_t* __restrict__ keys, float* __restrict__ logits) {
   constexpr int E = Vec<T>::N;
-  extern __shared__ float u_s[];  // [kTileM][r]
-  __shared__ uint64_t best_s[kWarps][kTileM];
+  constexpr int VS = E + UPad<T>::v;
+  extern __shared__ __align__(16) float u_s[];  // [MT][r/E][VS]
+  __shared__ uint64_t best_s[kWarps][MT];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int m0 = blockIdx.y * kTileM;
-  const int mt = min(kTileM, M - m0);
-  for (int i = threadIdx.x; i < kTileM * r; i += kThreads) {
-    int m = i / r;
-    u_s[i] = (m < mt) ? u[(size_t)(m0 + m) * r + (i % r)] : 0.f;
+  const int nqv = r / E;
+  const int m0 = blockIdx.y * MT;
+  const int mt = min(MT, M - m0);
+  for (int i = threadIdx.x; i < MT * r; i += kThreads) {
+    const int m = i / r, k = i % r;
+    u_s[(m * nqv + k / E) * VS + k % E] = (m < mt) ? u[(size_t)(m0 + m) * r + k] : 0.f;
   }
   __syncthreads();
-  uint64_t best[kTileM];
+  uint64_t best[MT];
 #pragma unroll
-  for (int m = 0; m < kTileM; ++m) best[m] = 0ull;
+  for (int m = 0; m < MT; ++m) best[m] = 0ull;
   for (int v = blockIdx.x * kWarps + warp; v < V; v += gridDim.x * kWarps) {
-    float acc[kTileM];
+    float acc[MT];
 #pragma unroll
-    for (int m = 0; m < kTileM; ++m) acc[m] = 0.f;
+    for (int m = 0; m < MT; ++m) acc[m] = 0.f;
     const T* wrow = W2 + (size_t)v * r;
-    for (int q = lane; q < r / E; q += 32) {
+    for (int q = lane; q < nqv; q += 32) {
       float w[E];
       widen(ldg16(wrow + q * E), w);
 #pragma unroll
-      for (int m = 0; m < kTileM; ++m) {
+      for (int m = 0; m < MT; ++m) {
+        const float4* up = reinterpret_cast<const float4*>(u_s + (m * nqv + q) * VS);
 #pragma unroll
-        for (int e = 0; e < E; ++e) acc[m] = fmaf(w[e], u_s[m * r + q * E + e], acc[m]);
+        for (int h = 0; h < E / 4; ++h) {
+          const float4 x = up[h];
+          acc[m] = fmaf(w[4 * h], x.x, acc[m]);
+          acc[m] = fmaf(w[4 * h + 1], x.y, acc[m]);
+          acc[m] = fmaf(w[4 * h + 2], x.z, acc[m]);
+          acc[m] = fmaf(w[4 * h + 3], x.w, acc[m]);
+        }
       }
     }
 #pragma unroll
-    for (int m = 0; m < kTileM; ++m) {
+    for (int m = 0; m < MT; ++m) {
       float s = warp_sum(acc[m]);
       if (lane == 0 && m < mt) {
         size_t row = (size_t)(m0 + m) * l_mul + l_add;
@@ -146,7 +160,7 @@ __global__ void __launch_bounds__(kThreads) k_w2(const T* __restrict__ W2, int r
   if (keys) {
     if (lane == 0) {
 #pragma unroll
-      for (int m = 0; m < kTileM; ++m) best_s[warp][m] = best[m];
+      for (int m = 0; m < MT; ++m) best_s[warp][m] = best[m];
     }
     __syncthreads();
     if (threadIdx.x < mt) {
@@ -314,7 +328,7 @@ cudaError_t launch_hproj(const Shape& s, const void* W1, const void* hidden, int
     k_hproj<float><<<grid, kThreads, 0, st>>>((const float*)W1, s.d + s.Hs, (const float*)hidden, N, s.d, s.r, P);
   else
     k_hproj<bf16><<<grid, kThreads, 0, st>>>((const bf16*)W1, s.d + s.Hs, (const bf16*)hidden, N, s.d, s.r, P);
-  return cudaGetLastError();
+  return note_launch(cudaGetLastError());
 }
 
 cudaError_t launch_u(const Shape& s, const void* W1, const float* P, int p_mul, int p_add, const float* S,
@@ -326,7 +340,31 @@ cudaError_t launch_u(const Shape& s, const void* W1, const float* P, int p_mul, 
   else
     k_u<bf16><<<grid, kThreads, 0, st>>>((const bf16*)W1, s.d + s.Hs, s.d, s.Hs, s.r, P, p_mul, p_add, S,
                                          s_stride, M, u);
+  return note_launch(cudaGetLastError());
+}
+
+template <typename T, int MT>
+cudaError_t launch_w2_t(const Shape& s, const void* W2, const float* u, int M, const void* Lb, int l_mul, int l_add,
+                        uint64_t* keys, float* logits, unsigned gx, cudaStream_t st) {
+  constexpr int E = Vec<T>::N;
+  dim3 grid(gx, cdiv(M, MT));
+  size_t smem = (size_t)MT * (s.r / E) * (E + UPad<T>::v) * sizeof(float);
+  auto kern = k_w2<T, MT>;
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+  }
+  kern<<<grid, kThreads, smem, st>>>((const T*)W2, s.r, s.V, u, M, (const T*)Lb, l_mul, l_add, keys, logits);
   return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t launch_w2_dt(const Shape& s, const void* W2, const float* u, int M, const void* Lb, int l_mul, int l_add,
+                         uint64_t* keys, float* logits, unsigned gx, cudaStream_t st) {
+  if (M >= 8) return launch_w2_t<T, 8>(s, W2, u, M, Lb, l_mul, l_add, keys, logits, gx, st);
+  if (M >= 4) return launch_w2_t<T, 4>(s, W2, u, M, Lb, l_mul, l_add, keys, logits, gx, st);
+  if (M >= 2) return launch_w2_t<T, 2>(s, W2, u, M, Lb, l_mul, l_add, keys, logits, gx, st);
+  return launch_w2_t<T, 1>(s, W2, u, M, Lb, l_mul, l_add, keys, logits, gx, st);
 }
 
 cudaError_t launch_w2(const Shape& s, const void* W2, const float* u, int M, const void* Lb, int l_mul, int l_add,
@@ -335,15 +373,9 @@ cudaError_t launch_w2(const Shape& s, const void* W2, const float* u, int M, con
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   unsigned gx = (unsigned)min((size_t)sms * 4, (size_t)cdiv(s.V, kWarps));
-  dim3 grid(gx, cdiv(M, kTileM));
-  size_t smem = (size_t)kTileM * s.r * sizeof(float);
-  if (s.dtype == 0)
-    k_w2<float><<<grid, kThreads, smem, st>>>((const float*)W2, s.r, s.V, u, M, (const float*)Lb, l_mul, l_add,
-                                              keys, logits);
-  else
-    k_w2<bf16><<<grid, kThreads, smem, st>>>((const bf16*)W2, s.r, s.V, u, M, (const bf16*)Lb, l_mul, l_add, keys,
-                                             logits);
-  return cudaGetLastError();
+  cudaError_t e = (s.dtype == 0) ? launch_w2_dt<float>(s, W2, u, M, Lb, l_mul, l_add, keys, logits, gx, st)
+                                 : launch_w2_dt<bf16>(s, W2, u, M, Lb, l_mul, l_add, keys, logits, gx, st);
+  return note_launch(e);
 }
 
 cudaError_t launch_gru(const Shape& s, const void* embed, const void* W_ih, const void* W_hh, const void* b_ih,
@@ -361,31 +393,31 @@ cudaError_t launch_gru(const Shape& s, const void* embed, const void* W_ih, cons
                                            (const bf16*)b_ih, (const bf16*)b_hh, s.d, s.Hs, s.V, tok_keys, tokens,
                                            tok_mul, tok_add, Sin, sin_stride, Sout, sout_stride, Sout2, sout2_stride,
                                            M, status);
-  return cudaGetLastError();
+  return note_launch(cudaGetLastError());
 }
 
 cudaError_t launch_tokens_from_keys(const uint64_t* keys, int B, int L, int32_t* tokens, cudaStream_t st) {
   k_tokens_from_keys<<<cdiv((size_t)B * L, 256), 256, 0, st>>>(keys, B, L, tokens);
-  return cudaGetLastError();
+  return note_launch(cudaGetLastError());
 }
 
 cudaError_t launch_copy_rows(const float* src, size_t src_stride, float* dst, size_t dst_stride, int rows, int n,
                              cudaStream_t st) {
   unsigned g = min(cdiv((size_t)rows * n, 256), 4096u);
   k_copy_rows<<<g, 256, 0, st>>>(src, src_stride, dst, dst_stride, rows, n);
-  return cudaGetLastError();
+  return note_launch(cudaGetLastError());
 }
 
 cudaError_t launch_row_argmax(const float* T, int rows, int V, uint64_t* keys, cudaStream_t st) {
   dim3 grid(cdiv(V, kArgChunk), rows);
   k_row_argmax<<<grid, 256, 0, st>>>(T, V, keys);
-  return cudaGetLastError();
+  return note_launch(cudaGetLastError());
 }
 
 cudaError_t launch_accept_count(const int32_t* draft, const uint64_t* keys, int B, int L, int32_t* out,
                                 cudaStream_t st) {
   k_accept_count<<<cdiv(B, 128), 128, 0, st>>>(draft, keys, B, L, out);
-  return cudaGetLastError();
+  return note_launch(cudaGetLastError());
 }
 
 }  // namespace domino

@@ -32,7 +32,8 @@ _TORCH_DTYPE = {DTYPE_F32: torch.float32, DTYPE_BF16: torch.bfloat16}
 
 EXPORTS = ("domino_workspace_bytes", "domino_draft_greedy", "domino_teacher_forced",
            "domino_accept_workspace_bytes", "domino_accept_len", "domino_status_string",
-           "domino_abi_version", "domino_debug_set_spin_limit")
+           "domino_abi_version", "domino_debug_set_spin_limit", "domino_launch_count",
+           "domino_greedy_plan")
 
 
 class DominoError(RuntimeError):
@@ -78,6 +79,10 @@ def lib(path: str = LIB_PATH) -> ctypes.CDLL:
         L.domino_abi_version.restype = i32
         L.domino_debug_set_spin_limit.argtypes = [ctypes.c_uint64]
         L.domino_debug_set_spin_limit.restype = ctypes.c_int
+        L.domino_launch_count.argtypes = []
+        L.domino_launch_count.restype = ctypes.c_uint64
+        L.domino_greedy_plan.argtypes = [ctypes.POINTER(Shape)]
+        L.domino_greedy_plan.restype = ctypes.c_char_p
         _lib = L
     return _lib
 
@@ -88,6 +93,16 @@ def status_string(code: int) -> str:
 
 def abi_version() -> int:
     return int(lib().domino_abi_version())
+
+
+def launch_count() -> int:
+    """Kernels the library has enqueued in this process so far."""
+    return int(lib().domino_launch_count())
+
+
+def greedy_plan(shape: Shape) -> str:
+    """Which kernels draft_greedy runs for this shape."""
+    return lib().domino_greedy_plan(ctypes.byref(shape)).decode()
 
 
 def set_spin_limit(limit: int) -> None:

@@ -147,6 +147,14 @@ DOMINO_API const char* domino_status_string(int code);
 /* DOMINO_ABI_VERSION of the loaded library. */
 DOMINO_API int32_t domino_abi_version(void);
 
+/* Number of kernels this library has enqueued in this process so far (all entry points, all
+ * devices).  Reading it before and after a region counts the library's launches in it. */
+DOMINO_API uint64_t domino_launch_count(void);
+
+/* Short static description of the kernel sequence domino_draft_greedy runs for `shape`
+ * (e.g. which fused kernel, or the per-phase kernels), or "invalid shape". */
+DOMINO_API const char* domino_greedy_plan(const domino_shape_t* shape);
+
 /* Test hook: iteration limit of the library's bounded device-wide waits (0 restores the
  * default, about one second).  A tiny limit makes waits give up early, which exercises the
  * DOMINO_STATUS_DEVICE_TIMEOUT path without faulting or hanging the GPU.  Process-wide; takes

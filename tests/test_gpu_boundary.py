@@ -84,3 +84,64 @@ def test_accept_len_workspace_from_head_sizing():
             k += 1
         want.append(k)
     assert acc.cpu().numpy().tolist() == want
+
+
+def _persistent_case(B=1, seed=300):
+    wl = dict(B=B, L=16, d=512, Hs=256, r=256, V=12000, dtype=1, weight_seed=seed, input_seed=seed + 1,
+              s0_std=0.2, peak=2.0, name="persistent")
+    return synth.make_workload(wl)
+
+
+def test_plan_names_the_fused_kernel_for_small_batches():
+    data = _persistent_case()
+    w, lb, h, S0 = G.device_inputs(data)
+    assert "persistent" in domino.greedy_plan(domino.make_shape(w, 1, 16))
+    assert "persistent" in domino.greedy_plan(domino.make_shape(w, 4, 16))
+    assert "per-phase" in domino.greedy_plan(domino.make_shape(w, 32, 16))
+
+
+def test_bounded_barrier_gives_up_with_status_and_the_context_survives():
+    """A spin limit of one poll makes the grid barriers give up at once: the kernel must report
+    DOMINO_STATUS_DEVICE_TIMEOUT and return; the next call with the default limit is correct."""
+    data = _persistent_case(B=2)
+    w, lb, h, S0 = G.device_inputs(data)
+    good, _, _ = domino.draft_greedy(w, lb, h, S0)
+    torch.cuda.synchronize()
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    domino.set_spin_limit(1)
+    try:
+        domino.draft_greedy(w, lb, h, S0, status=status)
+        torch.cuda.synchronize()
+    finally:
+        domino.set_spin_limit(0)
+    assert int(status.item()) == domino.STATUS_DEVICE_TIMEOUT
+    status.zero_()
+    again, _, _ = domino.draft_greedy(w, lb, h, S0, status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    assert torch.equal(again, good)
+
+
+def test_persistent_and_per_phase_paths_agree():
+    """B = 4 runs the fused kernel; the same rows drafted inside a B = 32 batch run the per-phase
+    kernels.  Tokens agree wherever the oracle replay margin is above 2e-2."""
+    import oracle
+    data4 = _persistent_case(B=4, seed=310)
+    w, lb, h, S0 = G.device_inputs(data4)
+    t4, l4, _ = domino.draft_greedy(w, lb, h, S0, logits_out=True)
+    lb32, h32, S032 = lb.repeat(8, 1, 1), h.repeat(8, 1, 1), S0.repeat(8, 1)
+    t32, l32, _ = domino.draft_greedy(w, lb32, h32, S032, logits_out=True)
+    torch.cuda.synchronize()
+    t4 = t4.cpu().numpy()
+    t32 = t32.cpu().numpy()[:4]
+    ref = oracle.head(data4["shape"], data4["weights"], data4["base_logits"], data4["hidden"], data4["S0"],
+                      tokens=np.ascontiguousarray(t4))
+    firm = ref["margin"] > G.MARGIN
+    # identical up to the first position where either path met a near-tie
+    for b in range(4):
+        for i in range(16):
+            if not firm[b, i]:
+                break
+            assert t4[b, i] == t32[b, i]
+    err = np.abs(l4.cpu().numpy() - ref["logits"])
+    assert (err <= G.LOGIT_ATOL + G.LOGIT_RTOL * np.abs(ref["logits"])).all()

@@ -28,6 +28,11 @@ SMALL = [
     _custom(2, 16, 512, 256, 256, 20008, 1, 120),         # bf16, full block, r = 256
     _custom(1, 1, 64, 64, 32, 64, 1, 130),                # a single position: no GRU update
     _custom(17, 3, 128, 64, 32, 3000, 1, 140),            # B not a multiple of the row tiles
+    # shapes the fused persistent kernel takes (bf16, r = 256, d and Hs multiples of 256, B <= 4)
+    _custom(3, 16, 256, 256, 256, 1000, 1, 150),          # odd B, vocabulary smaller than 8 rows/CTA
+    _custom(4, 9, 768, 512, 256, 33000, 1, 160),          # B = 4, odd L, ragged vocabulary slices
+    _custom(1, 1, 256, 256, 256, 5000, 1, 170),           # one position: no GRU update at all
+    _custom(2, 16, 1024, 256, 256, 40000, 1, 180, s0_std=1.0, peak=0.5),  # weak peaks: many near-ties
 ]
 
 

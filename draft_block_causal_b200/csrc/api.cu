@@ -123,6 +123,7 @@ const char* domino_status_string(int code) {
     case DOMINO_ERR_UNSUPPORTED: return "unsupported shape, layout or device";
     case DOMINO_ERR_CUDA: return "CUDA launch or query failed";
     case DOMINO_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case DOMINO_ERR_SCRATCH_LIMIT: return "shape needs more scratch than the library-owned array holds";
     case DOMINO_STATUS_DEVICE_TIMEOUT: return "device: a bounded wait gave up (outputs invalid)";
     case DOMINO_STATUS_BAD_TOKEN: return "device: teacher-forcing token outside [0, V)";
     default: return "unknown code";

@@ -23,6 +23,8 @@ ERR_INVALID_ARGUMENT = -1
 ERR_UNSUPPORTED = -2
 ERR_CUDA = -3
 ERR_WORKSPACE = -4
+ERR_SCRATCH_LIMIT = -5
+NOALLOC_SCRATCH_BYTES = 256 * 1024
 STATUS_DEVICE_TIMEOUT = 1
 STATUS_BAD_TOKEN = 2
 
@@ -33,7 +35,7 @@ _TORCH_DTYPE = {DTYPE_F32: torch.float32, DTYPE_BF16: torch.bfloat16}
 EXPORTS = ("domino_workspace_bytes", "domino_draft_greedy", "domino_teacher_forced",
            "domino_accept_workspace_bytes", "domino_accept_len", "domino_status_string",
            "domino_abi_version", "domino_debug_set_spin_limit", "domino_launch_count",
-           "domino_greedy_plan")
+           "domino_greedy_plan", "domino_draft_greedy_noalloc")
 
 
 class DominoError(RuntimeError):
@@ -81,6 +83,9 @@ def lib(path: str = LIB_PATH) -> ctypes.CDLL:
         L.domino_debug_set_spin_limit.restype = ctypes.c_int
         L.domino_launch_count.argtypes = []
         L.domino_launch_count.restype = ctypes.c_uint64
+        L.domino_draft_greedy_noalloc.argtypes = [ctypes.POINTER(Shape), ctypes.POINTER(Weights), vp, vp, vp, vp,
+                                                  vp, vp, vp, vp]
+        L.domino_draft_greedy_noalloc.restype = ctypes.c_int
         L.domino_greedy_plan.argtypes = [ctypes.POINTER(Shape)]
         L.domino_greedy_plan.restype = ctypes.c_char_p
         _lib = L
@@ -208,6 +213,34 @@ def draft_greedy(w: HeadWeights, base_logits, hidden, S0, tokens_out=None, logit
                                    _ptr(tokens_out), _ptr(logits_out), _ptr(states_out), _ptr(workspace),
                                    workspace.numel(), _ptr(status), _stream(stream))
     _check(rc, "domino_draft_greedy")
+    return tokens_out, logits_out, states_out
+
+
+def draft_greedy_noalloc(w: HeadWeights, base_logits, hidden, S0, tokens_out=None, logits_out=None,
+                         states_out=None, status=None, stream=None):
+    """Greedy drafting with no workspace (``domino_draft_greedy_noalloc``).
+
+    For callers that cannot allocate device memory at call time: the scratch is a fixed array
+    inside the library (NOALLOC_SCRATCH_BYTES per device).  Calls that overlap on the GPU share
+    that array and race -- keep them on one stream.  Pass preallocated output tensors to keep the
+    whole call free of allocations; ``logits_out=True`` / ``states_out=True`` allocate them here.
+    """
+    B, L, V = base_logits.shape
+    dev = base_logits.device
+    if tokens_out is None:
+        tokens_out = torch.empty((B, L), dtype=torch.int32, device=dev)
+    if logits_out is True:
+        logits_out = torch.empty((B, L, V), dtype=torch.float32, device=dev)
+    if states_out is True:
+        states_out = torch.empty((B, L, w.W_hh.shape[1]), dtype=torch.float32, device=dev)
+    logits_out = None if logits_out is False else logits_out
+    states_out = None if states_out is False else states_out
+    sh = make_shape(w, B, L)
+    ws = w.c_struct()
+    rc = lib().domino_draft_greedy_noalloc(ctypes.byref(sh), ctypes.byref(ws), _ptr(base_logits), _ptr(hidden),
+                                           _ptr(S0), _ptr(tokens_out), _ptr(logits_out), _ptr(states_out),
+                                           _ptr(status), _stream(stream))
+    _check(rc, "domino_draft_greedy_noalloc")
     return tokens_out, logits_out, states_out
 
 

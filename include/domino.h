@@ -60,6 +60,7 @@ extern "C" {
 #define DOMINO_ERR_UNSUPPORTED (-2)      /* valid but not handled (dims layout, device, grid)   */
 #define DOMINO_ERR_CUDA (-3)             /* a CUDA launch or query failed                       */
 #define DOMINO_ERR_WORKSPACE (-4)        /* workspace missing, misaligned (256 B) or too small  */
+#define DOMINO_ERR_SCRATCH_LIMIT (-5)    /* shape needs more than DOMINO_NOALLOC_SCRATCH_BYTES  */
 
 /* Device status codes written to *status_dev. */
 #define DOMINO_STATUS_OK 0
@@ -154,6 +155,37 @@ DOMINO_API uint64_t domino_launch_count(void);
 /* Short static description of the kernel sequence domino_draft_greedy runs for `shape`
  * (e.g. which fused kernel, or the per-phase kernels), or "invalid shape". */
 DOMINO_API const char* domino_greedy_plan(const domino_shape_t* shape);
+
+/* Greedy drafting without a workspace, for callers that cannot allocate device memory.
+ *
+ * The pages have no counterpart: this is a deployment convenience of this library.  Callers
+ * that cannot hand over a workspace include serving processes that reserved all free device
+ * memory for weights and KV cache at start-up (a later cudaMalloc would fail or fragment those
+ * pools), plugins whose host runtime owns the device allocator, and latency-critical loops that
+ * must not pay an allocation's implicit synchronisation.
+ *
+ * Same arguments, equations and outputs as domino_draft_greedy, minus the workspace.  The
+ * scratch memory is a library-owned, file-scope device array of DOMINO_NOALLOC_SCRATCH_BYTES
+ * bytes that every GPU which loads the library holds until the process exits; nothing is ever
+ * allocated or freed by this call.  Limits:
+ *   - only shapes the fused small-batch kernel handles (bf16, r = 256, B <= 4, d and Hs
+ *     multiples of 256) are accepted, else DOMINO_ERR_UNSUPPORTED;
+ *   - the kernel's scratch (about 4*B*L*(r+2) + 8*B*Hs bytes plus 768) must fit the array, else
+ *     DOMINO_ERR_SCRATCH_LIMIT -- e.g. B=4, L=16, Hs=1024 needs 99,328 bytes and fits;
+ *     B=4, L=64 does not;
+ *   - every call on a device shares that device's array, and the array keeps the previous
+ *     call's contents (the call clears what must start at zero).  Calls whose kernels overlap
+ *     on the GPU -- on different streams, or from different host threads -- race on the array
+ *     and give wrong results: order them on one stream.
+ *   - the first call on each device looks up the array's device address (cudaGetSymbolAddress,
+ *     with that device current); make that first call before any stream capture begins.
+ * status_dev may be NULL (the code then lands in the array).  Returns DOMINO_OK or a negative
+ * DOMINO_ERR_* code (nothing launched). */
+#define DOMINO_NOALLOC_SCRATCH_BYTES (256u * 1024u)
+DOMINO_API int domino_draft_greedy_noalloc(const domino_shape_t* shape, const domino_weights_t* weights,
+                                           const void* base_logits, const void* hidden, const float* S0,
+                                           int32_t* tokens_out, float* logits_out, float* states_out,
+                                           int32_t* status_dev, domino_stream_t stream);
 
 /* Test hook: iteration limit of the library's bounded device-wide waits (0 restores the
  * default, about one second).  A tiny limit makes waits give up early, which exercises the

@@ -360,8 +360,10 @@ def run_ours(args):
     return result
 
 
-def profile_driver(n: int, batch: int = 1):
-    """A short, fixed sequence of greedy calls for an external profiler (ncu -k ... -s ... -c ...)."""
+def profile_driver(n: int, batch: int = 1, trace: bool = False):
+    """A short, fixed sequence of greedy calls for an external profiler (ncu -k ... -s ... -c ...).
+    With `trace`, the last call records the fused kernel's phase clock stamps (CTA 0) and the
+    per-phase totals are printed as one JSON line."""
     import torch
     torch.cuda.set_device(0)
     device = torch.device("cuda", 0)
@@ -369,11 +371,35 @@ def profile_driver(n: int, batch: int = 1):
     pt = Point(wl, device)
     stream = torch.cuda.current_stream()
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
-    for _ in range(n):
+    L = pt.sh["L"]
+    buf = torch.zeros(4 + 10 * L, dtype=torch.int64, device=device)
+    for k in range(n):
         flush.zero_()
+        if trace and k == n - 1:
+            pt.domino.set_trace(buf)
         pt.greedy(stream)
     torch.cuda.synchronize()
+    pt.domino.set_trace(None)
     assert int(pt.status.item()) == 0
+    if trace:
+        t = buf.cpu().numpy().astype(np.int64)
+        mhz = torch.cuda.get_device_properties(0).clock_rate / 1e3 if hasattr(
+            torch.cuda.get_device_properties(0), "clock_rate") else 1965.0
+        names = ["stage_inputs", "w_hh", "w2_argmax", "argmax_barrier", "stage_embedding", "w_ih",
+                 "cell_w1_atomics", "state_barrier"]
+        tot = {k: 0 for k in names}
+        prev = t[2]
+        for i in range(L):
+            tb = 4 + 10 * i
+            marks = [tb + 0, tb + 1, tb + 2, tb + 3] + ([tb + 4, tb + 5, tb + 6, tb + 7] if i < L - 1 else [])
+            for name, m in zip(names, marks):
+                tot[name] += int(t[m] - prev)
+                prev = t[m]
+        res = {"plan": pt.domino.greedy_plan(pt.domino.make_shape(pt.w, pt.sh["B"], L)), "B": pt.sh["B"],
+               "clock_mhz_assumed": mhz, "prologue_us": round((t[1] - t[0]) / mhz, 2),
+               "first_barrier_us": round((t[2] - t[1]) / mhz, 2), "total_us": round((t[3] - t[0]) / mhz, 2),
+               "phases_us_summed_over_positions": {k: round(v / mhz, 2) for k, v in tot.items()}}
+        print(json.dumps(res), flush=True)
 
 
 def run_reference(args):
@@ -423,9 +449,11 @@ def main():
     ap.add_argument("--profile", type=int, default=0, metavar="N",
                     help="profiling driver: run N greedy calls of the headline workload (L2 flushed "
                          "before each) and exit without timing or output")
+    ap.add_argument("--profile-batch", type=int, default=1, help="batch of the profiling driver")
+    ap.add_argument("--trace", action="store_true", help="profiling driver: print the fused kernel's phase times")
     args = ap.parse_args()
     if args.profile:
-        profile_driver(args.profile)
+        profile_driver(args.profile, batch=args.profile_batch, trace=args.trace)
         return
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3

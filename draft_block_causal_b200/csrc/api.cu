@@ -3,6 +3,7 @@
 // never synchronises and never allocates.
 #include "domino.h"
 #include "internal.h"
+#include "gemm_tc.h"
 #include "persistent.h"
 
 #include <atomic>
@@ -13,6 +14,8 @@ namespace {
 
 std::atomic<uint64_t> g_spin_limit{0};
 std::atomic<uint64_t> g_launches{0};
+std::atomic<unsigned long long*> g_trace{nullptr};
+std::atomic<int> g_ntrace{0};
 
 inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
@@ -67,12 +70,13 @@ Workspace layout_workspace(const Shape& s, void* base) {
   w.sync = reinterpret_cast<uint32_t*>(take(kSyncWords * sizeof(uint32_t)));
   // sync, keys and a_acc are adjacent so that one memset clears all three
   w.keys = reinterpret_cast<uint64_t*>(take(BL * sizeof(uint64_t)));
-  w.a_acc = reinterpret_cast<float*>(take(BL * s.r * sizeof(float)));
+  w.a_acc = reinterpret_cast<float*>(take(BL * s.r * kAccReplicas * sizeof(float)));
   w.acc_keys = reinterpret_cast<uint64_t*>(take(BL * sizeof(uint64_t)));
   w.P = reinterpret_cast<float*>(take(BL * s.r * sizeof(float)));
   w.u = reinterpret_cast<float*>(take(BL * s.r * sizeof(float)));
   w.S = reinterpret_cast<float*>(take(2 * (size_t)s.B * s.Hs * sizeof(float)));
   w.states = reinterpret_cast<float*>(take(BL * s.Hs * sizeof(float)));
+  w.u16 = reinterpret_cast<__nv_bfloat16*>(take(BL * s.r * sizeof(__nv_bfloat16)));
   w.bytes = off;
   return w;
 }
@@ -82,6 +86,11 @@ size_t accept_workspace_bytes(int B, int L) {
   Shape s{B, L, 8, 8, 8, 8, DOMINO_DTYPE_F32};
   Workspace w = layout_workspace(s, nullptr);
   return w.bytes;
+}
+
+void debug_trace(unsigned long long** buf, int* n) {
+  *buf = g_trace.load(std::memory_order_relaxed);
+  *n = *buf ? g_ntrace.load(std::memory_order_relaxed) : 0;
 }
 
 cudaError_t note_launch(cudaError_t e) {
@@ -109,6 +118,13 @@ const char* domino_greedy_plan(const domino_shape_t* shape) {
   const Shape s = to_shape(shape);
   if (use_persistent_greedy(s)) return persistent_plan(s);
   return "per-phase kernels: k_hproj, then per position k_u + k_w2 (fused argmax) + k_gru, then k_tokens";
+}
+
+int domino_debug_set_trace(void* device_buf, int32_t n_entries) {
+  if (device_buf && (n_entries < 1 || (reinterpret_cast<uintptr_t>(device_buf) & 7u))) return DOMINO_ERR_INVALID_ARGUMENT;
+  g_ntrace.store(device_buf ? n_entries : 0, std::memory_order_relaxed);
+  g_trace.store(static_cast<unsigned long long*>(device_buf), std::memory_order_relaxed);
+  return DOMINO_OK;
 }
 
 int domino_debug_set_spin_limit(uint64_t limit) {
@@ -211,8 +227,17 @@ int domino_teacher_forced(const domino_shape_t* shape, const domino_weights_t* w
   for (int i = 0; i + 1 < s.L && e == cudaSuccess; ++i)
     e = launch_gru(s, w->embed, w->W_ih, w->W_hh, w->b_ih, w->b_hh, nullptr, tokens, s.L, i, SB + (size_t)i * s.Hs,
                    row, SB + (size_t)(i + 1) * s.Hs, row, nullptr, 0, s.B, st, cs);
-  if (e == cudaSuccess) e = launch_u(s, w->W1, ws.P, 1, 0, SB, s.Hs, (int)BL, ws.u, cs);
-  if (e == cudaSuccess) e = launch_w2(s, w->W2, ws.u, (int)BL, base_logits, 1, 0, nullptr, logits_out, cs);
+  // W2 product over all B*L positions at once: a tcgen05 GEMM with the L_base add fused into its
+  // epilogue (activations rounded to bf16 for the tensor cores), or the CUDA-core kernel.
+  const bool tc = s.dtype == DOMINO_DTYPE_BF16 && gemm_tc_supported(s.V, (int)BL, s.r, w->W2, ws.u16);
+  if (e == cudaSuccess) e = launch_u(s, w->W1, ws.P, 1, 0, SB, s.Hs, (int)BL, ws.u, cs, tc ? ws.u16 : nullptr);
+  if (e == cudaSuccess) {
+    if (tc)
+      e = gemm_tc_logits((const __nv_bfloat16*)w->W2, ws.u16, s.V, (int)BL, s.r, (const __nv_bfloat16*)base_logits,
+                         logits_out, st, spin_limit(), cs);
+    else
+      e = launch_w2(s, w->W2, ws.u, (int)BL, base_logits, 1, 0, nullptr, logits_out, cs);
+  }
   return cuda_rc(e);
 }
 

@@ -1,6 +1,7 @@
 // internal.h -- host-side declarations shared by the libdomino translation units.
 #pragma once
 
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -21,12 +22,19 @@ struct Workspace {
   float* u;            // [B*L][r] SiLU activations
   float* S;            // [2][B][Hs] greedy state ping-pong
   float* states;       // [B][L][Hs] teacher-forced states when the caller keeps none
-  float* a_acc;        // [L][B][r] pre-activation accumulators of the fused greedy kernel
+  __nv_bfloat16* u16;  // [B*L][r] activations rounded to bf16 (tensor-core W2 product)
+  float* a_acc;        // [L][kAccReplicas][B][r] pre-activation accumulators of the fused kernels
   size_t bytes;
 };
 constexpr int kSyncWords = 64;
+// The fused greedy kernels spread the W1 state-block partial sums over this many copies of the
+// accumulator (fewer atomics per address); the reader adds the copies.
+constexpr int kAccReplicas = 4;
 
 Workspace layout_workspace(const Shape& s, void* base);
+
+// Phase-trace buffer set by domino_debug_set_trace (null when off).
+void debug_trace(unsigned long long** buf, int* n);
 
 // Counts one enqueued kernel when `e` reports success; returns `e`.
 cudaError_t note_launch(cudaError_t e);
@@ -34,8 +42,9 @@ size_t accept_workspace_bytes(int B, int L);
 
 // ---- step kernels (one launch per phase; any storage type, any batch) ----
 cudaError_t launch_hproj(const Shape& s, const void* W1, const void* hidden, int N, float* P, cudaStream_t st);
+// u16 (optional): the same activations rounded to bf16, for the tensor-core W2 product.
 cudaError_t launch_u(const Shape& s, const void* W1, const float* P, int p_mul, int p_add, const float* S,
-                     size_t s_stride, int M, float* u, cudaStream_t st);
+                     size_t s_stride, int M, float* u, cudaStream_t st, __nv_bfloat16* u16 = nullptr);
 cudaError_t launch_w2(const Shape& s, const void* W2, const float* u, int M, const void* Lb, int l_mul,
                       int l_add, uint64_t* keys, float* logits, cudaStream_t st);
 cudaError_t launch_gru(const Shape& s, const void* embed, const void* W_ih, const void* W_hh, const void* b_ih,

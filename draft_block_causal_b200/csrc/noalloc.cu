@@ -42,7 +42,7 @@ Workspace compact_layout(const Shape& s, void* base) {
   w.status = reinterpret_cast<int32_t*>(take(sizeof(int32_t)));
   w.sync = reinterpret_cast<uint32_t*>(take(kSyncWords * sizeof(uint32_t)));
   w.keys = reinterpret_cast<uint64_t*>(take(BL * sizeof(uint64_t)));
-  w.a_acc = reinterpret_cast<float*>(take(BL * s.r * sizeof(float)));
+  w.a_acc = reinterpret_cast<float*>(take(BL * s.r * kAccReplicas * sizeof(float)));
   w.S = reinterpret_cast<float*>(take(2 * (size_t)s.B * s.Hs * sizeof(float)));
   w.bytes = off;
   return w;

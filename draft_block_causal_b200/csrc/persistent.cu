@@ -419,8 +419,11 @@ bool use_persistent_greedy(const Shape& s) {
 }
 
 const char* persistent_plan(const Shape& s) {
-  (void)s;
-  return "k_greedy_persistent: one cooperative launch, one CTA per SM, 16 positions with bounded grid barriers";
+  if (tmem_plan_fits(s, num_sms()))
+    return "k_greedy_tmem: one cooperative launch, one CTA per SM, GRU rows resident in TMEM, "
+           "positions separated by bounded grid barriers";
+  return "k_greedy_persistent: one cooperative launch, one CTA per SM, weights streamed from L2/HBM, "
+         "positions separated by bounded grid barriers";
 }
 
 cudaError_t launch_persistent_greedy(const Shape& s, const domino_weights_t& w, const void* base_logits,
@@ -429,6 +432,9 @@ cudaError_t launch_persistent_greedy(const Shape& s, const domino_weights_t& w, 
                                      cudaStream_t st) {
   const int G = num_sms();
   if (G < 1) return cudaErrorNoDevice;
+  if (tmem_plan_fits(s, G))
+    return launch_greedy_tmem(s, w, base_logits, hidden, S0, tokens_out, logits_out, states_out, ws, status, spin, G,
+                              st);
   PArgs a{};
   a.embed = (const bf16*)w.embed; a.W_ih = (const bf16*)w.W_ih; a.W_hh = (const bf16*)w.W_hh;
   a.b_ih = (const bf16*)w.b_ih; a.b_hh = (const bf16*)w.b_hh; a.W1 = (const bf16*)w.W1; a.W2 = (const bf16*)w.W2;

@@ -65,7 +65,7 @@ template <typename T>
 __global__ void __launch_bounds__(kThreads) k_u(const T* __restrict__ W1, int ldw, int d, int Hs, int r,
                                                 const float* __restrict__ P, int p_mul, int p_add,
                                                 const float* __restrict__ S, size_t s_stride, int M,
-                                                float* __restrict__ u) {
+                                                float* __restrict__ u, bf16* __restrict__ u16) {
   constexpr int E = Vec<T>::N;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int k = blockIdx.x * kWarps + warp;
@@ -93,7 +93,9 @@ __global__ void __launch_bounds__(kThreads) k_u(const T* __restrict__ W1, int ld
     float s = warp_sum(acc[m]);
     if (lane == 0 && m0 + m < M) {
       float a = P[(size_t)((m0 + m) * p_mul + p_add) * r + k] + s;
-      u[(size_t)(m0 + m) * r + k] = siluf_(a);
+      const float v = siluf_(a);
+      u[(size_t)(m0 + m) * r + k] = v;
+      if (u16) u16[(size_t)(m0 + m) * r + k] = __float2bfloat16_rn(v);
     }
   }
 }
@@ -332,14 +334,14 @@ cudaError_t launch_hproj(const Shape& s, const void* W1, const void* hidden, int
 }
 
 cudaError_t launch_u(const Shape& s, const void* W1, const float* P, int p_mul, int p_add, const float* S,
-                     size_t s_stride, int M, float* u, cudaStream_t st) {
+                     size_t s_stride, int M, float* u, cudaStream_t st, bf16* u16) {
   dim3 grid(cdiv(s.r, kWarps), cdiv(M, kTileM));
   if (s.dtype == 0)
     k_u<float><<<grid, kThreads, 0, st>>>((const float*)W1, s.d + s.Hs, s.d, s.Hs, s.r, P, p_mul, p_add, S,
-                                          s_stride, M, u);
+                                          s_stride, M, u, u16);
   else
     k_u<bf16><<<grid, kThreads, 0, st>>>((const bf16*)W1, s.d + s.Hs, s.d, s.Hs, s.r, P, p_mul, p_add, S,
-                                         s_stride, M, u);
+                                         s_stride, M, u, u16);
   return note_launch(cudaGetLastError());
 }
 

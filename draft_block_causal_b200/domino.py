@@ -24,7 +24,7 @@ ERR_UNSUPPORTED = -2
 ERR_CUDA = -3
 ERR_WORKSPACE = -4
 ERR_SCRATCH_LIMIT = -5
-NOALLOC_SCRATCH_BYTES = 256 * 1024
+NOALLOC_SCRATCH_BYTES = 1024 * 1024
 STATUS_DEVICE_TIMEOUT = 1
 STATUS_BAD_TOKEN = 2
 
@@ -35,7 +35,7 @@ _TORCH_DTYPE = {DTYPE_F32: torch.float32, DTYPE_BF16: torch.bfloat16}
 EXPORTS = ("domino_workspace_bytes", "domino_draft_greedy", "domino_teacher_forced",
            "domino_accept_workspace_bytes", "domino_accept_len", "domino_status_string",
            "domino_abi_version", "domino_debug_set_spin_limit", "domino_launch_count",
-           "domino_greedy_plan", "domino_draft_greedy_noalloc")
+           "domino_greedy_plan", "domino_draft_greedy_noalloc", "domino_debug_set_trace")
 
 
 class DominoError(RuntimeError):
@@ -86,6 +86,8 @@ def lib(path: str = LIB_PATH) -> ctypes.CDLL:
         L.domino_draft_greedy_noalloc.argtypes = [ctypes.POINTER(Shape), ctypes.POINTER(Weights), vp, vp, vp, vp,
                                                   vp, vp, vp, vp]
         L.domino_draft_greedy_noalloc.restype = ctypes.c_int
+        L.domino_debug_set_trace.argtypes = [vp, i32]
+        L.domino_debug_set_trace.restype = ctypes.c_int
         L.domino_greedy_plan.argtypes = [ctypes.POINTER(Shape)]
         L.domino_greedy_plan.restype = ctypes.c_char_p
         _lib = L
@@ -108,6 +110,15 @@ def launch_count() -> int:
 def greedy_plan(shape: Shape) -> str:
     """Which kernels draft_greedy runs for this shape."""
     return lib().domino_greedy_plan(ctypes.byref(shape)).decode()
+
+
+def set_trace(buf) -> None:
+    """Profiling hook: a CUDA int64 tensor receives SM-clock stamps of the fused kernel's phases
+    (CTA 0); None turns it off.  Layout in include/domino.h (domino_debug_set_trace)."""
+    if buf is None:
+        _check(lib().domino_debug_set_trace(None, 0), "domino_debug_set_trace")
+    else:
+        _check(lib().domino_debug_set_trace(ctypes.c_void_p(buf.data_ptr()), buf.numel()), "domino_debug_set_trace")
 
 
 def set_spin_limit(limit: int) -> None:

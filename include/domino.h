@@ -170,9 +170,9 @@ DOMINO_API const char* domino_greedy_plan(const domino_shape_t* shape);
  * allocated or freed by this call.  Limits:
  *   - only shapes the fused small-batch kernel handles (bf16, r = 256, B <= 4, d and Hs
  *     multiples of 256) are accepted, else DOMINO_ERR_UNSUPPORTED;
- *   - the kernel's scratch (about 4*B*L*(r+2) + 8*B*Hs bytes plus 768) must fit the array, else
- *     DOMINO_ERR_SCRATCH_LIMIT -- e.g. B=4, L=16, Hs=1024 needs 99,328 bytes and fits;
- *     B=4, L=64 does not;
+ *   - the kernel's scratch (16*B*L*r + 8*B*L + 8*B*Hs + 512 bytes, each piece rounded up to 256)
+ *     must fit the array, else DOMINO_ERR_SCRATCH_LIMIT -- e.g. B=4, L=16, Hs=1024 needs
+ *     295,936 bytes and fits; B=4, L=64 does not;
  *   - every call on a device shares that device's array, and the array keeps the previous
  *     call's contents (the call clears what must start at zero).  Calls whose kernels overlap
  *     on the GPU -- on different streams, or from different host threads -- race on the array
@@ -181,11 +181,19 @@ DOMINO_API const char* domino_greedy_plan(const domino_shape_t* shape);
  *     with that device current); make that first call before any stream capture begins.
  * status_dev may be NULL (the code then lands in the array).  Returns DOMINO_OK or a negative
  * DOMINO_ERR_* code (nothing launched). */
-#define DOMINO_NOALLOC_SCRATCH_BYTES (256u * 1024u)
+#define DOMINO_NOALLOC_SCRATCH_BYTES (1024u * 1024u)
 DOMINO_API int domino_draft_greedy_noalloc(const domino_shape_t* shape, const domino_weights_t* weights,
                                            const void* base_logits, const void* hidden, const float* S0,
                                            int32_t* tokens_out, float* logits_out, float* states_out,
                                            int32_t* status_dev, domino_stream_t stream);
+
+/* Profiling hook: when `device_buf` is non-NULL (8-byte aligned device memory of n_entries u64),
+ * the TMEM-resident fused greedy kernel records the SM clock of CTA 0 at its phase boundaries:
+ * [0] start, [1] prologue done, [2] first barrier passed, [3] end, and for position i at
+ * 4 + 10*i + {0: inputs staged, 1: W_hh products done, 2: W2 pass + CTA argmax done,
+ * 3: argmax barrier passed, 4: embedding row staged, 5: W_ih products done, 6: state and W1
+ * partials done, 7: state barrier passed}.  NULL turns it off.  Process-wide. */
+DOMINO_API int domino_debug_set_trace(void* device_buf, int32_t n_entries);
 
 /* Test hook: iteration limit of the library's bounded device-wide waits (0 restores the
  * default, about one second).  A tiny limit makes waits give up early, which exercises the

@@ -86,8 +86,8 @@ def test_accept_len_workspace_from_head_sizing():
     assert acc.cpu().numpy().tolist() == want
 
 
-def _persistent_case(B=1, seed=300):
-    wl = dict(B=B, L=16, d=512, Hs=256, r=256, V=12000, dtype=1, weight_seed=seed, input_seed=seed + 1,
+def _persistent_case(B=1, seed=300, Hs=256):
+    wl = dict(B=B, L=16, d=512, Hs=Hs, r=256, V=12000, dtype=1, weight_seed=seed, input_seed=seed + 1,
               s0_std=0.2, peak=2.0, name="persistent")
     return synth.make_workload(wl)
 
@@ -95,15 +95,20 @@ def _persistent_case(B=1, seed=300):
 def test_plan_names_the_fused_kernel_for_small_batches():
     data = _persistent_case()
     w, lb, h, S0 = G.device_inputs(data)
-    assert "persistent" in domino.greedy_plan(domino.make_shape(w, 1, 16))
-    assert "persistent" in domino.greedy_plan(domino.make_shape(w, 4, 16))
+    assert "k_greedy_persistent" in domino.greedy_plan(domino.make_shape(w, 1, 16))
+    assert "k_greedy_persistent" in domino.greedy_plan(domino.make_shape(w, 4, 16))
     assert "per-phase" in domino.greedy_plan(domino.make_shape(w, 32, 16))
+    data = _persistent_case(Hs=512)
+    w, lb, h, S0 = G.device_inputs(data)
+    assert "k_greedy_tmem" in domino.greedy_plan(domino.make_shape(w, 2, 16))
 
 
-def test_bounded_barrier_gives_up_with_status_and_the_context_survives():
+@pytest.mark.parametrize("Hs", [256, 512], ids=["l2-streamed", "tmem-resident"])
+def test_bounded_barrier_gives_up_with_status_and_the_context_survives(Hs):
     """A spin limit of one poll makes the grid barriers give up at once: the kernel must report
-    DOMINO_STATUS_DEVICE_TIMEOUT and return; the next call with the default limit is correct."""
-    data = _persistent_case(B=2)
+    DOMINO_STATUS_DEVICE_TIMEOUT and return (the TMEM variant freeing its tensor memory first);
+    the next call with the default limit is correct."""
+    data = _persistent_case(B=2, Hs=Hs)
     w, lb, h, S0 = G.device_inputs(data)
     good, _, _ = domino.draft_greedy(w, lb, h, S0)
     torch.cuda.synchronize()

@@ -33,6 +33,11 @@ SMALL = [
     _custom(4, 9, 768, 512, 256, 33000, 1, 160),          # B = 4, odd L, ragged vocabulary slices
     _custom(1, 1, 256, 256, 256, 5000, 1, 170),           # one position: no GRU update at all
     _custom(2, 16, 1024, 256, 256, 40000, 1, 180, s0_std=1.0, peak=0.5),  # weak peaks: many near-ties
+    # shapes the TMEM-resident variant takes (d and Hs multiples of 512)
+    _custom(3, 16, 1024, 512, 256, 9000, 1, 190),         # odd B, several GRU units per CTA
+    _custom(2, 5, 512, 512, 256, 3000, 1, 200),           # short block, small vocabulary
+    _custom(4, 16, 2560, 1024, 256, 20000, 1, 210),       # Qwen3-4B widths, B = 4
+    _custom(1, 16, 4096, 1024, 256, 7992, 1, 220, s0_std=1.0, peak=0.5),  # 8B widths, many near-ties
 ]
 
 
@@ -43,7 +48,13 @@ def test_greedy_small(wl):
     print(wl["name"], {k: v for k, v in res.items() if k != "tokens"})
 
 
-@pytest.mark.parametrize("wl", SMALL[1:4], ids=lambda w: w["name"] + f"-B{w['B']}")
+TF_CASES = SMALL[1:4] + [
+    _custom(20, 16, 512, 256, 256, 3000, 1, 230),   # B*L = 320: two column tiles, ragged vocabulary tile
+    _custom(1, 7, 256, 256, 128, 1024, 1, 240),     # exactly 8 vocabulary tiles, 7 positions
+]
+
+
+@pytest.mark.parametrize("wl", TF_CASES, ids=lambda w: w["name"] + f"-B{w['B']}")
 def test_teacher_forced_small(wl):
     data = synth.make_workload(wl, with_tokens=True)
     res = G.tf_parity(data)

@@ -86,7 +86,7 @@ def test_noalloc_without_status_pointer_or_optional_outputs():
 
 
 def test_noalloc_long_block_that_still_fits():
-    # B = 2 rows of 64 positions: 64 KiB of keys/accumulators per row, within the array
+    # B = 2 rows of 64 positions: about 0.5 MiB of keys and accumulators, within the array
     w, lb, h, S0 = _case(2, 64, 440)
     t_ref, l_ref, s_ref = domino.draft_greedy(w, lb, h, S0, logits_out=True, states_out=True)
     t, l, s = domino.draft_greedy_noalloc(w, lb, h, S0, logits_out=True, states_out=True)
@@ -101,7 +101,7 @@ def test_noalloc_rejects_shapes_beyond_its_scratch_and_unsupported_shapes():
     L = domino.lib()
     ws = w.c_struct()
     p = ctypes.c_void_p(lb.data_ptr())  # never dereferenced: the checks fail before any launch
-    # B = 4 rows of 64 positions need more than the 256 KiB array
+    # B = 4 rows of 64 positions need more than the 1 MiB array
     big = domino.Shape(4, 64, 512, 256, 256, 12000, 1)
     assert L.domino_draft_greedy_noalloc(ctypes.byref(big), ctypes.byref(ws), p, p, p, p, None, None,
                                          None, None) == domino.ERR_SCRATCH_LIMIT

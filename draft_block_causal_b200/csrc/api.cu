@@ -47,6 +47,7 @@ int check_weights(const domino_weights_t* w) {
   const void* p[] = {w->embed, w->W_ih, w->W_hh, w->b_ih, w->b_hh, w->W1, w->W2};
   for (const void* q : p)
     if (!q || !aligned16(q)) return DOMINO_ERR_INVALID_ARGUMENT;
+  if (w->embed_proj && !aligned16(w->embed_proj)) return DOMINO_ERR_INVALID_ARGUMENT;
   return DOMINO_OK;
 }
 
@@ -146,6 +147,30 @@ const char* domino_status_string(int code) {
   }
 }
 
+size_t domino_embed_proj_bytes(const domino_shape_t* shape) {
+  if (check_shape(shape) != DOMINO_OK) return 0;
+  return (size_t)shape->V * 3 * shape->Hs * sizeof(float);
+}
+
+int domino_project_embeddings(const domino_shape_t* shape, const domino_weights_t* w, float* embed_proj,
+                              int32_t* status_dev, domino_stream_t stream) {
+  int rc = check_shape(shape);
+  if (rc != DOMINO_OK) return rc;
+  if (!w || !w->embed || !w->W_ih || !embed_proj || !aligned16(w->embed) || !aligned16(w->W_ih) ||
+      !aligned16(embed_proj))
+    return DOMINO_ERR_INVALID_ARGUMENT;
+  const Shape s = to_shape(shape);
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  int32_t* st = status_dev;
+  cudaError_t e;
+  if (s.dtype == DOMINO_DTYPE_BF16 && gemm_tc_supported(s.V, 3 * s.Hs, s.d, w->embed, w->W_ih))
+    e = gemm_tc_store_f32((const __nv_bfloat16*)w->embed, (const __nv_bfloat16*)w->W_ih, s.V, 3 * s.Hs, s.d,
+                          embed_proj, 3 * s.Hs, st, spin_limit(), cs);
+  else
+    e = launch_project_simple(s, w->embed, w->W_ih, embed_proj, cs);
+  return cuda_rc(e);
+}
+
 size_t domino_workspace_bytes(const domino_shape_t* shape) {
   if (check_shape(shape) != DOMINO_OK) return 0;
   return layout_workspace(to_shape(shape), nullptr).bytes;
@@ -192,7 +217,7 @@ int domino_draft_greedy(const domino_shape_t* shape, const domino_weights_t* w, 
       float* S_next = ws.S + (size_t)(i & 1) * s.B * s.Hs;
       e = launch_gru(s, w->embed, w->W_ih, w->W_hh, w->b_ih, w->b_hh, ws.keys + (size_t)i * s.B, nullptr, 0, 0,
                      S_cur, s.Hs, S_next, s.Hs, states_out ? states_out + (size_t)(i + 1) * s.Hs : nullptr,
-                     (size_t)s.L * s.Hs, s.B, st, cs);
+                     (size_t)s.L * s.Hs, s.B, st, cs, w->embed_proj);
       S_cur = S_next;
     }
   }
@@ -226,7 +251,7 @@ int domino_teacher_forced(const domino_shape_t* shape, const domino_weights_t* w
   if (e == cudaSuccess) e = launch_copy_rows(S0, s.Hs, SB, row, s.B, s.Hs, cs);
   for (int i = 0; i + 1 < s.L && e == cudaSuccess; ++i)
     e = launch_gru(s, w->embed, w->W_ih, w->W_hh, w->b_ih, w->b_hh, nullptr, tokens, s.L, i, SB + (size_t)i * s.Hs,
-                   row, SB + (size_t)(i + 1) * s.Hs, row, nullptr, 0, s.B, st, cs);
+                   row, SB + (size_t)(i + 1) * s.Hs, row, nullptr, 0, s.B, st, cs, w->embed_proj);
   // W2 product over all B*L positions at once: a tcgen05 GEMM with the L_base add fused into its
   // epilogue (activations rounded to bf16 for the tensor cores), or the CUDA-core kernel.
   const bool tc = s.dtype == DOMINO_DTYPE_BF16 && gemm_tc_supported(s.V, (int)BL, s.r, w->W2, ws.u16);

@@ -197,7 +197,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   __syncthreads();
   tmem_fence_after_sync();
   if (warp == 1) tmem_dealloc(tbase, C::kTmemCols);
-  if (threadIdx.x == 0 && *abort_s) set_status(status, DOMINO_STATUS_DEVICE_TIMEOUT);
+  if (threadIdx.x == 0 && *abort_s && status) set_status(status, DOMINO_STATUS_DEVICE_TIMEOUT);
 }
 
 // ---- tensor maps ----

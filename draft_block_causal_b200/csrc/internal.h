@@ -50,7 +50,9 @@ cudaError_t launch_w2(const Shape& s, const void* W2, const float* u, int M, con
 cudaError_t launch_gru(const Shape& s, const void* embed, const void* W_ih, const void* W_hh, const void* b_ih,
                        const void* b_hh, const uint64_t* tok_keys, const int32_t* tokens, int tok_mul, int tok_add,
                        const float* Sin, size_t sin_stride, float* Sout, size_t sout_stride, float* Sout2,
-                       size_t sout2_stride, int M, int32_t* status, cudaStream_t st);
+                       size_t sout2_stride, int M, int32_t* status, cudaStream_t st, const float* Xp = nullptr);
+// Xp[v][n] = sum_c W_ih[n][c] embed[v][c] on CUDA cores (the tensor-core path lives in gemm_tc).
+cudaError_t launch_project_simple(const Shape& s, const void* embed, const void* W_ih, float* Xp, cudaStream_t st);
 cudaError_t launch_tokens_from_keys(const uint64_t* keys, int B, int L, int32_t* tokens, cudaStream_t st);
 cudaError_t launch_copy_rows(const float* src, size_t src_stride, float* dst, size_t dst_stride, int rows, int n,
                              cudaStream_t st);

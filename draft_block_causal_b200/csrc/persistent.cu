@@ -53,6 +53,7 @@ struct PArgs {
   int32_t* status;
   int B, L, d, Hs, V, maxu;
   unsigned long long spin_limit;
+  const float* Xp;  // [V][3Hs] input projection of the embedding table, or null
 };
 
 __device__ __forceinline__ unsigned ld_acquire(const unsigned* p) {
@@ -322,15 +323,23 @@ __global__ void __launch_bounds__(kPThreads, 1) k_greedy_persistent(PArgs p) {
     if (!grid_sync(p, epoch, flag_s)) return;
     if (i == L - 1) break;
 
-    // t_i, x = embed[t_i], gi = W_ih . x for the own units, GRU cell -> S_i
-    for (int t = tid; t < B * (d / 8); t += kPThreads) {
+    // t_i, x = embed[t_i], gi = W_ih . x for the own units (or gathered from the projection
+    // table), GRU cell -> S_i
+    if (p.Xp) {
+      for (int t = tid; t < B * 3 * nu; t += kPThreads) {
+        const int b = t / (3 * nu), R = t % (3 * nu), g = R / nu, jj = R % nu;
+        const int tok = min(max(key_index(__ldcg(p.keys + (size_t)i * B + b)), 0), V - 1);
+        gi_s[b * 3 * maxu + R] = __ldg(p.Xp + (size_t)tok * 3 * Hs + (size_t)g * Hs + j0 + jj);
+      }
+    }
+    for (int t = tid; t < (p.Xp ? 0 : B * (d / 8)); t += kPThreads) {
       const int b = t / (d / 8), q = t % (d / 8);
       // the key of a finished argmax always names a row in [0, V); the clamp only guards the load
       const int tok = min(max(key_index(__ldcg(p.keys + (size_t)i * B + b)), 0), V - 1);
       reinterpret_cast<uint4*>(x_s + (size_t)b * d)[q] = ldg16(p.embed + (size_t)tok * d + q * 8);
     }
     __syncthreads();
-    if (nu > 0) {
+    if (nu > 0 && !p.Xp) {
       auto rowp = [&](int row) { return p.W_ih + ((size_t)(row / nu) * Hs + j0 + row % nu) * d; };
       cta_rows_dot<BMAX, bf16>(rowp, 3 * nu, d, x_s, B, gi_s, 3 * maxu, warp, lane);
     }
@@ -419,7 +428,7 @@ bool use_persistent_greedy(const Shape& s) {
 }
 
 const char* persistent_plan(const Shape& s) {
-  if (tmem_plan_fits(s, num_sms()))
+  if (tmem_plan_fits(s, num_sms(), false))
     return "k_greedy_tmem: one cooperative launch, one CTA per SM, GRU rows resident in TMEM, "
            "positions separated by bounded grid barriers";
   return "k_greedy_persistent: one cooperative launch, one CTA per SM, weights streamed from L2/HBM, "
@@ -432,7 +441,7 @@ cudaError_t launch_persistent_greedy(const Shape& s, const domino_weights_t& w, 
                                      cudaStream_t st) {
   const int G = num_sms();
   if (G < 1) return cudaErrorNoDevice;
-  if (tmem_plan_fits(s, G))
+  if (tmem_plan_fits(s, G, w.embed_proj != nullptr))
     return launch_greedy_tmem(s, w, base_logits, hidden, S0, tokens_out, logits_out, states_out, ws, status, spin, G,
                               st);
   PArgs a{};
@@ -444,6 +453,7 @@ cudaError_t launch_persistent_greedy(const Shape& s, const domino_weights_t& w, 
   a.B = s.B; a.L = s.L; a.d = s.d; a.Hs = s.Hs; a.V = s.V;
   a.maxu = (s.Hs + G - 1) / G;
   a.spin_limit = spin;
+  a.Xp = w.embed_proj;
   // barrier counter, argmax keys and accumulators are contiguous in the workspace: one memset
   const size_t zero_bytes = (size_t)((char*)(ws.a_acc + (size_t)s.L * s.B * s.r) - (char*)ws.sync);
   cudaError_t e = cudaMemsetAsync(ws.sync, 0, zero_bytes, st);

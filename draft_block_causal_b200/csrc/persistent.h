@@ -16,7 +16,7 @@ const char* persistent_plan(const Shape& s);
 
 // The TMEM-resident variant (persistent_tmem.cu): fits when d and Hs are multiples of 512 and a
 // CTA's GRU rows fit in its 512 TMEM columns.
-bool tmem_plan_fits(const Shape& s, int G);
+bool tmem_plan_fits(const Shape& s, int G, bool proj);
 cudaError_t launch_greedy_tmem(const Shape& s, const domino_weights_t& w, const void* base_logits, const void* hidden,
                                const float* S0, int32_t* tokens_out, float* logits_out, float* states_out,
                                const Workspace& ws, int32_t* status, uint64_t spin, int G, cudaStream_t st);

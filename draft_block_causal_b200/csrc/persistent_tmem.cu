@@ -49,6 +49,7 @@ struct TArgs {
   unsigned long long spin_limit;
   unsigned long long* trace;  // [ntrace] SM clock stamps, or null
   int ntrace;
+  const float* Xp;  // [V][3Hs] input projection of the embedding table, or null
 };
 
 __device__ __forceinline__ unsigned ld_acquire_u32(const unsigned* p) {
@@ -260,7 +261,8 @@ __global__ void __launch_bounds__(kThreads2, 1) k_greedy_tmem(TArgs p) {
   const int nu = j1 - j0;
   const int ldw1 = d + Hs;
   const int cpri = d / 256, cprh = Hs / 256;       // TMEM columns per W_ih / W_hh row
-  const int colh = 3 * nu * cpri;                  // first W_hh column
+  const bool proj = p.Xp != nullptr;               // GRU input half gathered from the projection table
+  const int colh = proj ? 0 : 3 * nu * cpri;       // first W_hh column (W_ih rows are not kept with proj)
   const int rep = c % kRep;
 
   // shared memory
@@ -305,7 +307,8 @@ __global__ void __launch_bounds__(kThreads2, 1) k_greedy_tmem(TArgs p) {
       const int g = R / nu, jj = R % nu;
       const uint32_t* ri = reinterpret_cast<const uint32_t*>(p.W_ih + ((size_t)g * Hs + j0 + jj) * d) + l * cpri;
       const uint32_t* rh = reinterpret_cast<const uint32_t*>(p.W_hh + ((size_t)g * Hs + j0 + jj) * Hs) + l * cprh;
-      if (cpri % 4 == 0) {
+      if (proj) {
+      } else if (cpri % 4 == 0) {
         for (int cc = 0; cc < cpri; cc += 4)
           tmem_st4(ta + (uint32_t)(R * cpri + cc), __ldg(reinterpret_cast<const uint4*>(ri + cc)));
       } else {
@@ -463,9 +466,16 @@ __global__ void __launch_bounds__(kThreads2, 1) k_greedy_tmem(TArgs p) {
     // embedding table into L2 (the global winner's row is then an L2 hit for every CTA), and do
     // the W_hh half of the GRU, which does not depend on the argmax.
     if (i < L - 1) {
-      for (int t = tid; t < B * (d / 64); t += kThreads2) {
-        const int b = t / (d / 64), ln = t % (d / 64);
-        prefetch_l2(p.embed + (size_t)tok_s[b] * d + ln * 64);
+      if (proj) {
+        for (int t = tid; t < B * (3 * Hs / 32); t += kThreads2) {
+          const int b = t / (3 * Hs / 32), ln = t % (3 * Hs / 32);
+          prefetch_l2(p.Xp + (size_t)tok_s[b] * 3 * Hs + ln * 32);
+        }
+      } else {
+        for (int t = tid; t < B * (d / 64); t += kThreads2) {
+          const int b = t / (d / 64), ln = t % (d / 64);
+          prefetch_l2(p.embed + (size_t)tok_s[b] * d + ln * 64);
+        }
       }
       const float* Sprev = (i == 0) ? p.S0 : p.Sbuf + (size_t)((i - 1) & 1) * B * Hs;
       for (int t = tid; t < B * Hs; t += kThreads2) {
@@ -479,16 +489,27 @@ __global__ void __launch_bounds__(kThreads2, 1) k_greedy_tmem(TArgs p) {
     stamp(p.trace, p.ntrace, tb + 3);
     if (i == L - 1) break;
 
-    // t_i, x = embed[t_i] in the lane-sliced layout, gi = W_ih . x from TMEM, GRU cell -> S_i
-    for (int t = tid; t < B * (d / 2); t += kThreads2) {
-      const int b = t / (d / 2), w = t % (d / 2);
-      const int tok = min(max(key_index(__ldcg(p.keys + (size_t)i * B + b)), 0), V - 1);
-      x_t[((size_t)b * cpri + w % cpri) * 128 + w / cpri] =
-          __ldg(reinterpret_cast<const uint32_t*>(p.embed + (size_t)tok * d) + w);
+    // t_i; gi = W_ih . embed[t_i] for the own units: gathered from the projection table, or
+    // computed from TMEM with the embedding row staged in the lane-sliced layout; GRU cell -> S_i
+    if (proj) {
+      for (int t = tid; t < B * 3 * nu; t += kThreads2) {
+        const int b = t / (3 * nu), R = t % (3 * nu), g = R / nu, jj = R % nu;
+        const int tok = min(max(key_index(__ldcg(p.keys + (size_t)i * B + b)), 0), V - 1);
+        gi_s[b * 3 * maxu + R] = __ldg(p.Xp + (size_t)tok * 3 * Hs + (size_t)g * Hs + j0 + jj);
+      }
+      __syncthreads();
+      stamp(p.trace, p.ntrace, tb + 4);
+    } else {
+      for (int t = tid; t < B * (d / 2); t += kThreads2) {
+        const int b = t / (d / 2), w = t % (d / 2);
+        const int tok = min(max(key_index(__ldcg(p.keys + (size_t)i * B + b)), 0), V - 1);
+        x_t[((size_t)b * cpri + w % cpri) * 128 + w / cpri] =
+            __ldg(reinterpret_cast<const uint32_t*>(p.embed + (size_t)tok * d) + w);
+      }
+      __syncthreads();
+      stamp(p.trace, p.ntrace, tb + 4);
+      if (nu > 0) tmem_rows_dot<BMAX, uint32_t>(tbase, 0, cpri, 3 * nu, x_t, B, gi_s, 3 * maxu, warp, lane);
     }
-    __syncthreads();
-    stamp(p.trace, p.ntrace, tb + 4);
-    if (nu > 0) tmem_rows_dot<BMAX, uint32_t>(tbase, 0, cpri, 3 * nu, x_t, B, gi_s, 3 * maxu, warp, lane);
     __syncthreads();
     stamp(p.trace, p.ntrace, tb + 5);
     float* Snext = p.Sbuf + (size_t)(i & 1) * B * Hs;
@@ -562,10 +583,11 @@ cudaError_t launch_tmem_t(const TArgs& a, int G, size_t smem, cudaStream_t st) {
 
 }  // namespace
 
-bool tmem_plan_fits(const Shape& s, int G) {
+bool tmem_plan_fits(const Shape& s, int G, bool proj) {
   if (G < 1 || s.d % 512 != 0 || s.Hs % 512 != 0) return false;
   const int maxu = (s.Hs + G - 1) / G;
-  return 3 * maxu * (s.d / 256 + s.Hs / 256) <= kTmemCols && smem_bytes_tmem(4, s.d, s.Hs, maxu) <= 200 * 1024;
+  return 3 * maxu * ((proj ? 0 : s.d / 256) + s.Hs / 256) <= kTmemCols &&
+         smem_bytes_tmem(4, s.d, s.Hs, maxu) <= 200 * 1024;
 }
 
 cudaError_t launch_greedy_tmem(const Shape& s, const domino_weights_t& w, const void* base_logits, const void* hidden,
@@ -580,6 +602,7 @@ cudaError_t launch_greedy_tmem(const Shape& s, const domino_weights_t& w, const 
   a.B = s.B; a.L = s.L; a.d = s.d; a.Hs = s.Hs; a.V = s.V;
   a.maxu = (s.Hs + G - 1) / G;
   a.spin_limit = spin;
+  a.Xp = w.embed_proj;
   debug_trace(&a.trace, &a.ntrace);
   const size_t zero_bytes = (size_t)((char*)(ws.a_acc + (size_t)s.L * kRep * s.B * s.r) - (char*)ws.sync);
   cudaError_t e = cudaMemsetAsync(ws.sync, 0, zero_bytes, st);

@@ -176,6 +176,7 @@ __global__ void __launch_bounds__(kThreads) k_w2(const T* __restrict__ W2, int r
 // GRU update, PyTorch GRUCell form, for every row m < M and unit j < Hs:
 //   t = tok_keys ? index(tok_keys[m]) : tokens[m*tok_mul + tok_add];  x = embed[t];  h = Sin[m]
 //   r = sig(gi_r + gh_r), z = sig(gi_z + gh_z), n = tanh(gi_n + r * gh_n), h' = (1-z) n + z h[j]
+// gi = W_ih x is read from the projection table Xp[t] when one is given, else computed here.
 template <typename T>
 __global__ void __launch_bounds__(kThreads) k_gru(const T* __restrict__ embed, const T* __restrict__ W_ih,
                                                   const T* __restrict__ W_hh, const T* __restrict__ b_ih,
@@ -185,13 +186,14 @@ __global__ void __launch_bounds__(kThreads) k_gru(const T* __restrict__ embed, c
                                                   const float* __restrict__ Sin, size_t sin_stride,
                                                   float* __restrict__ Sout, size_t sout_stride,
                                                   float* __restrict__ Sout2, size_t sout2_stride, int M,
-                                                  int32_t* __restrict__ status) {
+                                                  int32_t* __restrict__ status, const float* __restrict__ Xp) {
   constexpr int E = Vec<T>::N;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int j = blockIdx.x * kWarps + warp;
   if (j >= Hs) return;
   const int m0 = blockIdx.y * kTileM;
   const T* xrow[kTileM];
+  int tk[kTileM];
   bool ok[kTileM];
 #pragma unroll
   for (int m = 0; m < kTileM; ++m) {
@@ -202,14 +204,15 @@ __global__ void __launch_bounds__(kThreads) k_gru(const T* __restrict__ embed, c
       ok[m] = (t >= 0 && t < V);
       if (!ok[m] && lane == 0 && j == 0) set_status(status, 2 /* DOMINO_STATUS_BAD_TOKEN */);
     }
-    xrow[m] = embed + (size_t)(ok[m] ? t : 0) * d;
+    tk[m] = ok[m] ? t : 0;
+    xrow[m] = embed + (size_t)tk[m] * d;
   }
   float gi[3][kTileM], gh[3][kTileM];
 #pragma unroll
   for (int g = 0; g < 3; ++g)
 #pragma unroll
     for (int m = 0; m < kTileM; ++m) gi[g][m] = gh[g][m] = 0.f;
-  for (int q = lane; q < d / E; q += 32) {
+  for (int q = lane; q < (Xp ? 0 : d / E); q += 32) {
     float w[3][E];
 #pragma unroll
     for (int g = 0; g < 3; ++g) widen(ldg16(W_ih + ((size_t)g * Hs + j) * d + q * E), w[g]);
@@ -252,7 +255,7 @@ __global__ void __launch_bounds__(kThreads) k_gru(const T* __restrict__ embed, c
     float si[3], sh[3];
 #pragma unroll
     for (int g = 0; g < 3; ++g) {
-      si[g] = warp_sum(gi[g][m]) + bi[g];
+      si[g] = (Xp ? (ok[m] ? Xp[(size_t)tk[m] * 3 * Hs + (size_t)g * Hs + j] : 0.f) : warp_sum(gi[g][m])) + bi[g];
       sh[g] = warp_sum(gh[g][m]) + bh[g];
     }
     if (lane == 0 && m0 + m < M) {
@@ -264,6 +267,38 @@ __global__ void __launch_bounds__(kThreads) k_gru(const T* __restrict__ embed, c
       Sout[(size_t)(m0 + m) * sout_stride + j] = hn;
       if (Sout2) Sout2[(size_t)(m0 + m) * sout2_stride + j] = hn;
     }
+  }
+}
+
+// Xp[v][n] = sum_c W_ih[n][c] embed[v][c] on CUDA cores (any storage type): a warp per (v, 8 n).
+template <typename T>
+__global__ void __launch_bounds__(kThreads) k_project(const T* __restrict__ embed, const T* __restrict__ W_ih, int V,
+                                                      int d, int N, float* __restrict__ Xp) {
+  constexpr int E = Vec<T>::N;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int v = blockIdx.y;
+  const int n0 = (blockIdx.x * kWarps + warp) * 8;
+  if (n0 >= N) return;
+  float acc[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) acc[k] = 0.f;
+  for (int q = lane; q < d / E; q += 32) {
+    float x[E];
+    widen(ldg16(embed + (size_t)v * d + q * E), x);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      if (n0 + k < N) {
+        float w[E];
+        widen(ldg16(W_ih + (size_t)(n0 + k) * d + q * E), w);
+#pragma unroll
+        for (int e = 0; e < E; ++e) acc[k] = fmaf(w[e], x[e], acc[k]);
+      }
+    }
+  }
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const float s = warp_sum(acc[k]);
+    if (lane == 0 && n0 + k < N) Xp[(size_t)v * N + n0 + k] = s;
   }
 }
 
@@ -383,18 +418,28 @@ cudaError_t launch_w2(const Shape& s, const void* W2, const float* u, int M, con
 cudaError_t launch_gru(const Shape& s, const void* embed, const void* W_ih, const void* W_hh, const void* b_ih,
                        const void* b_hh, const uint64_t* tok_keys, const int32_t* tokens, int tok_mul, int tok_add,
                        const float* Sin, size_t sin_stride, float* Sout, size_t sout_stride, float* Sout2,
-                       size_t sout2_stride, int M, int32_t* status, cudaStream_t st) {
+                       size_t sout2_stride, int M, int32_t* status, cudaStream_t st, const float* Xp) {
   dim3 grid(cdiv(s.Hs, kWarps), cdiv(M, kTileM));
   if (s.dtype == 0)
     k_gru<float><<<grid, kThreads, 0, st>>>((const float*)embed, (const float*)W_ih, (const float*)W_hh,
                                             (const float*)b_ih, (const float*)b_hh, s.d, s.Hs, s.V, tok_keys, tokens,
                                             tok_mul, tok_add, Sin, sin_stride, Sout, sout_stride, Sout2,
-                                            sout2_stride, M, status);
+                                            sout2_stride, M, status, Xp);
   else
     k_gru<bf16><<<grid, kThreads, 0, st>>>((const bf16*)embed, (const bf16*)W_ih, (const bf16*)W_hh,
                                            (const bf16*)b_ih, (const bf16*)b_hh, s.d, s.Hs, s.V, tok_keys, tokens,
                                            tok_mul, tok_add, Sin, sin_stride, Sout, sout_stride, Sout2, sout2_stride,
-                                           M, status);
+                                           M, status, Xp);
+  return note_launch(cudaGetLastError());
+}
+
+cudaError_t launch_project_simple(const Shape& s, const void* embed, const void* W_ih, float* Xp, cudaStream_t st) {
+  const int N = 3 * s.Hs;
+  dim3 grid(cdiv(N, kWarps * 8), s.V);
+  if (s.dtype == 0)
+    k_project<float><<<grid, kThreads, 0, st>>>((const float*)embed, (const float*)W_ih, s.V, s.d, N, Xp);
+  else
+    k_project<bf16><<<grid, kThreads, 0, st>>>((const bf16*)embed, (const bf16*)W_ih, s.V, s.d, N, Xp);
   return note_launch(cudaGetLastError());
 }
 

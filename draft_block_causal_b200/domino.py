@@ -35,7 +35,8 @@ _TORCH_DTYPE = {DTYPE_F32: torch.float32, DTYPE_BF16: torch.bfloat16}
 EXPORTS = ("domino_workspace_bytes", "domino_draft_greedy", "domino_teacher_forced",
            "domino_accept_workspace_bytes", "domino_accept_len", "domino_status_string",
            "domino_abi_version", "domino_debug_set_spin_limit", "domino_launch_count",
-           "domino_greedy_plan", "domino_draft_greedy_noalloc", "domino_debug_set_trace")
+           "domino_greedy_plan", "domino_draft_greedy_noalloc", "domino_debug_set_trace",
+           "domino_embed_proj_bytes", "domino_project_embeddings")
 
 
 class DominoError(RuntimeError):
@@ -49,7 +50,7 @@ class Shape(ctypes.Structure):
 
 
 class Weights(ctypes.Structure):
-    _fields_ = [(n, ctypes.c_void_p) for n in ("embed", "W_ih", "W_hh", "b_ih", "b_hh", "W1", "W2")]
+    _fields_ = [(n, ctypes.c_void_p) for n in ("embed", "W_ih", "W_hh", "b_ih", "b_hh", "W1", "W2", "embed_proj")]
 
 
 _lib = None
@@ -86,6 +87,10 @@ def lib(path: str = LIB_PATH) -> ctypes.CDLL:
         L.domino_draft_greedy_noalloc.argtypes = [ctypes.POINTER(Shape), ctypes.POINTER(Weights), vp, vp, vp, vp,
                                                   vp, vp, vp, vp]
         L.domino_draft_greedy_noalloc.restype = ctypes.c_int
+        L.domino_embed_proj_bytes.argtypes = [ctypes.POINTER(Shape)]
+        L.domino_embed_proj_bytes.restype = sz
+        L.domino_project_embeddings.argtypes = [ctypes.POINTER(Shape), ctypes.POINTER(Weights), vp, vp, vp]
+        L.domino_project_embeddings.restype = ctypes.c_int
         L.domino_debug_set_trace.argtypes = [vp, i32]
         L.domino_debug_set_trace.restype = ctypes.c_int
         L.domino_greedy_plan.argtypes = [ctypes.POINTER(Shape)]
@@ -153,6 +158,7 @@ class HeadWeights:
     b_hh: torch.Tensor
     W1: torch.Tensor
     W2: torch.Tensor
+    embed_proj: "torch.Tensor | None" = None  # [V, 3Hs] fp32 from project_embeddings, optional
 
     @property
     def dtype_code(self) -> int:
@@ -173,7 +179,11 @@ class HeadWeights:
             t = getattr(self, n)
             if not t.is_contiguous() or t.dtype != self.W2.dtype or not t.is_cuda:
                 raise ValueError(f"weight {n} must be a contiguous CUDA tensor of dtype {self.W2.dtype}")
-        return Weights(*(self.__dict__[n].data_ptr() for n in ("embed", "W_ih", "W_hh", "b_ih", "b_hh", "W1", "W2")))
+        xp = self.embed_proj
+        if xp is not None and (xp.dtype != torch.float32 or not xp.is_contiguous() or not xp.is_cuda):
+            raise ValueError("embed_proj must be a contiguous CUDA float32 tensor [V, 3Hs]")
+        ptrs = [self.__dict__[n].data_ptr() for n in ("embed", "W_ih", "W_hh", "b_ih", "b_hh", "W1", "W2")]
+        return Weights(*ptrs, xp.data_ptr() if xp is not None else None)
 
 
 def make_shape(w: HeadWeights, B: int, L: int) -> Shape:
@@ -186,6 +196,19 @@ def workspace_bytes(w: HeadWeights, B: int, L: int) -> int:
     if n == 0:
         raise DominoError(ERR_INVALID_ARGUMENT, "domino_workspace_bytes")
     return n
+
+
+def project_embeddings(w: HeadWeights, out=None, status=None, stream=None) -> torch.Tensor:
+    """The GRU input projection of every embedding row, [V, 3Hs] fp32 (domino_project_embeddings).
+    Assign the result to ``w.embed_proj`` to have every entry point gather it per token."""
+    d, Hs, r, V = w.dims()
+    if out is None:
+        out = torch.empty((V, 3 * Hs), dtype=torch.float32, device=w.W2.device)
+    sh = make_shape(w, 1, 1)
+    ws = w.c_struct()
+    rc = lib().domino_project_embeddings(ctypes.byref(sh), ctypes.byref(ws), _ptr(out), _ptr(status), _stream(stream))
+    _check(rc, "domino_project_embeddings")
+    return out
 
 
 def accept_workspace_bytes(B: int, L: int) -> int:

@@ -47,7 +47,7 @@ extern "C" {
 #define DOMINO_API
 #endif
 
-#define DOMINO_ABI_VERSION 1
+#define DOMINO_ABI_VERSION 2
 #define DOMINO_MAX_L 64
 
 /* Storage type of the weights, embedding table, base logits and hidden states. */
@@ -85,10 +85,28 @@ typedef struct {
  *   W2    [V, r]
  * The GRU cell is the PyTorch nn.GRUCell form:
  *   r = sig(W_ir x + b_ir + W_hr h + b_hr), z = sig(W_iz x + b_iz + W_hz h + b_hz),
- *   n = tanh(W_in x + b_in + r * (W_hn h + b_hn)), h' = (1 - z) * n + z * h.            */
+ *   n = tanh(W_in x + b_in + r * (W_hn h + b_hn)), h' = (1 - z) * n + z * h.
+ *   embed_proj [V, 3Hs] fp32, optional (NULL = not prepared): the GRU input half of every token,
+ *                     embed_proj[v][g*Hs + j] = sum_c W_ih[g*Hs + j][c] * embed[v][c], filled once
+ *                     per weight set by domino_project_embeddings.  When present, every entry point
+ *                     gathers the drafted (or given) token's row instead of multiplying W_ih by the
+ *                     embedding at each position.                                          */
 typedef struct {
   const void *embed, *W_ih, *W_hh, *b_ih, *b_hh, *W1, *W2;
+  const float* embed_proj;
 } domino_weights_t;
+
+/* Bytes of the optional input-projection table (V * 3Hs * 4), or 0 for an invalid shape. */
+DOMINO_API size_t domino_embed_proj_bytes(const domino_shape_t* shape);
+
+/* Fills embed_proj [V, 3Hs] fp32 with embed . W_ih^T (the GRU's input projection applied to every
+ * row of the embedding table at once) -- an algebraic precomputation of the encoder's input half
+ * (the drafted tokens' embeddings feed the GRU: review page section 二, GRU causal encoder), done
+ * once per weight set.  bf16 storage uses the tensor cores (fp32 accumulation); fp32 storage a
+ * CUDA-core kernel.  Only shape->d, Hs, V and dtype are used.  weights->embed_proj is ignored.
+ * Returns DOMINO_OK or a negative DOMINO_ERR_* code (nothing launched). */
+DOMINO_API int domino_project_embeddings(const domino_shape_t* shape, const domino_weights_t* weights,
+                                         float* embed_proj, int32_t* status_dev, domino_stream_t stream);
 
 /* Workspace bytes needed by domino_draft_greedy, domino_teacher_forced and domino_accept_len
  * for `shape` (the largest of the three), or 0 if the shape is invalid.  The workspace must be

@@ -40,8 +40,8 @@ def test_every_declared_symbol_is_exported(L):
 
 
 def test_abi_version_and_status_strings(L):
-    assert domino.abi_version() == 1
-    for code in (0, -1, -2, -3, -4, 1, 2):
+    assert domino.abi_version() == 2
+    for code in (0, -1, -2, -3, -4, -5, 1, 2):
         s = domino.status_string(code)
         assert s and s != "unknown code"
     assert domino.status_string(12345) == "unknown code"

@@ -6,6 +6,7 @@
 #include "gemm_tc.h"
 #include "persistent.h"
 
+#include <algorithm>
 #include <atomic>
 
 namespace domino {
@@ -57,6 +58,29 @@ inline int cuda_rc(cudaError_t e) { return e == cudaSuccess ? DOMINO_OK : DOMINO
 
 }  // namespace
 
+// One GRU update on the tensor cores for B rows: gh = W_hh . S from the two-term bf16 split of S
+// held in ws.S_hl (one GEMM with W_hh repeated along K), gi = W_ih . embed[t] from precomputed
+// columns of Gx, or a gather + GEMM here (need_gx), or the projection table; then the cell kernel,
+// which also refreshes ws.S_hl with the split of the new state.  Tokens come from keys[b] or
+// tokens[b * tok_mul + tok_add]; the Gx column of row b is b*xper + xoff.
+cudaError_t gru_step_tc(const Shape& s, const domino_weights_t& w, const Workspace& ws, const float* S_in,
+                        size_t s_stride, const uint64_t* keys, const int32_t* tokens, int tok_mul, int tok_add,
+                        float* Gx, int ldx, int xper, int xoff, bool need_gx, float* S_out, size_t so_stride,
+                        float* S_keep, size_t sk_stride, int32_t* status, cudaStream_t cs) {
+  using bf = __nv_bfloat16;
+  cudaError_t e = gemm_tc_store_f32_bn32((const bf*)w.W_hh, ws.S_hl, 3 * s.Hs, s.B, 2 * s.Hs, s.Hs, ws.Gh, s.B,
+                                         status, spin_limit(), cs);
+  if (e == cudaSuccess && !w.embed_proj && need_gx) {
+    e = launch_gather_rows((const bf*)w.embed, keys, tokens, 1, tok_mul, s.B, s.d, s.V, ws.X, cs);
+    if (e == cudaSuccess)
+      e = gemm_tc_store_f32_bn32((const bf*)w.W_ih, ws.X, 3 * s.Hs, s.B, s.d, 0, Gx, ldx, status, spin_limit(), cs);
+  }
+  if (e == cudaSuccess)
+    e = launch_cell(s, Gx, ldx, xper, xoff, w.embed_proj, ws.Gh, w.b_ih, w.b_hh, keys, tokens, tok_mul, tok_add,
+                    S_in, s_stride, S_out, so_stride, S_keep, sk_stride, status, cs, ws.S_hl);
+  return e;
+}
+
 Workspace layout_workspace(const Shape& s, void* base) {
   Workspace w{};
   char* p = static_cast<char*>(base);
@@ -78,6 +102,10 @@ Workspace layout_workspace(const Shape& s, void* base) {
   w.S = reinterpret_cast<float*>(take(2 * (size_t)s.B * s.Hs * sizeof(float)));
   w.states = reinterpret_cast<float*>(take(BL * s.Hs * sizeof(float)));
   w.u16 = reinterpret_cast<__nv_bfloat16*>(take(BL * s.r * sizeof(__nv_bfloat16)));
+  w.X = reinterpret_cast<__nv_bfloat16*>(take(BL * s.d * sizeof(__nv_bfloat16)));
+  w.Gx = reinterpret_cast<float*>(take(3 * (size_t)s.Hs * BL * sizeof(float)));
+  w.Gh = reinterpret_cast<float*>(take(3 * (size_t)s.Hs * s.B * sizeof(float)));
+  w.S_hl = reinterpret_cast<__nv_bfloat16*>(take(2 * BL * s.Hs * sizeof(__nv_bfloat16)));
   w.bytes = off;
   return w;
 }
@@ -118,6 +146,9 @@ const char* domino_greedy_plan(const domino_shape_t* shape) {
   if (check_shape(shape) != DOMINO_OK) return "invalid shape";
   const Shape s = to_shape(shape);
   if (use_persistent_greedy(s)) return persistent_plan(s);
+  if (s.dtype == DOMINO_DTYPE_BF16 && s.d % 64 == 0 && s.r % 64 == 0)
+    return "per-phase kernels: tcgen05 H-projection GEMM, then per position k_u + tcgen05 W2 GEMM with the argmax "
+           "in its epilogue + k_gru, then k_tokens";
   return "per-phase kernels: k_hproj, then per position k_u + k_w2 (fused argmax) + k_gru, then k_tokens";
 }
 
@@ -205,19 +236,52 @@ int domino_draft_greedy(const domino_shape_t* shape, const domino_weights_t* w, 
                                                                          spin_limit(), cs));
 
   const size_t BL = (size_t)s.B * s.L;
+  // Batches the fused kernel does not take: one launch per phase and position.  With bf16 storage
+  // the H-projection and the W2 product run on the tensor cores (tcgen05 GEMMs; the W2 product
+  // batch-major with the argmax folded into its epilogue), else on CUDA cores.
+  const bool tc = s.dtype == DOMINO_DTYPE_BF16 && s.d % 64 == 0 && s.r % 64 == 0 &&
+                  gemm_tc_supported((int)BL, s.r, s.d, hidden, w->W1) &&
+                  gemm_tc_supported(s.B, s.V, s.r, ws.u16, w->W2);
+  const bool tc_gru = tc && s.Hs % 64 == 0;
   cudaError_t e = cudaMemsetAsync(ws.keys, 0, BL * sizeof(uint64_t), cs);
-  if (e == cudaSuccess) e = launch_hproj(s, w->W1, hidden, (int)BL, ws.P, cs);
+  if (e == cudaSuccess) {
+    if (tc)  // P[n][k] = sum_c H[n][c] W1[k][c]: H [B*L x d], the first d columns of W1 (row stride d + Hs)
+      e = gemm_tc_store_f32_bn64((const __nv_bfloat16*)hidden, (const __nv_bfloat16*)w->W1, (int)BL, s.r, s.d,
+                                 s.d + s.Hs, ws.P, s.r, st, spin_limit(), cs);
+    else
+      e = launch_hproj(s, w->W1, hidden, (int)BL, ws.P, cs);
+  }
   if (e == cudaSuccess && states_out) e = launch_copy_rows(S0, s.Hs, states_out, (size_t)s.L * s.Hs, s.B, s.Hs, cs);
   const float* S_cur = S0;
+  if (e == cudaSuccess && tc_gru) e = launch_split_state(S0, s.Hs, s.B, s.Hs, ws.S_hl, cs);
   for (int i = 0; i < s.L && e == cudaSuccess; ++i) {
-    e = launch_u(s, w->W1, ws.P, s.L, i, S_cur, s.Hs, s.B, ws.u, cs);
-    if (e == cudaSuccess)
+    if (tc_gru)  // u = SiLU(P_i + W1[:, d:] . S) as one GEMM on the split state
+      e = gemm_tc_silu_u((const __nv_bfloat16*)w->W1 + s.d, s.d + s.Hs, ws.S_hl, s.r, s.B, s.Hs, ws.P + (size_t)i * s.r,
+                         (long long)s.L * s.r, ws.u16, nullptr, st, spin_limit(), cs);
+    else
+      e = launch_u(s, w->W1, ws.P, s.L, i, S_cur, s.Hs, s.B, ws.u, cs, tc ? ws.u16 : nullptr);
+    if (e == cudaSuccess && tc) {
+      for (int b0 = 0; b0 < s.B && e == cudaSuccess; b0 += 128) {  // bands of <= 128 batch rows
+        const size_t row0 = (size_t)b0 * s.L + i;                   // (row b0, position i)
+        e = gemm_tc_argmax(ws.u16 + (size_t)b0 * s.r, (const __nv_bfloat16*)w->W2, std::min(128, s.B - b0), s.V,
+                           s.r, (const __nv_bfloat16*)base_logits + row0 * s.V, (long long)s.L * s.V,
+                           ws.keys + (size_t)i * s.B + b0, logits_out ? logits_out + row0 * s.V : nullptr,
+                           (long long)s.L * s.V, st, spin_limit(), cs);
+      }
+    } else if (e == cudaSuccess) {
       e = launch_w2(s, w->W2, ws.u, s.B, base_logits, s.L, i, ws.keys + (size_t)i * s.B, logits_out, cs);
+    }
     if (e == cudaSuccess && i < s.L - 1) {
       float* S_next = ws.S + (size_t)(i & 1) * s.B * s.Hs;
-      e = launch_gru(s, w->embed, w->W_ih, w->W_hh, w->b_ih, w->b_hh, ws.keys + (size_t)i * s.B, nullptr, 0, 0,
-                     S_cur, s.Hs, S_next, s.Hs, states_out ? states_out + (size_t)(i + 1) * s.Hs : nullptr,
-                     (size_t)s.L * s.Hs, s.B, st, cs, w->embed_proj);
+      float* S_keep = states_out ? states_out + (size_t)(i + 1) * s.Hs : nullptr;
+      const uint64_t* keys_i = ws.keys + (size_t)i * s.B;
+      if (tc_gru) {
+        e = gru_step_tc(s, *w, ws, S_cur, s.Hs, keys_i, nullptr, 0, 0, ws.Gx, s.B, 1, 0, true, S_next, s.Hs, S_keep,
+                        (size_t)s.L * s.Hs, st, cs);
+      } else {
+        e = launch_gru(s, w->embed, w->W_ih, w->W_hh, w->b_ih, w->b_hh, keys_i, nullptr, 0, 0, S_cur, s.Hs, S_next,
+                       s.Hs, S_keep, (size_t)s.L * s.Hs, s.B, st, cs, w->embed_proj);
+      }
       S_cur = S_next;
     }
   }
@@ -247,17 +311,44 @@ int domino_teacher_forced(const domino_shape_t* shape, const domino_weights_t* w
   const size_t BL = (size_t)s.B * s.L;
   float* SB = states_out ? states_out : ws.states;  // [B][L][Hs]
   const size_t row = (size_t)s.L * s.Hs;
-  cudaError_t e = launch_hproj(s, w->W1, hidden, (int)BL, ws.P, cs);
+  using bf = __nv_bfloat16;
+  const bool tc = s.dtype == DOMINO_DTYPE_BF16 && s.d % 64 == 0 && s.r % 64 == 0 && s.Hs % 64 == 0 &&
+                  gemm_tc_supported((int)BL, s.r, s.d, hidden, w->W1);
+  cudaError_t e = tc ? gemm_tc_store_f32_bn64((const bf*)hidden, (const bf*)w->W1, (int)BL, s.r, s.d, s.d + s.Hs,
+                                              ws.P, s.r, st, spin_limit(), cs)
+                     : launch_hproj(s, w->W1, hidden, (int)BL, ws.P, cs);
   if (e == cudaSuccess) e = launch_copy_rows(S0, s.Hs, SB, row, s.B, s.Hs, cs);
-  for (int i = 0; i + 1 < s.L && e == cudaSuccess; ++i)
-    e = launch_gru(s, w->embed, w->W_ih, w->W_hh, w->b_ih, w->b_hh, nullptr, tokens, s.L, i, SB + (size_t)i * s.Hs,
-                   row, SB + (size_t)(i + 1) * s.Hs, row, nullptr, 0, s.B, st, cs, w->embed_proj);
+  if (e == cudaSuccess && tc) e = launch_split_state(S0, s.Hs, s.B, s.Hs, ws.S_hl, cs);
+  // The GRU input half for every given token at once (one GEMM over B*(L-1) gathered rows), unless
+  // the projection table already holds it.
+  const int NX = s.B * (s.L - 1);
+  if (e == cudaSuccess && tc && !w->embed_proj && NX > 0) {
+    e = launch_gather_rows((const bf*)w->embed, nullptr, tokens, s.L - 1, s.L, NX, s.d, s.V, ws.X, cs);
+    if (e == cudaSuccess)
+      e = gemm_tc_store_f32((const bf*)w->W_ih, ws.X, 3 * s.Hs, NX, s.d, ws.Gx, NX, st, spin_limit(), cs);
+  }
+  for (int i = 0; i + 1 < s.L && e == cudaSuccess; ++i) {
+    if (tc)
+      e = gru_step_tc(s, *w, ws, SB + (size_t)i * s.Hs, row, nullptr, tokens, s.L, i, ws.Gx, NX, s.L - 1, i, false,
+                      SB + (size_t)(i + 1) * s.Hs, row, nullptr, 0, st, cs);
+    else
+      e = launch_gru(s, w->embed, w->W_ih, w->W_hh, w->b_ih, w->b_hh, nullptr, tokens, s.L, i,
+                     SB + (size_t)i * s.Hs, row, SB + (size_t)(i + 1) * s.Hs, row, nullptr, 0, s.B, st, cs,
+                     w->embed_proj);
+  }
   // W2 product over all B*L positions at once: a tcgen05 GEMM with the L_base add fused into its
   // epilogue (activations rounded to bf16 for the tensor cores), or the CUDA-core kernel.
-  const bool tc = s.dtype == DOMINO_DTYPE_BF16 && gemm_tc_supported(s.V, (int)BL, s.r, w->W2, ws.u16);
-  if (e == cudaSuccess) e = launch_u(s, w->W1, ws.P, 1, 0, SB, s.Hs, (int)BL, ws.u, cs, tc ? ws.u16 : nullptr);
+  const bool tc_w2 = s.dtype == DOMINO_DTYPE_BF16 && gemm_tc_supported(s.V, (int)BL, s.r, w->W2, ws.u16);
+  if (e == cudaSuccess && tc && tc_w2) {  // u for every position: one GEMM on the split of all states
+    e = launch_split_state(SB, s.Hs, (int)BL, s.Hs, ws.S_hl, cs);
+    if (e == cudaSuccess)
+      e = gemm_tc_silu_u((const __nv_bfloat16*)w->W1 + s.d, s.d + s.Hs, ws.S_hl, s.r, (int)BL, s.Hs, ws.P, s.r,
+                         ws.u16, nullptr, st, spin_limit(), cs);
+  } else if (e == cudaSuccess) {
+    e = launch_u(s, w->W1, ws.P, 1, 0, SB, s.Hs, (int)BL, ws.u, cs, tc_w2 ? ws.u16 : nullptr);
+  }
   if (e == cudaSuccess) {
-    if (tc)
+    if (tc_w2)
       e = gemm_tc_logits((const __nv_bfloat16*)w->W2, ws.u16, s.V, (int)BL, s.r, (const __nv_bfloat16*)base_logits,
                          logits_out, st, spin_limit(), cs);
     else

@@ -18,6 +18,31 @@ bool gemm_tc_supported(int M, int N, int K, const void* A, const void* Bm);
 cudaError_t gemm_tc_store_f32(const __nv_bfloat16* A, const __nv_bfloat16* Bm, int M, int N, int K, float* out,
                               long long ldo, int32_t* status, uint64_t limit, cudaStream_t st);
 
+// Greedy step over a band of M <= 128 batch rows: for each row b < M,
+//   keys[b] = max(keys[b], key of argmax_v (Lb[b*ldl + v] + sum_k U[b][k] W2[v][k]))
+// (U [M x r], W2 [V x r] bf16; the argmax key orders by value, then lowest index).  When out is
+// non-null the logits are also stored: out[b * ldo + v].
+cudaError_t gemm_tc_argmax(const __nv_bfloat16* U, const __nv_bfloat16* W2, int M, int V, int r,
+                           const __nv_bfloat16* Lb, long long ldl, uint64_t* keys, float* out, long long ldo,
+                           int32_t* status, uint64_t limit, cudaStream_t st);
+
+// u16[n][k] = bf16(SiLU(P[n * ldp + k] + sum_j W1s[k][j] S[n][j])) for k < r, n < N, where the
+// fp32 state arrives as its two-term bf16 split S_hl [N x 2Hs] and W1s [r x Hs] has row stride ldw
+// (the state block of W1).  uf (optional) receives the fp32 activations.
+cudaError_t gemm_tc_silu_u(const __nv_bfloat16* W1s, long long ldw, const __nv_bfloat16* S_hl, int r, int N, int Hs,
+                           const float* P, long long ldp, __nv_bfloat16* u16, float* uf, int32_t* status,
+                           uint64_t limit, cudaStream_t st);
+
+// out[m * ldo + n] = sum_k A[m][k] Bm[n*ldb + k], with 64-wide output tiles (more CTAs for small N)
+cudaError_t gemm_tc_store_f32_bn64(const __nv_bfloat16* A, const __nv_bfloat16* Bm, int M, int N, int K,
+                                  long long ldb, float* out, long long ldo, int32_t* status, uint64_t limit,
+                                  cudaStream_t st);
+
+// out[m * ldo + n] = sum_k A[m][k mod a_kwrap] Bm[n][k] (a_kwrap = 0: no wrap), 32-wide output tiles.
+// With a_kwrap = K/2 and Bm = [hi | lo] this applies A to a two-term bf16 split of an fp32 operand.
+cudaError_t gemm_tc_store_f32_bn32(const __nv_bfloat16* A, const __nv_bfloat16* Bm, int M, int N, int K, int a_kwrap,
+                                  float* out, long long ldo, int32_t* status, uint64_t limit, cudaStream_t st);
+
 // logits[n][v] = Lb[n][v] + sum_k W2[v][k] U[n][k]   (W2 [V x r], U [N x r], Lb [N x V] bf16)
 cudaError_t gemm_tc_logits(const __nv_bfloat16* W2, const __nv_bfloat16* U, int V, int N, int r,
                            const __nv_bfloat16* Lb, float* logits, int32_t* status, uint64_t limit, cudaStream_t st);

@@ -23,6 +23,10 @@ struct Workspace {
   float* S;            // [2][B][Hs] greedy state ping-pong
   float* states;       // [B][L][Hs] teacher-forced states when the caller keeps none
   __nv_bfloat16* u16;  // [B*L][r] activations rounded to bf16 (tensor-core W2 product)
+  __nv_bfloat16* X;    // [B*L][d] gathered embedding rows (tensor-core GRU input product)
+  float* Gx;           // [3Hs][B*L] W_ih . x for every gathered row
+  float* Gh;           // [3Hs][B] W_hh . S
+  __nv_bfloat16* S_hl; // [B*L][2Hs] two-term bf16 split of states
   float* a_acc;        // [L][kAccReplicas][B][r] pre-activation accumulators of the fused kernels
   size_t bytes;
 };
@@ -53,6 +57,15 @@ cudaError_t launch_gru(const Shape& s, const void* embed, const void* W_ih, cons
                        size_t sout2_stride, int M, int32_t* status, cudaStream_t st, const float* Xp = nullptr);
 // Xp[v][n] = sum_c W_ih[n][c] embed[v][c] on CUDA cores (the tensor-core path lives in gemm_tc).
 cudaError_t launch_project_simple(const Shape& s, const void* embed, const void* W_ih, float* Xp, cudaStream_t st);
+// Large-batch GRU pieces for the tensor-core path (step_kernels.cu).
+cudaError_t launch_split_state(const float* S, size_t s_stride, int B, int Hs, __nv_bfloat16* S_hl, cudaStream_t st);
+cudaError_t launch_gather_rows(const __nv_bfloat16* embed, const uint64_t* keys, const int32_t* tokens, int per, int ld,
+                               int N, int d, int V, __nv_bfloat16* X, cudaStream_t st);
+cudaError_t launch_cell(const Shape& s, const float* Gx, int ldx, int xper, int xoff, const float* Xp, const float* Gh,
+                        const void* b_ih, const void* b_hh, const uint64_t* keys, const int32_t* tokens, int tok_mul,
+                        int tok_add, const float* Sin, size_t sin_stride, float* Sout, size_t sout_stride,
+                        float* Sout2, size_t sout2_stride, int32_t* status, cudaStream_t st,
+                        __nv_bfloat16* S_hl = nullptr);
 cudaError_t launch_tokens_from_keys(const uint64_t* keys, int B, int L, int32_t* tokens, cudaStream_t st);
 cudaError_t launch_copy_rows(const float* src, size_t src_stride, float* dst, size_t dst_stride, int rows, int n,
                              cudaStream_t st);

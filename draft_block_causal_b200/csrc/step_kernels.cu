@@ -302,6 +302,69 @@ __global__ void __launch_bounds__(kThreads) k_project(const T* __restrict__ embe
   }
 }
 
+// Two-term bf16 split of the fp32 state for the tensor cores: S_hl[b] = [hi | lo] with
+// hi = bf16(S), lo = bf16(S - hi), so hi + lo = S within 2^-16 |S|.
+__global__ void k_split_state(const float* __restrict__ S, size_t s_stride, int B, int Hs, bf16* __restrict__ S_hl) {
+  for (int t = blockIdx.x * blockDim.x + threadIdx.x; t < B * Hs; t += gridDim.x * blockDim.x) {
+    const int b = t / Hs, k = t % Hs;
+    const float v = S[(size_t)b * s_stride + k];
+    const bf16 hi = __float2bfloat16_rn(v);
+    S_hl[(size_t)b * 2 * Hs + k] = hi;
+    S_hl[(size_t)b * 2 * Hs + Hs + k] = __float2bfloat16_rn(v - __bfloat162float(hi));
+  }
+}
+
+// X[n] = embed[t_n] for n < N, t_n = key_index(keys[n]) (keys != null) or tokens[(n / per) * ld + n % per].
+__global__ void k_gather_rows(const bf16* __restrict__ embed, const uint64_t* __restrict__ keys,
+                              const int32_t* __restrict__ tokens, int per, int ld, int N, int d, int V,
+                              bf16* __restrict__ X) {
+  const int nv = d / 8;
+  for (int t = blockIdx.x * blockDim.x + threadIdx.x; t < N * nv; t += gridDim.x * blockDim.x) {
+    const int n = t / nv, q = t % nv;
+    int tok = keys ? key_index(keys[n]) : tokens[(size_t)(n / per) * ld + n % per];
+    tok = min(max(tok, 0), V - 1);  // out-of-range tokens are reported by the cell kernel
+    reinterpret_cast<uint4*>(X + (size_t)n * d)[q] = ldg16(embed + (size_t)tok * d + q * 8);
+  }
+}
+
+// GRU cell from precomputed gate pre-activations, PyTorch GRUCell form, for b < B, j < Hs:
+//   gi[g] = (Xp ? Xp[t][g*Hs + j] : Gx[(g*Hs + j) * ldx + cx(b)]) + b_ih,  gh[g] = Gh[(g*Hs+j)*B + b] + b_hh
+//   h' = (1 - z) n + z h,  r = sig(gi_r + gh_r), z = sig(gi_z + gh_z), n = tanh(gi_n + r gh_n)
+// cx(b) = b * xper + xoff.  Writes Sout (and Sout2) rows; t from keys[b] or tokens[b * tok_mul + tok_add].
+template <typename T>
+__global__ void k_cell(const float* __restrict__ Gx, int ldx, int xper, int xoff, const float* __restrict__ Xp,
+                       const float* __restrict__ Gh, const T* __restrict__ b_ih, const T* __restrict__ b_hh,
+                       const uint64_t* __restrict__ keys, const int32_t* __restrict__ tokens, int tok_mul, int tok_add,
+                       const float* __restrict__ Sin, size_t sin_stride, float* __restrict__ Sout, size_t sout_stride,
+                       float* __restrict__ Sout2, size_t sout2_stride, int B, int Hs, int V,
+                       int32_t* __restrict__ status, bf16* __restrict__ S_hl) {
+  for (int t = blockIdx.x * blockDim.x + threadIdx.x; t < B * Hs; t += gridDim.x * blockDim.x) {
+    const int b = t / Hs, j = t % Hs;
+    int tok = keys ? key_index(keys[b]) : tokens[(size_t)b * tok_mul + tok_add];
+    const bool ok = tok >= 0 && tok < V;
+    if (!ok && j == 0) set_status(status, 2 /* DOMINO_STATUS_BAD_TOKEN */);
+    tok = ok ? tok : 0;
+    float gi[3], gh[3];
+#pragma unroll
+    for (int g = 0; g < 3; ++g) {
+      const size_t row = (size_t)g * Hs + j;
+      gi[g] = (Xp ? Xp[(size_t)tok * 3 * Hs + row] : Gx[row * ldx + (size_t)b * xper + xoff]) + to_f32(b_ih[row]);
+      gh[g] = Gh[row * B + b] + to_f32(b_hh[row]);
+    }
+    const float rg = sigmoidf_(gi[0] + gh[0]);
+    const float zg = sigmoidf_(gi[1] + gh[1]);
+    const float ng = tanhf(gi[2] + rg * gh[2]);
+    const float hn = (1.f - zg) * ng + zg * Sin[(size_t)b * sin_stride + j];
+    Sout[(size_t)b * sout_stride + j] = hn;
+    if (Sout2) Sout2[(size_t)b * sout2_stride + j] = hn;
+    if (S_hl) {  // two-term bf16 split of the new state for the next tensor-core products
+      const bf16 hi = __float2bfloat16_rn(hn);
+      S_hl[(size_t)b * 2 * Hs + j] = hi;
+      S_hl[(size_t)b * 2 * Hs + Hs + j] = __float2bfloat16_rn(hn - __bfloat162float(hi));
+    }
+  }
+}
+
 __global__ void k_tokens_from_keys(const uint64_t* __restrict__ keys, int B, int L, int32_t* __restrict__ tokens) {
   int n = blockIdx.x * blockDim.x + threadIdx.x;
   if (n >= B * L) return;
@@ -440,6 +503,33 @@ cudaError_t launch_project_simple(const Shape& s, const void* embed, const void*
     k_project<float><<<grid, kThreads, 0, st>>>((const float*)embed, (const float*)W_ih, s.V, s.d, N, Xp);
   else
     k_project<bf16><<<grid, kThreads, 0, st>>>((const bf16*)embed, (const bf16*)W_ih, s.V, s.d, N, Xp);
+  return note_launch(cudaGetLastError());
+}
+
+cudaError_t launch_split_state(const float* S, size_t s_stride, int B, int Hs, bf16* S_hl, cudaStream_t st) {
+  k_split_state<<<min(cdiv((size_t)B * Hs, 256), 4096u), 256, 0, st>>>(S, s_stride, B, Hs, S_hl);
+  return note_launch(cudaGetLastError());
+}
+
+cudaError_t launch_gather_rows(const bf16* embed, const uint64_t* keys, const int32_t* tokens, int per, int ld, int N,
+                               int d, int V, bf16* X, cudaStream_t st) {
+  k_gather_rows<<<min(cdiv((size_t)N * (d / 8), 256), 8192u), 256, 0, st>>>(embed, keys, tokens, per, ld, N, d, V, X);
+  return note_launch(cudaGetLastError());
+}
+
+cudaError_t launch_cell(const Shape& s, const float* Gx, int ldx, int xper, int xoff, const float* Xp, const float* Gh,
+                        const void* b_ih, const void* b_hh, const uint64_t* keys, const int32_t* tokens, int tok_mul,
+                        int tok_add, const float* Sin, size_t sin_stride, float* Sout, size_t sout_stride,
+                        float* Sout2, size_t sout2_stride, int32_t* status, cudaStream_t st, bf16* S_hl) {
+  const unsigned g = min(cdiv((size_t)s.B * s.Hs, 256), 4096u);
+  if (s.dtype == 0)
+    k_cell<float><<<g, 256, 0, st>>>(Gx, ldx, xper, xoff, Xp, Gh, (const float*)b_ih, (const float*)b_hh, keys, tokens,
+                                     tok_mul, tok_add, Sin, sin_stride, Sout, sout_stride, Sout2, sout2_stride, s.B,
+                                     s.Hs, s.V, status, S_hl);
+  else
+    k_cell<bf16><<<g, 256, 0, st>>>(Gx, ldx, xper, xoff, Xp, Gh, (const bf16*)b_ih, (const bf16*)b_hh, keys, tokens,
+                                    tok_mul, tok_add, Sin, sin_stride, Sout, sout_stride, Sout2, sout2_stride, s.B, s.Hs,
+                                    s.V, status, S_hl);
   return note_launch(cudaGetLastError());
 }
 

@@ -53,6 +53,12 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
   return false;
 }
 
+// Warp-uniform bounded wait: every lane polls, and the warp succeeds only if every lane did.
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, uint64_t limit, volatile int* abort) {
+  const bool ok = mbar_wait_bounded(bar, parity, limit, abort);
+  return __all_sync(0xffffffffu, ok) != 0;
+}
+
 // ---------------- TMA (tiled, into this CTA only) ----------------
 __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* tmap, uint64_t* bar, int x, int y) {
   asm volatile(

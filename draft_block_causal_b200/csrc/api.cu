@@ -8,6 +8,7 @@
 
 #include <algorithm>
 #include <atomic>
+#include <string>
 
 namespace domino {
 
@@ -29,6 +30,8 @@ inline bool vec_layout_ok(int K, int dtype) {
   if (nv % 32 == 0) return true;
   return nv <= 32 && (nv & (nv - 1)) == 0;
 }
+
+}  // namespace
 
 int check_shape(const domino_shape_t* s) {
   if (!s) return DOMINO_ERR_INVALID_ARGUMENT;
@@ -52,6 +55,8 @@ int check_weights(const domino_weights_t* w) {
   return DOMINO_OK;
 }
 
+namespace {
+
 Shape to_shape(const domino_shape_t* s) { return Shape{s->B, s->L, s->d, s->Hs, s->r, s->V, s->dtype}; }
 
 inline int cuda_rc(cudaError_t e) { return e == cudaSuccess ? DOMINO_OK : DOMINO_ERR_CUDA; }
@@ -68,12 +73,13 @@ cudaError_t gru_step_tc(const Shape& s, const domino_weights_t& w, const Workspa
                         float* Gx, int ldx, int xper, int xoff, bool need_gx, float* S_out, size_t so_stride,
                         float* S_keep, size_t sk_stride, int32_t* status, cudaStream_t cs) {
   using bf = __nv_bfloat16;
-  cudaError_t e = gemm_tc_store_f32_bn32((const bf*)w.W_hh, ws.S_hl, 3 * s.Hs, s.B, 2 * s.Hs, s.Hs, ws.Gh, s.B,
-                                         status, spin_limit(), cs);
+  cudaError_t e = gemm_tc_store_f32_t((const bf*)w.W_hh, ws.S_hl, 3 * s.Hs, s.B, 2 * s.Hs, s.Hs, ws.Gh, 3 * s.Hs,
+                                      status, spin_limit(), cs);
   if (e == cudaSuccess && !w.embed_proj && need_gx) {
     e = launch_gather_rows((const bf*)w.embed, keys, tokens, 1, tok_mul, s.B, s.d, s.V, ws.X, cs);
     if (e == cudaSuccess)
-      e = gemm_tc_store_f32_bn32((const bf*)w.W_ih, ws.X, 3 * s.Hs, s.B, s.d, 0, Gx, ldx, status, spin_limit(), cs);
+      e = gemm_tc_store_f32_t((const bf*)w.W_ih, ws.X, 3 * s.Hs, s.B, s.d, 0, Gx, 3 * s.Hs, status,
+                              spin_limit(), cs, 1);
   }
   if (e == cudaSuccess)
     e = launch_cell(s, Gx, ldx, xper, xoff, w.embed_proj, ws.Gh, w.b_ih, w.b_hh, keys, tokens, tok_mul, tok_add,
@@ -146,10 +152,35 @@ const char* domino_greedy_plan(const domino_shape_t* shape) {
   if (check_shape(shape) != DOMINO_OK) return "invalid shape";
   const Shape s = to_shape(shape);
   if (use_persistent_greedy(s)) return persistent_plan(s);
-  if (s.dtype == DOMINO_DTYPE_BF16 && s.d % 64 == 0 && s.r % 64 == 0)
-    return "per-phase kernels: tcgen05 H-projection GEMM, then per position k_u + tcgen05 W2 GEMM with the argmax "
-           "in its epilogue + k_gru, then k_tokens";
+  if (s.dtype == DOMINO_DTYPE_BF16 && s.d % 64 == 0 && s.r % 64 == 0) {
+    if (s.Hs % 64 != 0)
+      return "per-phase kernels: tcgen05 H-projection GEMM, then per position k_u + tcgen05 W2 GEMM with the argmax "
+             "in its epilogue + k_gru, then k_tokens";
+    static thread_local std::string text;
+    int bn_h = 0, ks_h = 0, bn_i = 0, ks_i = 0;
+    gemm_tc_skinny_plan(3 * s.Hs + s.r, s.B, 2 * s.Hs, &bn_h, &ks_h);
+    gemm_tc_skinny_plan(3 * s.Hs, s.B, s.d, &bn_i, &ks_i);
+    text = "per-phase kernels: tcgen05 H-projection GEMM; per position a tcgen05 W2 GEMM with the argmax in its "
+           "epilogue, the GRU input half (" +
+           std::string("embedding gather + W_ih GEMM, tiles 128x") + std::to_string(bn_i) + " K-split " +
+           std::to_string(ks_i) + ", or a projection-table gather), k_cell, and one stacked W_hh|W1 GEMM (tiles 128x" +
+           std::to_string(bn_h) + " K-split " + std::to_string(ks_h) + ") for the next gh and activations; k_tokens";
+    return text.c_str();
+  }
   return "per-phase kernels: k_hproj, then per position k_u + k_w2 (fused argmax) + k_gru, then k_tokens";
+}
+
+int domino_debug_gemm(const void* A, const void* Bm, int32_t M, int32_t N, int32_t K, int32_t a_kwrap, float* out,
+                      int64_t ldo, int32_t trans, int32_t bn, int32_t ks, int32_t* status_dev,
+                      domino_stream_t stream) {
+  if (!A || !Bm || !out || M < 1 || N < 1 || K < 64 || K % 64 || a_kwrap < 0 || (a_kwrap && (a_kwrap % 64 || K % a_kwrap)))
+    return DOMINO_ERR_INVALID_ARGUMENT;
+  if (ldo < (trans ? M : N) || !aligned16(A) || !aligned16(Bm) || !aligned16(out)) return DOMINO_ERR_INVALID_ARGUMENT;
+  if (!((bn == 0 && ks == 0) || ((bn == 16 || bn == 32 || bn == 64 || bn == 128) && ks >= 1 && ks <= 8)))
+    return DOMINO_ERR_INVALID_ARGUMENT;
+  if (!gemm_tc_supported(M, N, K, A, Bm)) return DOMINO_ERR_UNSUPPORTED;
+  return cuda_rc(gemm_tc_debug((const __nv_bfloat16*)A, (const __nv_bfloat16*)Bm, M, N, K, a_kwrap, out, ldo, trans,
+                               bn, ks, status_dev, spin_limit(), static_cast<cudaStream_t>(stream)));
 }
 
 int domino_debug_set_trace(void* device_buf, int32_t n_entries) {
@@ -253,20 +284,28 @@ int domino_draft_greedy(const domino_shape_t* shape, const domino_weights_t* w, 
   }
   if (e == cudaSuccess && states_out) e = launch_copy_rows(S0, s.Hs, states_out, (size_t)s.L * s.Hs, s.B, s.Hs, cs);
   const float* S_cur = S0;
-  if (e == cudaSuccess && tc_gru) e = launch_split_state(S0, s.Hs, s.B, s.Hs, ws.S_hl, cs);
+  using bf = __nv_bfloat16;
+  const bf* W1s = (const bf*)w->W1 + s.d;  // state block of W1, row stride d + Hs
+  // tensor-core GRU: the split state feeds one GEMM that yields W_hh . S (for the next cell) and the
+  // next position's activations u = SiLU(P + W1_s . S)
+  const bool stacked = tc_gru && (3 * s.Hs) % 128 == 0;
+  if (e == cudaSuccess && tc_gru) {
+    e = launch_split_state(S0, s.Hs, s.B, s.Hs, ws.S_hl, cs);
+    if (e == cudaSuccess)
+      e = stacked ? gemm_tc_gru_u((const bf*)w->W_hh, W1s, s.d + s.Hs, ws.S_hl, s.Hs, s.r, s.B, ws.Gh, ws.P,
+                                  (long long)s.L * s.r, ws.u16, st, spin_limit(), cs)
+                  : gemm_tc_silu_u(W1s, s.d + s.Hs, ws.S_hl, s.r, s.B, s.Hs, ws.P, (long long)s.L * s.r, ws.u16,
+                                   nullptr, st, spin_limit(), cs);
+  }
   for (int i = 0; i < s.L && e == cudaSuccess; ++i) {
-    if (tc_gru)  // u = SiLU(P_i + W1[:, d:] . S) as one GEMM on the split state
-      e = gemm_tc_silu_u((const __nv_bfloat16*)w->W1 + s.d, s.d + s.Hs, ws.S_hl, s.r, s.B, s.Hs, ws.P + (size_t)i * s.r,
-                         (long long)s.L * s.r, ws.u16, nullptr, st, spin_limit(), cs);
-    else
-      e = launch_u(s, w->W1, ws.P, s.L, i, S_cur, s.Hs, s.B, ws.u, cs, tc ? ws.u16 : nullptr);
+    if (!tc_gru) e = launch_u(s, w->W1, ws.P, s.L, i, S_cur, s.Hs, s.B, ws.u, cs, tc ? ws.u16 : nullptr);
     if (e == cudaSuccess && tc) {
       for (int b0 = 0; b0 < s.B && e == cudaSuccess; b0 += 128) {  // bands of <= 128 batch rows
         const size_t row0 = (size_t)b0 * s.L + i;                   // (row b0, position i)
-        e = gemm_tc_argmax(ws.u16 + (size_t)b0 * s.r, (const __nv_bfloat16*)w->W2, std::min(128, s.B - b0), s.V,
-                           s.r, (const __nv_bfloat16*)base_logits + row0 * s.V, (long long)s.L * s.V,
-                           ws.keys + (size_t)i * s.B + b0, logits_out ? logits_out + row0 * s.V : nullptr,
-                           (long long)s.L * s.V, st, spin_limit(), cs);
+        e = gemm_tc_argmax(ws.u16 + (size_t)b0 * s.r, (const bf*)w->W2, std::min(128, s.B - b0), s.V, s.r,
+                           (const bf*)base_logits + row0 * s.V, (long long)s.L * s.V, ws.keys + (size_t)i * s.B + b0,
+                           logits_out ? logits_out + row0 * s.V : nullptr, (long long)s.L * s.V, st, spin_limit(),
+                           cs);
       }
     } else if (e == cudaSuccess) {
       e = launch_w2(s, w->W2, ws.u, s.B, base_logits, s.L, i, ws.keys + (size_t)i * s.B, logits_out, cs);
@@ -276,8 +315,27 @@ int domino_draft_greedy(const domino_shape_t* shape, const domino_weights_t* w, 
       float* S_keep = states_out ? states_out + (size_t)(i + 1) * s.Hs : nullptr;
       const uint64_t* keys_i = ws.keys + (size_t)i * s.B;
       if (tc_gru) {
-        e = gru_step_tc(s, *w, ws, S_cur, s.Hs, keys_i, nullptr, 0, 0, ws.Gx, s.B, 1, 0, true, S_next, s.Hs, S_keep,
-                        (size_t)s.L * s.Hs, st, cs);
+        if (!stacked)
+          e = gemm_tc_store_f32_t((const bf*)w->W_hh, ws.S_hl, 3 * s.Hs, s.B, 2 * s.Hs, s.Hs, ws.Gh, 3 * s.Hs,
+                                  st, spin_limit(), cs);
+        if (e == cudaSuccess && !w->embed_proj) {  // gi = W_ih . embed[t_i] for every row
+          e = launch_gather_rows((const bf*)w->embed, keys_i, nullptr, 1, 0, s.B, s.d, s.V, ws.X, cs);
+          if (e == cudaSuccess)
+            e = gemm_tc_store_f32_t((const bf*)w->W_ih, ws.X, 3 * s.Hs, s.B, s.d, 0, ws.Gx, 3 * s.Hs, st,
+                                    spin_limit(), cs, 1);
+        }
+        if (e == cudaSuccess)
+          e = launch_cell(s, ws.Gx, 3 * s.Hs, 1, 0, w->embed_proj, ws.Gh, w->b_ih, w->b_hh, keys_i, nullptr, 0, 0, S_cur,
+                          s.Hs, S_next, s.Hs, S_keep, (size_t)s.L * s.Hs, st, cs, ws.S_hl);
+        if (e == cudaSuccess) {  // gh for the next cell and the next position's activations
+          const float* P_next = ws.P + (size_t)(i + 1) * s.r;
+          if (stacked && i + 1 < s.L - 1)
+            e = gemm_tc_gru_u((const bf*)w->W_hh, W1s, s.d + s.Hs, ws.S_hl, s.Hs, s.r, s.B, ws.Gh, P_next,
+                              (long long)s.L * s.r, ws.u16, st, spin_limit(), cs);
+          else
+            e = gemm_tc_silu_u(W1s, s.d + s.Hs, ws.S_hl, s.r, s.B, s.Hs, P_next, (long long)s.L * s.r, ws.u16,
+                               nullptr, st, spin_limit(), cs);
+        }
       } else {
         e = launch_gru(s, w->embed, w->W_ih, w->W_hh, w->b_ih, w->b_hh, keys_i, nullptr, 0, 0, S_cur, s.Hs, S_next,
                        s.Hs, S_keep, (size_t)s.L * s.Hs, s.B, st, cs, w->embed_proj);
@@ -325,11 +383,11 @@ int domino_teacher_forced(const domino_shape_t* shape, const domino_weights_t* w
   if (e == cudaSuccess && tc && !w->embed_proj && NX > 0) {
     e = launch_gather_rows((const bf*)w->embed, nullptr, tokens, s.L - 1, s.L, NX, s.d, s.V, ws.X, cs);
     if (e == cudaSuccess)
-      e = gemm_tc_store_f32((const bf*)w->W_ih, ws.X, 3 * s.Hs, NX, s.d, ws.Gx, NX, st, spin_limit(), cs);
+      e = gemm_tc_store_f32((const bf*)w->W_ih, ws.X, 3 * s.Hs, NX, s.d, ws.Gx, 3 * s.Hs, st, spin_limit(), cs, 1);
   }
   for (int i = 0; i + 1 < s.L && e == cudaSuccess; ++i) {
     if (tc)
-      e = gru_step_tc(s, *w, ws, SB + (size_t)i * s.Hs, row, nullptr, tokens, s.L, i, ws.Gx, NX, s.L - 1, i, false,
+      e = gru_step_tc(s, *w, ws, SB + (size_t)i * s.Hs, row, nullptr, tokens, s.L, i, ws.Gx, 3 * s.Hs, s.L - 1, i, false,
                       SB + (size_t)(i + 1) * s.Hs, row, nullptr, 0, st, cs);
     else
       e = launch_gru(s, w->embed, w->W_ih, w->W_hh, w->b_ih, w->b_hh, nullptr, tokens, s.L, i,

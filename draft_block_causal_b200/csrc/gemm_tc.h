@@ -10,13 +10,15 @@
 
 namespace domino {
 
+
 // True when the tensor-core GEMM handles these sizes and pointers (K a multiple of 64, 16-byte
 // aligned operands, the driver's tensor-map encoder available).
 bool gemm_tc_supported(int M, int N, int K, const void* A, const void* Bm);
 
-// out[m * ldo + n] = sum_k A[m][k] Bm[n][k]   (A [M x K], Bm [N x K] bf16; out fp32)
+// out[m * ldo + n] (or out[n * ldo + m] when trans) = sum_k A[m][k] Bm[n][k]
+// (A [M x K], Bm [N x K] bf16; out fp32)
 cudaError_t gemm_tc_store_f32(const __nv_bfloat16* A, const __nv_bfloat16* Bm, int M, int N, int K, float* out,
-                              long long ldo, int32_t* status, uint64_t limit, cudaStream_t st);
+                              long long ldo, int32_t* status, uint64_t limit, cudaStream_t st, int trans = 0);
 
 // Greedy step over a band of M <= 128 batch rows: for each row b < M,
 //   keys[b] = max(keys[b], key of argmax_v (Lb[b*ldl + v] + sum_k U[b][k] W2[v][k]))
@@ -33,15 +35,34 @@ cudaError_t gemm_tc_silu_u(const __nv_bfloat16* W1s, long long ldw, const __nv_b
                            const float* P, long long ldp, __nv_bfloat16* u16, float* uf, int32_t* status,
                            uint64_t limit, cudaStream_t st);
 
+// One GEMM for both state products of a GRU step, on the two-term split S_hl [N x 2Hs]:
+//   Gh[n * 3Hs + m] = sum_j W_hh[m][j] S[n][j]                            (m < 3Hs)
+//   u16[n * r + k] = bf16(SiLU(P[n * ldp + k] + sum_j W1s[k][j] S[n][j])) (k < r)
+// W1s [r x Hs] has row stride ldw (the state block of W1).  3Hs must be a multiple of 128.
+cudaError_t gemm_tc_gru_u(const __nv_bfloat16* W_hh, const __nv_bfloat16* W1s, long long ldw,
+                          const __nv_bfloat16* S_hl, int Hs, int r, int N, float* Gh, const float* P, long long ldp,
+                          __nv_bfloat16* u16, int32_t* status, uint64_t limit, cudaStream_t st);
+
 // out[m * ldo + n] = sum_k A[m][k] Bm[n*ldb + k], with 64-wide output tiles (more CTAs for small N)
 cudaError_t gemm_tc_store_f32_bn64(const __nv_bfloat16* A, const __nv_bfloat16* Bm, int M, int N, int K,
                                   long long ldb, float* out, long long ldo, int32_t* status, uint64_t limit,
                                   cudaStream_t st);
 
-// out[m * ldo + n] = sum_k A[m][k mod a_kwrap] Bm[n][k] (a_kwrap = 0: no wrap), 32-wide output tiles.
+// out[n * ldo + m] = sum_k A[m][k mod a_kwrap] Bm[n][k] (a_kwrap = 0: no wrap) for a skinny Bm
+// (N = a batch of rows), stored transposed (n-major) so that per-row consumers read contiguously.
 // With a_kwrap = K/2 and Bm = [hi | lo] this applies A to a two-term bf16 split of an fp32 operand.
-cudaError_t gemm_tc_store_f32_bn32(const __nv_bfloat16* A, const __nv_bfloat16* Bm, int M, int N, int K, int a_kwrap,
-                                  float* out, long long ldo, int32_t* status, uint64_t limit, cudaStream_t st);
+// a_stream: A is read once per call (no reuse by later calls): its lines are evicted from L2 first.
+cudaError_t gemm_tc_store_f32_t(const __nv_bfloat16* A, const __nv_bfloat16* Bm, int M, int N, int K, int a_kwrap,
+                                float* out, long long ldo, int32_t* status, uint64_t limit, cudaStream_t st,
+                                int a_stream = 0);
+
+// One store-epilogue product with a forced plan (bn in {16, 32, 64, 128}, ks in 1..8) or the
+// automatic skinny plan (bn = ks = 0); out[m * ldo + n], or out[n * ldo + m] when trans.
+cudaError_t gemm_tc_debug(const __nv_bfloat16* A, const __nv_bfloat16* Bm, int M, int N, int K, int a_kwrap,
+                          float* out, long long ldo, int trans, int bn, int ks, int32_t* status, uint64_t limit,
+                          cudaStream_t st);
+// The automatic skinny plan for an M x N x K product (tile width bn, K split ks).
+void gemm_tc_skinny_plan(int M, int N, int K, int* bn, int* ks);
 
 // logits[n][v] = Lb[n][v] + sum_k W2[v][k] U[n][k]   (W2 [V x r], U [N x r], Lb [N x V] bf16)
 cudaError_t gemm_tc_logits(const __nv_bfloat16* W2, const __nv_bfloat16* U, int V, int N, int r,

@@ -6,7 +6,13 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include "domino.h"
+
 namespace domino {
+
+// Host-side argument checks shared by the entry points (DOMINO_OK or a negative DOMINO_ERR_*).
+int check_shape(const domino_shape_t* s);
+int check_weights(const domino_weights_t* w);
 
 struct Shape {
   int B, L, d, Hs, r, V, dtype;
@@ -24,8 +30,8 @@ struct Workspace {
   float* states;       // [B][L][Hs] teacher-forced states when the caller keeps none
   __nv_bfloat16* u16;  // [B*L][r] activations rounded to bf16 (tensor-core W2 product)
   __nv_bfloat16* X;    // [B*L][d] gathered embedding rows (tensor-core GRU input product)
-  float* Gx;           // [3Hs][B*L] W_ih . x for every gathered row
-  float* Gh;           // [3Hs][B] W_hh . S
+  float* Gx;           // [B*L][3Hs] W_ih . x for every gathered row
+  float* Gh;           // [B][3Hs] W_hh . S
   __nv_bfloat16* S_hl; // [B*L][2Hs] two-term bf16 split of states
   float* a_acc;        // [L][kAccReplicas][B][r] pre-activation accumulators of the fused kernels
   size_t bytes;

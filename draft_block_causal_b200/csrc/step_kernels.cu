@@ -8,6 +8,7 @@
 // to a tile of up to kTileM right-hand vectors, so each weight row is read once per tile.
 #include "common.cuh"
 #include "internal.h"
+#include "launch.cuh"
 
 namespace domino {
 
@@ -305,6 +306,8 @@ __global__ void __launch_bounds__(kThreads) k_project(const T* __restrict__ embe
 // Two-term bf16 split of the fp32 state for the tensor cores: S_hl[b] = [hi | lo] with
 // hi = bf16(S), lo = bf16(S - hi), so hi + lo = S within 2^-16 |S|.
 __global__ void k_split_state(const float* __restrict__ S, size_t s_stride, int B, int Hs, bf16* __restrict__ S_hl) {
+  pdl_wait();
+  pdl_trigger();
   for (int t = blockIdx.x * blockDim.x + threadIdx.x; t < B * Hs; t += gridDim.x * blockDim.x) {
     const int b = t / Hs, k = t % Hs;
     const float v = S[(size_t)b * s_stride + k];
@@ -318,6 +321,8 @@ __global__ void k_split_state(const float* __restrict__ S, size_t s_stride, int 
 __global__ void k_gather_rows(const bf16* __restrict__ embed, const uint64_t* __restrict__ keys,
                               const int32_t* __restrict__ tokens, int per, int ld, int N, int d, int V,
                               bf16* __restrict__ X) {
+  pdl_wait();
+  pdl_trigger();
   const int nv = d / 8;
   for (int t = blockIdx.x * blockDim.x + threadIdx.x; t < N * nv; t += gridDim.x * blockDim.x) {
     const int n = t / nv, q = t % nv;
@@ -328,7 +333,7 @@ __global__ void k_gather_rows(const bf16* __restrict__ embed, const uint64_t* __
 }
 
 // GRU cell from precomputed gate pre-activations, PyTorch GRUCell form, for b < B, j < Hs:
-//   gi[g] = (Xp ? Xp[t][g*Hs + j] : Gx[(g*Hs + j) * ldx + cx(b)]) + b_ih,  gh[g] = Gh[(g*Hs+j)*B + b] + b_hh
+//   gi[g] = (Xp ? Xp[t][g*Hs + j] : Gx[cx(b) * ldx + g*Hs + j]) + b_ih,  gh[g] = Gh[b * 3Hs + g*Hs + j] + b_hh
 //   h' = (1 - z) n + z h,  r = sig(gi_r + gh_r), z = sig(gi_z + gh_z), n = tanh(gi_n + r gh_n)
 // cx(b) = b * xper + xoff.  Writes Sout (and Sout2) rows; t from keys[b] or tokens[b * tok_mul + tok_add].
 template <typename T>
@@ -338,6 +343,8 @@ __global__ void k_cell(const float* __restrict__ Gx, int ldx, int xper, int xoff
                        const float* __restrict__ Sin, size_t sin_stride, float* __restrict__ Sout, size_t sout_stride,
                        float* __restrict__ Sout2, size_t sout2_stride, int B, int Hs, int V,
                        int32_t* __restrict__ status, bf16* __restrict__ S_hl) {
+  pdl_wait();
+  pdl_trigger();
   for (int t = blockIdx.x * blockDim.x + threadIdx.x; t < B * Hs; t += gridDim.x * blockDim.x) {
     const int b = t / Hs, j = t % Hs;
     int tok = keys ? key_index(keys[b]) : tokens[(size_t)b * tok_mul + tok_add];
@@ -348,8 +355,8 @@ __global__ void k_cell(const float* __restrict__ Gx, int ldx, int xper, int xoff
 #pragma unroll
     for (int g = 0; g < 3; ++g) {
       const size_t row = (size_t)g * Hs + j;
-      gi[g] = (Xp ? Xp[(size_t)tok * 3 * Hs + row] : Gx[row * ldx + (size_t)b * xper + xoff]) + to_f32(b_ih[row]);
-      gh[g] = Gh[row * B + b] + to_f32(b_hh[row]);
+      gi[g] = (Xp ? Xp[(size_t)tok * 3 * Hs + row] : Gx[((size_t)b * xper + xoff) * ldx + row]) + to_f32(b_ih[row]);
+      gh[g] = Gh[(size_t)b * 3 * Hs + row] + to_f32(b_hh[row]);
     }
     const float rg = sigmoidf_(gi[0] + gh[0]);
     const float zg = sigmoidf_(gi[1] + gh[1]);
@@ -366,6 +373,8 @@ __global__ void k_cell(const float* __restrict__ Gx, int ldx, int xper, int xoff
 }
 
 __global__ void k_tokens_from_keys(const uint64_t* __restrict__ keys, int B, int L, int32_t* __restrict__ tokens) {
+  pdl_wait();
+  pdl_trigger();
   int n = blockIdx.x * blockDim.x + threadIdx.x;
   if (n >= B * L) return;
   int b = n / L, i = n % L;
@@ -374,6 +383,8 @@ __global__ void k_tokens_from_keys(const uint64_t* __restrict__ keys, int B, int
 
 __global__ void k_copy_rows(const float* __restrict__ src, size_t src_stride, float* __restrict__ dst,
                             size_t dst_stride, int rows, int n) {
+  pdl_wait();
+  pdl_trigger();
   for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < rows * n; i += gridDim.x * blockDim.x) {
     int m = i / n, c = i % n;
     dst[(size_t)m * dst_stride + c] = src[(size_t)m * src_stride + c];
@@ -383,6 +394,8 @@ __global__ void k_copy_rows(const float* __restrict__ src, size_t src_stride, fl
 // keys[n] = max over the row of argmax_key(T[n][v], v); blockIdx.y = row, blockIdx.x = chunk.
 constexpr int kArgChunk = 8192;
 __global__ void __launch_bounds__(256) k_row_argmax(const float* __restrict__ T, int V, uint64_t* __restrict__ keys) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ uint64_t red[8];
   const int n = blockIdx.y;
   const int v0 = blockIdx.x * kArgChunk;
@@ -408,6 +421,8 @@ __global__ void __launch_bounds__(256) k_row_argmax(const float* __restrict__ T,
 
 __global__ void k_accept_count(const int32_t* __restrict__ draft, const uint64_t* __restrict__ keys, int B, int L,
                                int32_t* __restrict__ out) {
+  pdl_wait();
+  pdl_trigger();
   int b = blockIdx.x * blockDim.x + threadIdx.x;
   if (b >= B) return;
   int k = 0;
@@ -507,14 +522,16 @@ cudaError_t launch_project_simple(const Shape& s, const void* embed, const void*
 }
 
 cudaError_t launch_split_state(const float* S, size_t s_stride, int B, int Hs, bf16* S_hl, cudaStream_t st) {
-  k_split_state<<<min(cdiv((size_t)B * Hs, 256), 4096u), 256, 0, st>>>(S, s_stride, B, Hs, S_hl);
-  return note_launch(cudaGetLastError());
+  cudaError_t e = launch_pdl(k_split_state, dim3(min(cdiv((size_t)B * Hs, 256), 4096u)), dim3(256), 0, st, S, s_stride,
+                             B, Hs, S_hl);
+  return note_launch(e);
 }
 
 cudaError_t launch_gather_rows(const bf16* embed, const uint64_t* keys, const int32_t* tokens, int per, int ld, int N,
                                int d, int V, bf16* X, cudaStream_t st) {
-  k_gather_rows<<<min(cdiv((size_t)N * (d / 8), 256), 8192u), 256, 0, st>>>(embed, keys, tokens, per, ld, N, d, V, X);
-  return note_launch(cudaGetLastError());
+  cudaError_t e = launch_pdl(k_gather_rows, dim3(min(cdiv((size_t)N * (d / 8), 256), 8192u)), dim3(256), 0, st, embed,
+                             keys, tokens, per, ld, N, d, V, X);
+  return note_launch(e);
 }
 
 cudaError_t launch_cell(const Shape& s, const float* Gx, int ldx, int xper, int xoff, const float* Xp, const float* Gh,
@@ -522,39 +539,40 @@ cudaError_t launch_cell(const Shape& s, const float* Gx, int ldx, int xper, int 
                         int tok_add, const float* Sin, size_t sin_stride, float* Sout, size_t sout_stride,
                         float* Sout2, size_t sout2_stride, int32_t* status, cudaStream_t st, bf16* S_hl) {
   const unsigned g = min(cdiv((size_t)s.B * s.Hs, 256), 4096u);
+  cudaError_t e;
   if (s.dtype == 0)
-    k_cell<float><<<g, 256, 0, st>>>(Gx, ldx, xper, xoff, Xp, Gh, (const float*)b_ih, (const float*)b_hh, keys, tokens,
-                                     tok_mul, tok_add, Sin, sin_stride, Sout, sout_stride, Sout2, sout2_stride, s.B,
-                                     s.Hs, s.V, status, S_hl);
+    e = launch_pdl(k_cell<float>, dim3(g), dim3(256), 0, st, Gx, ldx, xper, xoff, Xp, Gh, (const float*)b_ih,
+                   (const float*)b_hh, keys, tokens, tok_mul, tok_add, Sin, sin_stride, Sout, sout_stride, Sout2,
+                   sout2_stride, s.B, s.Hs, s.V, status, S_hl);
   else
-    k_cell<bf16><<<g, 256, 0, st>>>(Gx, ldx, xper, xoff, Xp, Gh, (const bf16*)b_ih, (const bf16*)b_hh, keys, tokens,
-                                    tok_mul, tok_add, Sin, sin_stride, Sout, sout_stride, Sout2, sout2_stride, s.B, s.Hs,
-                                    s.V, status, S_hl);
-  return note_launch(cudaGetLastError());
+    e = launch_pdl(k_cell<bf16>, dim3(g), dim3(256), 0, st, Gx, ldx, xper, xoff, Xp, Gh, (const bf16*)b_ih,
+                   (const bf16*)b_hh, keys, tokens, tok_mul, tok_add, Sin, sin_stride, Sout, sout_stride, Sout2,
+                   sout2_stride, s.B, s.Hs, s.V, status, S_hl);
+  return note_launch(e);
 }
 
 cudaError_t launch_tokens_from_keys(const uint64_t* keys, int B, int L, int32_t* tokens, cudaStream_t st) {
-  k_tokens_from_keys<<<cdiv((size_t)B * L, 256), 256, 0, st>>>(keys, B, L, tokens);
-  return note_launch(cudaGetLastError());
+  cudaError_t e = launch_pdl(k_tokens_from_keys, dim3(cdiv((size_t)B * L, 256)), dim3(256), 0, st, keys, B, L, tokens);
+  return note_launch(e);
 }
 
 cudaError_t launch_copy_rows(const float* src, size_t src_stride, float* dst, size_t dst_stride, int rows, int n,
                              cudaStream_t st) {
   unsigned g = min(cdiv((size_t)rows * n, 256), 4096u);
-  k_copy_rows<<<g, 256, 0, st>>>(src, src_stride, dst, dst_stride, rows, n);
-  return note_launch(cudaGetLastError());
+  cudaError_t e = launch_pdl(k_copy_rows, dim3(g), dim3(256), 0, st, src, src_stride, dst, dst_stride, rows, n);
+  return note_launch(e);
 }
 
 cudaError_t launch_row_argmax(const float* T, int rows, int V, uint64_t* keys, cudaStream_t st) {
   dim3 grid(cdiv(V, kArgChunk), rows);
-  k_row_argmax<<<grid, 256, 0, st>>>(T, V, keys);
-  return note_launch(cudaGetLastError());
+  cudaError_t e = launch_pdl(k_row_argmax, grid, dim3(256), 0, st, T, V, keys);
+  return note_launch(e);
 }
 
 cudaError_t launch_accept_count(const int32_t* draft, const uint64_t* keys, int B, int L, int32_t* out,
                                 cudaStream_t st) {
-  k_accept_count<<<cdiv(B, 128), 128, 0, st>>>(draft, keys, B, L, out);
-  return note_launch(cudaGetLastError());
+  cudaError_t e = launch_pdl(k_accept_count, dim3(cdiv(B, 128)), dim3(128), 0, st, draft, keys, B, L, out);
+  return note_launch(e);
 }
 
 }  // namespace domino

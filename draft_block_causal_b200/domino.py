@@ -36,7 +36,8 @@ EXPORTS = ("domino_workspace_bytes", "domino_draft_greedy", "domino_teacher_forc
            "domino_accept_workspace_bytes", "domino_accept_len", "domino_status_string",
            "domino_abi_version", "domino_debug_set_spin_limit", "domino_launch_count",
            "domino_greedy_plan", "domino_draft_greedy_noalloc", "domino_debug_set_trace",
-           "domino_embed_proj_bytes", "domino_project_embeddings")
+           "domino_embed_proj_bytes", "domino_project_embeddings", "domino_arena_bytes",
+           "domino_pack_weights", "domino_set_l2_persistence", "domino_debug_gemm")
 
 
 class DominoError(RuntimeError):
@@ -95,6 +96,15 @@ def lib(path: str = LIB_PATH) -> ctypes.CDLL:
         L.domino_debug_set_trace.restype = ctypes.c_int
         L.domino_greedy_plan.argtypes = [ctypes.POINTER(Shape)]
         L.domino_greedy_plan.restype = ctypes.c_char_p
+        L.domino_arena_bytes.argtypes = [ctypes.POINTER(Shape)]
+        L.domino_arena_bytes.restype = sz
+        L.domino_pack_weights.argtypes = [ctypes.POINTER(Shape), ctypes.POINTER(Weights), vp, sz,
+                                          ctypes.POINTER(Weights), vp]
+        L.domino_pack_weights.restype = ctypes.c_int
+        L.domino_set_l2_persistence.argtypes = [ctypes.POINTER(Shape), ctypes.POINTER(Weights), vp, ctypes.c_float]
+        L.domino_set_l2_persistence.restype = ctypes.c_int
+        L.domino_debug_gemm.argtypes = [vp, vp, i32, i32, i32, i32, vp, ctypes.c_int64, i32, i32, i32, vp, vp]
+        L.domino_debug_gemm.restype = ctypes.c_int
         _lib = L
     return _lib
 
@@ -208,6 +218,57 @@ def project_embeddings(w: HeadWeights, out=None, status=None, stream=None) -> to
     ws = w.c_struct()
     rc = lib().domino_project_embeddings(ctypes.byref(sh), ctypes.byref(ws), _ptr(out), _ptr(status), _stream(stream))
     _check(rc, "domino_project_embeddings")
+    return out
+
+
+def arena_bytes(w: HeadWeights) -> int:
+    n = int(lib().domino_arena_bytes(ctypes.byref(make_shape(w, 1, 1))))
+    if n == 0:
+        raise DominoError(ERR_INVALID_ARGUMENT, "domino_arena_bytes")
+    return n
+
+
+def pack_weights(w: HeadWeights, stream=None) -> HeadWeights:
+    """Copy W2, W1, W_hh, W_ih, b_ih, b_hh into one contiguous arena (domino_pack_weights) and return
+    HeadWeights whose tensors are views of it (embed and embed_proj are shared with ``w``)."""
+    nbytes = arena_bytes(w)
+    arena = torch.empty(nbytes, dtype=torch.uint8, device=w.W2.device)
+    sh = make_shape(w, 1, 1)
+    src = w.c_struct()
+    out = Weights()
+    rc = lib().domino_pack_weights(ctypes.byref(sh), ctypes.byref(src), ctypes.c_void_p(arena.data_ptr()),
+                                   nbytes, ctypes.byref(out), _stream(stream))
+    _check(rc, "domino_pack_weights")
+    dt = w.W2.dtype
+    es = torch.empty((), dtype=dt).element_size()
+
+    def view(name):
+        t = getattr(w, name)
+        off = getattr(out, name) - arena.data_ptr()
+        return arena[off:off + t.numel() * es].view(dt).view(t.shape)
+
+    return HeadWeights(embed=w.embed, W_ih=view("W_ih"), W_hh=view("W_hh"), b_ih=view("b_ih"), b_hh=view("b_hh"),
+                       W1=view("W1"), W2=view("W2"), embed_proj=w.embed_proj)
+
+
+def set_l2_persistence(w: HeadWeights, stream, hit_ratio: float = 1.0) -> None:
+    """Opt-in L2 residency of packed weights for kernels on ``stream`` (domino_set_l2_persistence);
+    ``hit_ratio=0`` clears it and restores the context's persisting-L2 set-aside."""
+    sh = make_shape(w, 1, 1)
+    ws = w.c_struct()
+    rc = lib().domino_set_l2_persistence(ctypes.byref(sh), ctypes.byref(ws), _stream(stream), float(hit_ratio))
+    _check(rc, "domino_set_l2_persistence")
+
+
+def debug_gemm(A, B, out=None, trans=False, a_kwrap=0, bn=0, ks=0, status=None, stream=None) -> torch.Tensor:
+    """The tensor-core GEMM engine on its own (domino_debug_gemm): fp32 A[:, k mod K'] . B^T for bf16
+    A [M, K'] and B [N, K]; [M, N], or [N, M] when ``trans``.  bn/ks force a plan (0, 0: automatic)."""
+    M, N, K = A.shape[0], B.shape[0], B.shape[1]
+    if out is None:
+        out = torch.empty((N, M) if trans else (M, N), dtype=torch.float32, device=A.device)
+    rc = lib().domino_debug_gemm(_ptr(A), _ptr(B), M, N, K, int(a_kwrap), _ptr(out), out.shape[1], int(bool(trans)),
+                                 int(bn), int(ks), _ptr(status), _stream(stream))
+    _check(rc, "domino_debug_gemm")
     return out
 
 

@@ -108,6 +108,40 @@ DOMINO_API size_t domino_embed_proj_bytes(const domino_shape_t* shape);
 DOMINO_API int domino_project_embeddings(const domino_shape_t* shape, const domino_weights_t* weights,
                                          float* embed_proj, int32_t* status_dev, domino_stream_t stream);
 
+/* ---- Weight arena and L2 residency (opt-in) ----
+ *
+ * Every position of a block re-reads W2, W1's state block, W_hh and (without the projection
+ * table) W_ih: about 110 MB at the pages' Qwen3-8B shapes, which B200's L2 (126 MB) can hold
+ * between positions and, with a persisting window, between blocks.
+ *
+ * domino_arena_bytes: bytes of one contiguous arena holding W2, W1, W_hh, W_ih, b_ih and b_hh in
+ * that order (each region 256-byte aligned; the embedding table and the projection table stay
+ * where the caller keeps them), or 0 for an invalid shape.  Only d, Hs, r, V and dtype are used.
+ *
+ * domino_pack_weights: copies the six tensors of `src` into `arena` (device memory, 256-byte
+ * aligned, at least domino_arena_bytes long; caller-owned) with device-to-device copies on
+ * `stream`, and fills `packed` with pointers into the arena (embed and embed_proj are copied
+ * from `src` unchanged).  `packed` is usable by every entry point once the copies have run.
+ * Returns DOMINO_OK, DOMINO_ERR_INVALID_ARGUMENT, DOMINO_ERR_WORKSPACE (arena missing, misaligned
+ * or too small) or DOMINO_ERR_CUDA.
+ *
+ * domino_set_l2_persistence: with 0 < hit_ratio <= 1, sets the access-policy window of `stream`
+ * (a created stream, not the legacy default stream) over the packed hot range -- W2 through W_ih,
+ * or through W_hh when weights->embed_proj is set -- with persisting hits and streaming misses,
+ * and raises this context's persisting-L2 set-aside to min(range, device maximum); when the
+ * range exceeds the set-aside, only that fraction of its lines (times hit_ratio) is marked
+ * persisting.  Kernels launched on `stream` afterwards keep those weights in L2 across calls.
+ * hit_ratio = 0 clears the window, returns persisting lines to normal and restores the
+ * set-aside the context had before the first window.  The set-aside belongs to the calling
+ * process's context on the current device and ends with it.  Returns DOMINO_OK,
+ * DOMINO_ERR_INVALID_ARGUMENT (weights not packed, stream NULL, hit_ratio outside [0, 1]),
+ * DOMINO_ERR_UNSUPPORTED (no persisting L2 on this device) or DOMINO_ERR_CUDA. */
+DOMINO_API size_t domino_arena_bytes(const domino_shape_t* shape);
+DOMINO_API int domino_pack_weights(const domino_shape_t* shape, const domino_weights_t* src, void* arena,
+                                   size_t arena_bytes, domino_weights_t* packed, domino_stream_t stream);
+DOMINO_API int domino_set_l2_persistence(const domino_shape_t* shape, const domino_weights_t* weights,
+                                         domino_stream_t stream, float hit_ratio);
+
 /* Workspace bytes needed by domino_draft_greedy, domino_teacher_forced and domino_accept_len
  * for `shape` (the largest of the three), or 0 if the shape is invalid.  The workspace must be
  * device memory aligned to 256 bytes; its contents need no initialisation. */
@@ -212,6 +246,20 @@ DOMINO_API int domino_draft_greedy_noalloc(const domino_shape_t* shape, const do
  * 3: argmax barrier passed, 4: embedding row staged, 5: W_ih products done, 6: state and W1
  * partials done, 7: state barrier passed}.  NULL turns it off.  Process-wide. */
 DOMINO_API int domino_debug_set_trace(void* device_buf, int32_t n_entries);
+
+/* Test and tuning hook for the tensor-core GEMM engine behind the batched paths:
+ *   out[m * ldo + n] = sum_k A[m][k mod K'] * B[n][k]      (trans = 0)
+ *   out[n * ldo + m] = the same                             (trans = 1)
+ * A [M, K'] bf16 with K' = a_kwrap (0: K' = K; else K is a multiple of K'), B [N, K] bf16, out fp32,
+ * all device memory, 16-byte aligned; K a multiple of 64.  bn (16, 32, 64 or 128: output tile width)
+ * and ks (1..8: K split over a cluster of ks CTAs, partials added in a fixed order) force a plan;
+ * bn = ks = 0 takes the plan the library would choose for a batch-sized N.  The profiling hook
+ * (domino_debug_set_trace) also receives this kernel's per-CTA stamps when its buffer holds
+ * 16 entries per CTA.  Returns DOMINO_OK, DOMINO_ERR_INVALID_ARGUMENT, DOMINO_ERR_UNSUPPORTED or
+ * DOMINO_ERR_CUDA (e.g. a forced cluster that cannot launch). */
+DOMINO_API int domino_debug_gemm(const void* A, const void* B, int32_t M, int32_t N, int32_t K, int32_t a_kwrap,
+                                 float* out, int64_t ldo, int32_t trans, int32_t bn, int32_t ks,
+                                 int32_t* status_dev, domino_stream_t stream);
 
 /* Test hook: iteration limit of the library's bounded device-wide waits (0 restores the
  * default, about one second).  A tiny limit makes waits give up early, which exercises the

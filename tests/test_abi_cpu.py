@@ -108,3 +108,29 @@ def test_invalid_arguments_are_rejected_before_any_launch(L):
                                None) == domino.ERR_INVALID_ARGUMENT
     assert L.domino_accept_len(i32(1), i32(16), i32(151936), fake, fake, fake, fake, 16, None,
                                None) == domino.ERR_WORKSPACE
+
+
+def test_arena_host_logic(L):
+    sh = _shape()
+    n = L.domino_arena_bytes(ctypes.byref(sh))
+    # W2, W1, W_hh, W_ih, b_ih, b_hh at the 8B shapes, bf16, each region rounded up to 256 bytes
+    parts = [151936 * 256, 256 * (4096 + 1024), 3072 * 1024, 3072 * 4096, 3072, 3072]
+    assert n == sum((2 * p + 255) // 256 * 256 for p in parts)
+    assert L.domino_arena_bytes(ctypes.byref(_shape(V=999))) == 0
+    w = domino.Weights(*([0x10000] * 7))
+    out = domino.Weights()
+    fake = ctypes.c_void_p(0x100000)
+    # arena missing, misaligned or too small: rejected before any copy
+    assert L.domino_pack_weights(ctypes.byref(sh), ctypes.byref(w), None, n, ctypes.byref(out),
+                                 None) == domino.ERR_WORKSPACE
+    assert L.domino_pack_weights(ctypes.byref(sh), ctypes.byref(w), ctypes.c_void_p(0x100010), n,
+                                 ctypes.byref(out), None) == domino.ERR_WORKSPACE
+    assert L.domino_pack_weights(ctypes.byref(sh), ctypes.byref(w), fake, n - 256, ctypes.byref(out),
+                                 None) == domino.ERR_WORKSPACE
+    assert L.domino_pack_weights(ctypes.byref(sh), ctypes.byref(w), fake, n, None,
+                                 None) == domino.ERR_INVALID_ARGUMENT
+    # persistence: the legacy default stream and out-of-range ratios are refused on the host
+    assert L.domino_set_l2_persistence(ctypes.byref(sh), ctypes.byref(w), None,
+                                       ctypes.c_float(1.0)) == domino.ERR_INVALID_ARGUMENT
+    assert L.domino_set_l2_persistence(ctypes.byref(sh), ctypes.byref(w), ctypes.c_void_p(0x1000),
+                                       ctypes.c_float(1.5)) == domino.ERR_INVALID_ARGUMENT

@@ -218,6 +218,46 @@ def time_steps(pt: Point, steps: int, warmup: int, flush, stream, dist=None):
     return step, greedy, launches
 
 
+def time_steps_persisting(pt: Point, steps: int, warmup: int, flush, stream):
+    """time_steps with the weights packed into one arena and an L2 persisting window over it on
+    `stream` (the warm regime: L2 is still flushed before every step, but the window's lines are
+    kept).  The window is cleared and the set-aside restored afterwards.  None when the device has
+    no persisting L2."""
+    domino = pt.domino
+    w0 = pt.w
+    try:
+        pt.w = domino.pack_weights(w0, stream=stream)
+        stream.synchronize()
+        domino.set_l2_persistence(pt.w, stream, 1.0)
+    except domino.DominoError:
+        pt.w = w0
+        return None
+    try:
+        return time_steps(pt, steps, warmup, flush, stream)
+    finally:
+        domino.set_l2_persistence(pt.w, stream, 0.0)
+        pt.torch.cuda.synchronize()
+        pt.w = w0
+
+
+def w2_kernel_us(pt: Point, flush, stream) -> float:
+    """Device time of the last position's W2 argmax GEMM in one greedy call, from the GEMM's own
+    stamps: latest CTA end minus the earliest moment a CTA's wait on the previous grid returned."""
+    torch, domino = pt.torch, pt.domino
+    buf = torch.zeros(148 * 16, dtype=torch.int64, device=pt.lb.device)
+    flush.zero_()
+    torch.cuda.synchronize()
+    domino.set_trace(buf)
+    try:
+        pt.greedy(stream)
+        torch.cuda.synchronize()
+    finally:
+        domino.set_trace(None)
+    t = buf.view(-1, 16).cpu().numpy()
+    t = t[(t[:, 1] != 0) & (t[:, 15] != 0)]
+    return float((t[:, 1].max() - t[:, 15].min()) / 1e3)
+
+
 def time_e2e(pt: Point, steps: int, warmup: int, flush, stream):
     """Same step through the public API from pinned host buffers: each step copies its inputs
     host->device and reads the tokens and accept lengths back, all inside the timed region."""
@@ -346,6 +386,16 @@ def run_ours(args):
                          "algorithmic_bytes": vb},
             "note": "GRU input half gathered from embed . W_ih^T (prepared once per weight set, untimed)",
         }
+        warm = time_steps_persisting(pt, args.steps, args.warmup, flush, stream)
+        if warm is not None:
+            w_step, w_greedy, _ = warm
+            variants["l2_persisting"] = {
+                "blocks_per_s": round(B * len(w_step) / (sum(w_step) * 1e-3), 2),
+                "us_per_block": round(1e3 * statistics.mean(w_step) / B, 3),
+                "greedy_ms": round(statistics.mean(w_greedy), 4),
+                "note": "warm regime: weights packed into one arena under an L2 persisting access-policy "
+                        "window (domino_set_l2_persistence); L2 still flushed before every step",
+            }
         points = {}
         if not args.no_points:
             del pt
@@ -357,6 +407,8 @@ def run_ours(args):
                 psh = p.sh
                 ga = statistics.mean(g_ms)
                 fl = greedy_flops(psh)
+                w2_us = w2_kernel_us(p, flush, stream)
+                w2_flops = 2.0 * psh["B"] * psh["V"] * psh["r"]
                 points[str(pb)] = {
                     "blocks_per_s": round(pb * len(s_ms) / (sum(s_ms) * 1e-3), 1),
                     "us_per_block": round(1e3 * statistics.mean(s_ms) / pb, 3),
@@ -365,7 +417,14 @@ def run_ours(args):
                     "hbm_frac": round(greedy_bytes(psh) / (ga * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
                     "tensor_frac": round(fl / (ga * 1e-3) / 1e12 / peaks["bf16_tflops"], 4),
                     "greedy_tflops": round(fl / (ga * 1e-3) / 1e12, 2),
+                    "w2_argmax_gemm": {"us": round(w2_us, 2), "tflops": round(w2_flops / (w2_us * 1e-6) / 1e12, 1),
+                                       "tensor_frac": round(w2_flops / (w2_us * 1e-6) / 1e12 / peaks["bf16_tflops"], 4),
+                                       "note": "last position's W2 GEMM with fused argmax, one launch, from its "
+                                               "own device clock stamps"},
                 }
+                warm = time_steps_persisting(p, max(3, args.steps // 2), args.warmup, flush, stream)
+                if warm is not None:
+                    points[str(pb)]["l2_persisting_blocks_per_s"] = round(pb * len(warm[0]) / (sum(warm[0]) * 1e-3), 1)
                 del p
                 torch.cuda.empty_cache()
         cpu = None if args.no_cpu_baseline else cpu_baseline(args.cpu_seconds)

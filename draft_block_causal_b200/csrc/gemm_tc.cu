@@ -109,28 +109,25 @@ struct EpiLogits {  // logits[n][m] = D + Lb[n][m]   (m = vocabulary row, n = (r
 };
 
 // Greedy step, batch-major: m = batch row b (< M), n = vocabulary row v.
-//   z = D + Lb[b][v] (Lb row stride ldl), running argmax over the thread's columns in four
-//   independent chains (column j of a 16-column group goes to chain j % 4; each chain visits its
-//   columns in ascending order and strict > keeps its lowest index), finish: keys[b] = max(keys[b],
-//   max over chains of key(best)) -- the key orders by value, then lowest index, so the chains
-//   combine to the row's lowest-index maximum.  When out is set, z is also stored to
+//   z = D + Lb[b][v] (Lb row stride ldl); per 16-column group the maximum (a tree of 15 max
+//   operations) is compared with the running best, and only a group that beats it (strict >, so
+//   the earliest group wins ties) is searched for the lowest column holding its maximum -- after
+//   the first groups that is rare, so the common cost is an add and a max per element.
+//   finish: keys[b] = max(keys[b], key(best)).  When out is set, z is also stored to
 //   out[b * ldo + v].
 template <bool ARES>
 struct EpiArgmaxT {
   static constexpr bool kSide = true;  // the L_base tile [128 rows b x BN columns v]
   static constexpr bool kARes = ARES;  // the activation band is loaded once per CTA
   struct State {
-    float best[4];
-    int idx[4];
+    float best;
+    int idx;
   };
   uint64_t* keys;
   int M;
   float* out;
   long long ldo;
-  __device__ __forceinline__ void init(State& s) const {
-#pragma unroll
-    for (int c = 0; c < 4; ++c) { s.best[c] = -INFINITY; s.idx[c] = -1; }
-  }
+  __device__ __forceinline__ void init(State& s) const { s.best = -INFINITY; s.idx = -1; }
   __device__ __forceinline__ void apply(State& s, int m, int n0, const float (&v)[16], int N, const uint8_t* side,
                                         int row, int c0) const {
     if (m >= M) return;
@@ -144,9 +141,23 @@ struct EpiArgmaxT {
     for (int j = 0; j < 8; ++j) l[8 + j] = a[j];
     float z[16];
 #pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      z[j] = v[j] + l[j];
-      if (n0 + j < N && z[j] > s.best[j & 3]) { s.best[j & 3] = z[j]; s.idx[j & 3] = n0 + j; }
+    for (int j = 0; j < 16; ++j) z[j] = v[j] + l[j];
+    float zm[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) zm[j] = (n0 + 16 <= N || n0 + j < N) ? z[j] : -INFINITY;  // ragged last tile
+    float t8[8], t4[4];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) t8[j] = fmaxf(zm[j], zm[j + 8]);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) t4[j] = fmaxf(t8[j], t8[j + 4]);
+    const float mx = fmaxf(fmaxf(t4[0], t4[2]), fmaxf(t4[1], t4[3]));
+    if (mx > s.best) {  // the lowest column of this group holding its maximum
+      int jj = 15;
+#pragma unroll
+      for (int j = 15; j >= 0; --j)
+        if (zm[j] == mx) jj = j;
+      s.best = mx;
+      s.idx = n0 + jj;
     }
     if (out) {
       if (n0 + 16 <= N) {
@@ -159,11 +170,8 @@ struct EpiArgmaxT {
     }
   }
   __device__ __forceinline__ void finish(State& s, int m) const {
-    uint64_t key = 0;
-#pragma unroll
-    for (int c = 0; c < 4; ++c)
-      if (s.idx[c] >= 0) key = umax64(key, argmax_key(s.best[c], s.idx[c]));
-    if (m < M && key) atomicMax(reinterpret_cast<unsigned long long*>(keys + m), (unsigned long long)key);
+    if (m < M && s.idx >= 0)
+      atomicMax(reinterpret_cast<unsigned long long*>(keys + m), (unsigned long long)argmax_key(s.best, s.idx));
   }
 };
 
@@ -231,7 +239,8 @@ struct EpiSiluU {
 // globaltimer at start/end; 2 clock at start, 3 setup done, 4 first stage ready (MMA), 5 last
 // accumulator committed (MMA), 6 first accumulator received (epilogue), 7 epilogue work done, 8
 // cluster barrier passed, 9 split reduction done, 10 end, 11 last load issued (producer), 12 items,
-// 13 first item's epilogue done, 14 first item's accumulator committed (MMA).
+// 13 first item's epilogue done, 14 first item's accumulator committed (MMA), 15 globaltimer when
+// the producer's wait for the previous grid returned.
 constexpr int kTraceSlots = 16;
 __device__ __forceinline__ void stamp(unsigned long long* trace, int k, unsigned long long v) {
   if (trace) trace[blockIdx.x * kTraceSlots + k] = v;
@@ -379,6 +388,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
       }
       pdl_wait();
+      stamp(trace, 15, globaltimer_ns());
       if constexpr (Epi::kARes) {  // A once: all of K for the single 128-row band
         mbar_arrive_expect_tx(a_full, (uint32_t)kblocks * kABytes);
         for (int kb = 0; kb < kblocks; ++kb) tma_load_2d(ares + kb * kABytes, &tmA, a_full, kb * kBK, 0);
@@ -391,6 +401,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const bool second = a_split && m0 >= a_split;
         const CUtensorMap* ta = second ? &tmA2 : &tmA;
         const int ay = second ? m0 - a_split : m0;
+        if constexpr (Epi::kSide || Epi::kARes) {
+          // streamed operands two tiles ahead into L2, so that the stage and side loads of that tile
+          // meet L2 latency rather than HBM latency
+          const int ta2i = t + 2 * (int)gridDim.x;
+          if (ta2i < items) {
+            const int tile2 = ta2i / ksplit;
+            const int m2 = (tile2 / n_tiles) * kBM, n2 = (tile2 % n_tiles) * BN;
+            if constexpr (Epi::kARes)
+              for (int kb = 0; kb < kblocks; ++kb) tma_prefetch_l2(&tmB, kb * kBK, n2);
+            if constexpr (Epi::kSide)
+              for (int bx = 0; bx < BN / 64; ++bx) tma_prefetch_l2(&tmS, n2 + bx * 64, m2);
+          }
+        }
         for (int kb = kb0; kb < kb1; kb += C::kKBS, ++it) {
           const int s = it % S;
           const uint32_t ph = (it / S) & 1u;

@@ -380,9 +380,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           const int kb0 = piece * kblocks / ksplit, kb1 = (piece + 1) * kblocks / ksplit;
           const bool second = a_split && m0 >= a_split;
           for (int kb = kb0; kb < kb1; ++kb, ++boxes) {
-            if ((indep & 1) && !Epi::kARes)
-              tma_prefetch_l2(second ? &tmA2 : &tmA, a_kwrap ? (kb * kBK) % a_kwrap : kb * kBK,
-                              second ? m0 - a_split : m0);
+            if ((indep & 1) && !Epi::kARes) {
+              const CUtensorMap* pa = second ? &tmA2 : &tmA;
+              const int px = a_kwrap ? (kb * kBK) % a_kwrap : kb * kBK, py = second ? m0 - a_split : m0;
+              if (a_stream)  // the same eviction priority as the load that will use it
+                tma_prefetch_l2_hint(pa, px, py, pol_first);
+              else
+                tma_prefetch_l2(pa, px, py);
+            }
             if (indep & 2) tma_prefetch_l2(&tmB, kb * kBK, n0);
           }
         }
@@ -411,7 +416,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             if constexpr (Epi::kARes)
               for (int kb = 0; kb < kblocks; ++kb) tma_prefetch_l2(&tmB, kb * kBK, n2);
             if constexpr (Epi::kSide)
-              for (int bx = 0; bx < BN / 64; ++bx) tma_prefetch_l2(&tmS, n2 + bx * 64, m2);
+              for (int bx = 0; bx < BN / 64; ++bx) tma_prefetch_l2_hint(&tmS, n2 + bx * 64, m2, pol_first);
           }
         }
         for (int kb = kb0; kb < kb1; kb += C::kKBS, ++it) {

@@ -74,6 +74,13 @@ __device__ __forceinline__ void tma_prefetch_l2(const CUtensorMap* tmap, int x, 
                : "memory");
 }
 
+// tma_prefetch_l2 with an L2 cache-policy operand.
+__device__ __forceinline__ void tma_prefetch_l2_hint(const CUtensorMap* tmap, int x, int y, uint64_t policy) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile.L2::cache_hint [%0, {%1, %2}], %3;" ::"l"(tmap),
+               "r"(x), "r"(y), "l"(policy)
+               : "memory");
+}
+
 // L2 policy that marks the lines a load brings in as the first to evict (streamed operands that are
 // read once, so that they do not push re-read weights out of L2).
 __device__ __forceinline__ uint64_t l2_policy_evict_first() {

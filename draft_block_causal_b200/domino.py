@@ -37,7 +37,8 @@ EXPORTS = ("domino_workspace_bytes", "domino_draft_greedy", "domino_teacher_forc
            "domino_abi_version", "domino_debug_set_spin_limit", "domino_launch_count",
            "domino_greedy_plan", "domino_draft_greedy_noalloc", "domino_debug_set_trace",
            "domino_embed_proj_bytes", "domino_project_embeddings", "domino_arena_bytes",
-           "domino_pack_weights", "domino_set_l2_persistence", "domino_debug_gemm")
+           "domino_pack_weights", "domino_set_l2_persistence", "domino_debug_gemm",
+           "domino_debug_read_passes")
 
 
 class DominoError(RuntimeError):
@@ -105,6 +106,8 @@ def lib(path: str = LIB_PATH) -> ctypes.CDLL:
         L.domino_set_l2_persistence.restype = ctypes.c_int
         L.domino_debug_gemm.argtypes = [vp, vp, i32, i32, i32, i32, vp, ctypes.c_int64, i32, i32, i32, vp, vp]
         L.domino_debug_gemm.restype = ctypes.c_int
+        L.domino_debug_read_passes.argtypes = [vp, sz, i32, vp]
+        L.domino_debug_read_passes.restype = ctypes.c_int
         _lib = L
     return _lib
 
@@ -270,6 +273,12 @@ def debug_gemm(A, B, out=None, trans=False, a_kwrap=0, bn=0, ks=0, status=None, 
                                  int(bn), int(ks), _ptr(status), _stream(stream))
     _check(rc, "domino_debug_gemm")
     return out
+
+
+def debug_read_passes(buf, passes: int, stream=None) -> None:
+    """Re-read a device buffer `passes` times in one launch (domino_debug_read_passes)."""
+    rc = lib().domino_debug_read_passes(_ptr(buf), buf.numel() * buf.element_size(), int(passes), _stream(stream))
+    _check(rc, "domino_debug_read_passes")
 
 
 def accept_workspace_bytes(B: int, L: int) -> int:

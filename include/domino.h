@@ -261,6 +261,13 @@ DOMINO_API int domino_debug_gemm(const void* A, const void* B, int32_t M, int32_
                                  float* out, int64_t ldo, int32_t trans, int32_t bn, int32_t ks,
                                  int32_t* status_dev, domino_stream_t stream);
 
+/* Measurement aid: one launch in which each of one CTA per SM re-reads its contiguous slice of
+ * `buf` (device memory, 16-byte aligned, `bytes` long) `passes` times (1..1000) with 16-byte
+ * read-only loads, the access pattern of the fused kernel's W2 pass.  Timing 1 and n passes of a
+ * buffer that fits L2 gives the L2 re-read bandwidth used for the reuse-aware roofline.  Returns
+ * DOMINO_OK, DOMINO_ERR_INVALID_ARGUMENT or DOMINO_ERR_CUDA. */
+DOMINO_API int domino_debug_read_passes(const void* buf, size_t bytes, int32_t passes, domino_stream_t stream);
+
 /* Test hook: iteration limit of the library's bounded device-wide waits (0 restores the
  * default, about one second).  A tiny limit makes waits give up early, which exercises the
  * DOMINO_STATUS_DEVICE_TIMEOUT path without faulting or hanging the GPU.  Process-wide; takes

@@ -134,3 +134,10 @@ def test_arena_host_logic(L):
                                        ctypes.c_float(1.0)) == domino.ERR_INVALID_ARGUMENT
     assert L.domino_set_l2_persistence(ctypes.byref(sh), ctypes.byref(w), ctypes.c_void_p(0x1000),
                                        ctypes.c_float(1.5)) == domino.ERR_INVALID_ARGUMENT
+
+
+def test_read_passes_argument_checks(L):
+    assert L.domino_debug_read_passes(None, 1 << 20, 1, None) == domino.ERR_INVALID_ARGUMENT
+    assert L.domino_debug_read_passes(ctypes.c_void_p(0x10004), 1 << 20, 1, None) == domino.ERR_INVALID_ARGUMENT
+    assert L.domino_debug_read_passes(ctypes.c_void_p(0x10000), 1 << 20, 0, None) == domino.ERR_INVALID_ARGUMENT
+    assert L.domino_debug_read_passes(ctypes.c_void_p(0x10000), 8, 1, None) == domino.ERR_INVALID_ARGUMENT

@@ -71,3 +71,11 @@ def test_invalid_plans_are_refused_on_the_host():
     for bn, ks in ((48, 1), (16, 9), (0, 2), (128, 0)):
         with pytest.raises(domino.DominoError):
             domino.debug_gemm(A, B, bn=bn, ks=ks)
+
+
+def test_read_passes_runs_and_counts_one_launch():
+    buf = torch.ones(1 << 22, dtype=torch.uint8, device="cuda")
+    n0 = domino.launch_count()
+    domino.debug_read_passes(buf, 3)
+    torch.cuda.synchronize()
+    assert domino.launch_count() == n0 + 1

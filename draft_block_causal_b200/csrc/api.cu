@@ -99,7 +99,8 @@ Workspace layout_workspace(const Shape& s, void* base) {
   const size_t BL = (size_t)s.B * s.L;
   w.status = reinterpret_cast<int32_t*>(take(sizeof(int32_t)));
   w.sync = reinterpret_cast<uint32_t*>(take(kSyncWords * sizeof(uint32_t)));
-  // sync, keys and a_acc are adjacent so that one memset clears all three
+  // sync, claim, keys and a_acc are adjacent so that one memset clears them together
+  w.claim = reinterpret_cast<uint32_t*>(take(kClaimWords * sizeof(uint32_t)));
   w.keys = reinterpret_cast<uint64_t*>(take(BL * sizeof(uint64_t)));
   w.a_acc = reinterpret_cast<float*>(take(BL * s.r * kAccReplicas * sizeof(float)));
   w.acc_keys = reinterpret_cast<uint64_t*>(take(BL * sizeof(uint64_t)));
@@ -274,7 +275,8 @@ int domino_draft_greedy(const domino_shape_t* shape, const domino_weights_t* w, 
                   gemm_tc_supported((int)BL, s.r, s.d, hidden, w->W1) &&
                   gemm_tc_supported(s.B, s.V, s.r, ws.u16, w->W2);
   const bool tc_gru = tc && s.Hs % 64 == 0;
-  cudaError_t e = cudaMemsetAsync(ws.keys, 0, BL * sizeof(uint64_t), cs);
+  // work-slot claims and argmax keys are adjacent: one memset clears both
+  cudaError_t e = cudaMemsetAsync(ws.claim, 0, (char*)(ws.keys + BL) - (char*)ws.claim, cs);
   if (e == cudaSuccess) {
     if (tc)  // P[n][k] = sum_c H[n][c] W1[k][c]: H [B*L x d], the first d columns of W1 (row stride d + Hs)
       e = gemm_tc_store_f32_bn64((const __nv_bfloat16*)hidden, (const __nv_bfloat16*)w->W1, (int)BL, s.r, s.d,
@@ -302,10 +304,12 @@ int domino_draft_greedy(const domino_shape_t* shape, const domino_weights_t* w, 
     if (e == cudaSuccess && tc) {
       for (int b0 = 0; b0 < s.B && e == cudaSuccess; b0 += 128) {  // bands of <= 128 batch rows
         const size_t row0 = (size_t)b0 * s.L + i;                   // (row b0, position i)
+        // epochs distinct per launch of this call (the claims were zeroed above)
+        const uint32_t epoch = (uint32_t)(i * ((s.B + 127) / 128) + b0 / 128 + 1);
         e = gemm_tc_argmax(ws.u16 + (size_t)b0 * s.r, (const bf*)w->W2, std::min(128, s.B - b0), s.V, s.r,
                            (const bf*)base_logits + row0 * s.V, (long long)s.L * s.V, ws.keys + (size_t)i * s.B + b0,
                            logits_out ? logits_out + row0 * s.V : nullptr, (long long)s.L * s.V, st, spin_limit(),
-                           cs);
+                           cs, ws.claim, epoch);
       }
     } else if (e == cudaSuccess) {
       e = launch_w2(s, w->W2, ws.u, s.B, base_logits, s.L, i, ws.keys + (size_t)i * s.B, logits_out, cs);

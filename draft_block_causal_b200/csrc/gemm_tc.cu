@@ -39,7 +39,13 @@ namespace domino {
 namespace {
 
 constexpr int kBM = 128, kBK = 64;
-constexpr int kGemmThreads = 192;
+// Warps 0 and 1 produce and issue; 4 * kGroups epilogue warps follow (two warps per TMEM lane
+// quadrant, each on half of the tile's columns, for the argmax epilogue whose per-tile work is the
+// longest; one per quadrant otherwise).
+template <class Epi> struct EpiWarps {
+  static constexpr int kGroups = Epi::kSide ? 2 : 1;
+  static constexpr int kThreads = 64 + 128 * kGroups;
+};
 constexpr uint32_t kABytes = kBM * kBK * 2;
 
 // ---- epilogues ----
@@ -275,6 +281,53 @@ __device__ __forceinline__ void st_cluster_f4(uint32_t addr, float a, float b, f
                : "memory");
 }
 
+// ---- SM affinity of work slots ----
+// A persistent launch with one CTA per SM walks the tiles t = slot, slot + grid, ...  Choosing the
+// slot from the SM the CTA runs on (rather than from blockIdx) gives every tile the same SM at
+// every launch, so that its operand lines stay in the L2 partition next to that SM across
+// launches.  g_sm_rank maps %smid to a dense rank (filled once per device by k_sm_probe /
+// k_sm_rank); each launch claims slots with atomicExch against a per-launch epoch, so that every
+// slot is taken exactly once even when the scheduler places two CTAs on one SM.
+constexpr int kMaxSmid = 1024;
+__device__ int g_sm_of_cta[kMaxSmid];
+__device__ int g_sm_rank[kMaxSmid];
+
+__device__ __forceinline__ unsigned sm_id() {
+  unsigned s;
+  asm volatile("mov.u32 %0, %%smid;" : "=r"(s));
+  return s;
+}
+// Launched with more than half an SM's shared memory (unused): one CTA per SM.
+__global__ void k_sm_probe(int n) {
+  if (threadIdx.x == 0 && blockIdx.x < (unsigned)n) g_sm_of_cta[blockIdx.x] = (int)sm_id();
+}
+__global__ void k_sm_rank(int n) {  // one thread: dense rank of each recorded smid
+  if (threadIdx.x != 0 || blockIdx.x != 0) return;
+  for (int s = 0; s < kMaxSmid; ++s) g_sm_rank[s] = -1;
+  for (int i = 0; i < n; ++i) {
+    const int s = g_sm_of_cta[i];
+    if (s >= 0 && s < kMaxSmid) g_sm_rank[s] = 0;  // present
+  }
+  int r = 0;
+  for (int s = 0; s < kMaxSmid; ++s)
+    if (g_sm_rank[s] == 0) g_sm_rank[s] = ++r;
+  for (int s = 0; s < kMaxSmid; ++s)
+    if (g_sm_rank[s] > 0) --g_sm_rank[s];  // ranks 0 .. r-1
+}
+// Work slot of this CTA (thread 0 only).  claim == null: blockIdx.x.
+__device__ int claim_slot(uint32_t* claim, uint32_t epoch) {
+  if (!claim) return (int)blockIdx.x;
+  const int G = (int)gridDim.x;
+  const unsigned s = sm_id();
+  const int pref = s < (unsigned)kMaxSmid ? g_sm_rank[s] : -1;
+  if (pref >= 0 && pref < G && atomicExch(claim + pref, epoch) != epoch) return pref;
+  for (int k = 0; k < G; ++k) {  // taken (or no rank): the next free slot
+    const int c = ((int)blockIdx.x + k) % G;
+    if (atomicExch(claim + c, epoch) != epoch) return c;
+  }
+  return (int)blockIdx.x;  // unreachable: G CTAs, G slots
+}
+
 // Shared memory (from a 1024-aligned base): [resident A][stage ring][1024 B: mbarriers, TMEM slot]
 // [two side tiles][split-K receive buffer], plus 1024 bytes of slack for the alignment.  With a
 // resident A (K <= 256, one 128-row band of M) each stage carries two k-blocks of B; otherwise one
@@ -297,11 +350,12 @@ template <int BN, bool SIDE, bool ARES, bool SPLIT = false> struct Cfg {
 };
 
 template <int BN, class Epi, bool SPLIT>
-__global__ void __launch_bounds__(kGemmThreads, 1)
+__global__ void __launch_bounds__(EpiWarps<Epi>::kThreads, 1)
     k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmA2,
               const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmS, int M, int N, int K,
               Epi epi, int32_t* status, unsigned long long limit, int a_kwrap, int a_split, int ksplit,
-              int a_stream, int indep, unsigned long long* __restrict__ trace) {
+              int a_stream, int indep, uint32_t* __restrict__ claim, uint32_t epoch,
+              unsigned long long* __restrict__ trace) {
   static_assert(!SPLIT || (!Epi::kSide && !Epi::kARes), "split-K needs a plain epilogue");
   using C = Cfg<BN, Epi::kSide, Epi::kARes, SPLIT>;
   constexpr int S = C::kStages;
@@ -318,6 +372,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint64_t* a_full = sidee + 2;    // resident A landed
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(a_full + 1);
   volatile int* abort_s = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* slot_s = reinterpret_cast<volatile int*>(tmem_slot + 2);
   // after the barriers (1024 bytes) and the two side tiles: the split-K receive buffer
   uint8_t* const recv_buf = smem + (size_t)S * C::kStage + 1024 + 2 * C::kSideBytes;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -332,14 +387,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
-    for (int a = 0; a < 2; ++a) { mbar_init(&accf[a], 1); mbar_init(&acce[a], 4); }
+    for (int a = 0; a < 2; ++a) { mbar_init(&accf[a], 1); mbar_init(&acce[a], 4 * EpiWarps<Epi>::kGroups); }
     mbar_init(mma_done, 1);
     mbar_init(&sidef[0], 1);
     mbar_init(&sidef[1], 1);
-    mbar_init(&sidee[0], 4);
-    mbar_init(&sidee[1], 4);
+    mbar_init(&sidee[0], 4 * EpiWarps<Epi>::kGroups);
+    mbar_init(&sidee[1], 4 * EpiWarps<Epi>::kGroups);
     mbar_init(a_full, 1);
     *abort_s = 0;
+    *slot_s = claim_slot(claim, epoch);
     mbar_fence_init();
     tma_prefetch_desc(&tmA);
     if (a_split) tma_prefetch_desc(&tmA2);
@@ -354,6 +410,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   __syncthreads();
   tmem_fence_after_sync();
   const uint32_t tbase = *tmem_slot;
+  const int slot = *slot_s;  // this CTA's first work item (blockIdx.x unless SM-affine)
   if (threadIdx.x == 0) {
     stamp(trace, 3, clk());
     pdl_trigger();  // the next kernel on the stream may be scheduled (it waits for this grid to finish)
@@ -374,7 +431,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       // operands no earlier kernel writes (indep: bit 0 A, bit 1 B) into L2.
       if (indep) {
         int boxes = 0;
-        for (int t = blockIdx.x; t < items && boxes < 64; t += gridDim.x) {
+        for (int t = slot; t < items && boxes < 64; t += gridDim.x) {
           const int tile = t / ksplit, piece = t - tile * ksplit;
           const int m0 = (tile / n_tiles) * kBM, n0 = (tile % n_tiles) * BN;
           const int kb0 = piece * kblocks / ksplit, kb1 = (piece + 1) * kblocks / ksplit;
@@ -398,7 +455,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         mbar_arrive_expect_tx(a_full, (uint32_t)kblocks * kABytes);
         for (int kb = 0; kb < kblocks; ++kb) tma_load_2d(ares + kb * kABytes, &tmA, a_full, kb * kBK, 0);
       }
-      for (int t = blockIdx.x; t < items && ok; t += gridDim.x) {
+      for (int t = slot; t < items && ok; t += gridDim.x) {
         const int tile = t / ksplit, piece = t - tile * ksplit;
         const int m0 = (tile / n_tiles) * kBM, n0 = (tile % n_tiles) * BN;
         const int kb0 = piece * kblocks / ksplit, kb1 = (piece + 1) * kblocks / ksplit;
@@ -453,7 +510,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       uint32_t it = 0, acc_it = 0;
       bool ok = true;
       if constexpr (Epi::kARes) ok = mbar_wait_bounded(a_full, 0u, limit, abort_s);
-      for (int t = blockIdx.x; t < items && ok; t += gridDim.x, ++acc_it) {
+      for (int t = slot; t < items && ok; t += gridDim.x, ++acc_it) {
         const uint32_t a = acc_it & 1u, aph = (acc_it >> 1) & 1u;
         if (!mbar_wait_bounded(&acce[a], aph ^ 1u, limit, abort_s)) { ok = false; break; }
         tmem_fence_after_sync();
@@ -489,9 +546,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       umma_commit(mma_done);
       mbar_wait_bounded(mma_done, 0u, limit, &never);
     }
-  } else {  // ---- epilogue: warps 2..5 ----
+  } else {  // ---- epilogue: warps 2 .. 2 + 4 * kGroups - 1 ----
     pdl_wait();
-    const int q = warp & 3;
+    const int q = warp & 3;  // TMEM lane quadrant this warp may read
+    constexpr int G = EpiWarps<Epi>::kGroups, CW = BN / G;  // columns per epilogue group
+    const int cb = ((warp - 2) >> 2) * CW;                   // this warp's first column
     uint32_t acc_it = 0;
     typename Epi::State est;
     epi.init(est);
@@ -514,10 +573,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       return true;
     };
     uint32_t side_issued = 0;  // loads issued (meaningful in the issuing thread)
-    if (Epi::kSide && (int)blockIdx.x < tiles && side_issuer) {
-      if (side_load(0u, blockIdx.x)) side_issued = 1; else *abort_s = 1;
+    if (Epi::kSide && slot < tiles && side_issuer) {
+      if (side_load(0u, slot)) side_issued = 1; else *abort_s = 1;
     }
-    for (int t = blockIdx.x; t < items; t += gridDim.x, ++acc_it) {
+    for (int t = slot; t < items; t += gridDim.x, ++acc_it) {
       const uint32_t a = acc_it & 1u, aph = (acc_it >> 1) & 1u;
       if (Epi::kSide && t + (int)gridDim.x < tiles && side_issuer) {  // prefetch the next tile's side operand
         if (side_load(acc_it + 1u, t + gridDim.x)) ++side_issued; else *abort_s = 1;
@@ -563,12 +622,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         continue;
       }
       m_last = m;
-      // Software pipeline over 32-column steps: the next step's TMEM loads are in flight while this
-      // step is processed; one wait per step (it covers the loads issued just before).
-      constexpr int kStep = BN >= 32 ? 32 : 16, kSteps = BN / kStep;
+      // Software pipeline over 32-column steps of this warp's CW columns: the next step's TMEM
+      // loads are in flight while this step is processed; one wait per step (it covers the loads
+      // issued just before).
+      constexpr int kStep = CW >= 32 ? 32 : 16, kSteps = CW / kStep;
       uint32_t r[2][kStep];
-      tmem_ld16(taddr, &r[0][0]);
-      if (kStep == 32) tmem_ld16(taddr + 16, &r[0][16]);
+      tmem_ld16(taddr + cb, &r[0][0]);
+      if (kStep == 32) tmem_ld16(taddr + cb + 16, &r[0][16]);
       tmem_wait_ld();
 #pragma unroll
       for (int k = 0; k < kSteps; ++k) {
@@ -576,15 +636,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
         for (int j = 0; j < kStep; ++j) reg_fence(cur[j]);
         if (k + 1 < kSteps) {
-          tmem_ld16(taddr + (k + 1) * kStep, &r[(k + 1) & 1][0]);
-          if (kStep == 32) tmem_ld16(taddr + (k + 1) * kStep + 16, &r[(k + 1) & 1][16]);
+          tmem_ld16(taddr + cb + (k + 1) * kStep, &r[(k + 1) & 1][0]);
+          if (kStep == 32) tmem_ld16(taddr + cb + (k + 1) * kStep + 16, &r[(k + 1) & 1][16]);
         }
 #pragma unroll
         for (int h = 0; h < kStep / 16; ++h) {
           float v[16];
 #pragma unroll
           for (int j = 0; j < 16; ++j) v[j] = __uint_as_float(cur[16 * h + j]);
-          epi.apply(est, m, n0 + k * kStep + 16 * h, v, N, side, row, k * kStep + 16 * h);
+          const int c = cb + k * kStep + 16 * h;
+          epi.apply(est, m, n0 + c, v, N, side, row, c);
         }
         if (k + 1 < kSteps) tmem_wait_ld();
       }
@@ -626,7 +687,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const uint8_t* recv = recv_buf;
       typename Epi::State est;
       epi.init(est);
-      for (int li = (int)threadIdx.x - 64; li < u1 - u0; li += 128) {
+      for (int li = (int)threadIdx.x - 64; li < u1 - u0; li += 128 * EpiWarps<Epi>::kGroups) {
         const int u = u0 + li, g = u / kBM, row = u - g * kBM;
         float v[16];
 #pragma unroll
@@ -694,6 +755,24 @@ int sm_count() {
   return n;
 }
 
+// Fills g_sm_rank once per device (two small launches on `st`, no host synchronisation).
+cudaError_t ensure_sm_rank(cudaStream_t st) {
+  static std::atomic<uint64_t> done{0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const uint64_t bit = dev < 64 ? (1ull << dev) : 0;
+  if (bit && (done.load(std::memory_order_acquire) & bit)) return cudaSuccess;
+  const int n = std::min(sm_count(), kMaxSmid);
+  const int hold = 120 * 1024;  // more than half an SM's shared memory: one CTA per SM
+  cudaError_t e = cudaFuncSetAttribute(k_sm_probe, cudaFuncAttributeMaxDynamicSharedMemorySize, hold);
+  if (e != cudaSuccess) return e;
+  k_sm_probe<<<n, 32, hold, st>>>(n);
+  k_sm_rank<<<1, 32, 0, st>>>(n);
+  e = cudaGetLastError();
+  if (e == cudaSuccess && bit) done.fetch_or(bit, std::memory_order_acq_rel);
+  return e;
+}
+
 // The kernel's dynamic shared memory opt-in, set once per device.
 template <int BN, class Epi, bool SPLIT>
 cudaError_t set_smem_once(size_t smem) {
@@ -711,7 +790,8 @@ template <int BN, class Epi>
 cudaError_t launch_gemm(const void* A, const void* Bm, int M, int N, int K, const Epi& epi, int32_t* status,
                         uint64_t limit, cudaStream_t st, uint64_t lda = 0, uint64_t ldb = 0, int a_kwrap = 0,
                         const void* side = nullptr, uint64_t lds = 0, const void* A2 = nullptr, int a_split = 0,
-                        uint64_t lda2 = 0, int ksplit = 1, int a_stream = 0, int indep = 0) {
+                        uint64_t lda2 = 0, int ksplit = 1, int a_stream = 0, int indep = 0,
+                        uint32_t* claim = nullptr, uint32_t epoch = 0) {
   CUtensorMap ta, ta2, tb, ts;
   const uint64_t ka = a_kwrap ? (uint64_t)a_kwrap : (uint64_t)K;
   const uint64_t rows_a = a_split ? (uint64_t)a_split : (uint64_t)M;
@@ -743,7 +823,7 @@ cudaError_t launch_gemm(const void* A, const void* Bm, int M, int N, int K, cons
       if (e != cudaSuccess) return e;
       cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(tiles * ksplit));
-    cfg.blockDim = dim3(kGemmThreads);
+    cfg.blockDim = dim3(EpiWarps<Epi>::kThreads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
     cudaLaunchAttribute at[2];
@@ -757,7 +837,7 @@ cudaError_t launch_gemm(const void* A, const void* Bm, int M, int N, int K, cons
     cfg.numAttrs = 2;
     return note_launch(cudaLaunchKernelEx(&cfg, kern, ta, ta2, tb, ts, M, N, K, epi, status,
                                           (unsigned long long)limit, a_kwrap, a_split, ksplit, a_stream, indep,
-                                          trace));
+                                          (uint32_t*)nullptr, 0u, trace));
     }
   }
   if (ksplit > 1) return cudaErrorInvalidValue;
@@ -766,8 +846,9 @@ cudaError_t launch_gemm(const void* A, const void* Bm, int M, int N, int K, cons
   cudaError_t e = set_smem_once<BN, Epi, false>(smem);
   if (e != cudaSuccess) return e;
   const int grid = (int)grid_ctas;
-  return note_launch(launch_pdl(kern, dim3(grid), dim3(kGemmThreads), smem, st, ta, ta2, tb, ts, M, N, K, epi, status,
-                                (unsigned long long)limit, a_kwrap, a_split, 1, a_stream, indep, trace));
+  return note_launch(launch_pdl(kern, dim3(grid), dim3(EpiWarps<Epi>::kThreads), smem, st, ta, ta2, tb, ts, M, N, K, epi, status,
+                                (unsigned long long)limit, a_kwrap, a_split, 1, a_stream, indep,
+                                grid == sm_count() ? claim : nullptr, epoch, trace));
 }
 
 // A is a weight operand (no earlier kernel writes it): its first tiles are prefetched to L2.
@@ -804,7 +885,7 @@ int max_clusters(int ks) {
     int n = 0;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(ks * 16));
-    cfg.blockDim = dim3(kGemmThreads);
+    cfg.blockDim = dim3(EpiWarps<Epi>::kThreads);
     cfg.dynamicSmemBytes = smem;
     cudaLaunchAttribute at[1];
     at[0].id = cudaLaunchAttributeClusterDimension;
@@ -922,13 +1003,19 @@ cudaError_t gemm_tc_store_f32(const bf16* A, const bf16* Bm, int M, int N, int K
 
 cudaError_t gemm_tc_argmax(const bf16* U, const bf16* W2, int M, int V, int r, const bf16* Lb, long long ldl,
                            uint64_t* keys, float* out, long long ldo, int32_t* status, uint64_t limit,
-                           cudaStream_t st) {
+                           cudaStream_t st, uint32_t* claim, uint32_t epoch) {
+  if (claim) {
+    cudaError_t e = ensure_sm_rank(st);
+    if (e != cudaSuccess) return e;
+  }
   if (r % 128 == 0 && r <= 256) {  // the activation band stays in shared memory for every vocabulary tile
     EpiArgmaxT<true> e{keys, M, out, ldo};
-    return launch_gemm<128>(U, W2, M, V, r, e, status, limit, st, 0, 0, 0, Lb, (uint64_t)ldl, nullptr, 0, 0, 1, 0, 2);
+    return launch_gemm<128>(U, W2, M, V, r, e, status, limit, st, 0, 0, 0, Lb, (uint64_t)ldl, nullptr, 0, 0, 1, 0, 2,
+                            claim, epoch);
   }
   EpiArgmaxT<false> e{keys, M, out, ldo};
-  return launch_gemm<128>(U, W2, M, V, r, e, status, limit, st, 0, 0, 0, Lb, (uint64_t)ldl, nullptr, 0, 0, 1, 0, 2);
+  return launch_gemm<128>(U, W2, M, V, r, e, status, limit, st, 0, 0, 0, Lb, (uint64_t)ldl, nullptr, 0, 0, 1, 0, 2,
+                          claim, epoch);
 }
 
 cudaError_t gemm_tc_gru_u(const bf16* W_hh, const bf16* W1s, long long ldw, const bf16* S_hl, int Hs, int r, int N,

@@ -24,9 +24,14 @@ cudaError_t gemm_tc_store_f32(const __nv_bfloat16* A, const __nv_bfloat16* Bm, i
 //   keys[b] = max(keys[b], key of argmax_v (Lb[b*ldl + v] + sum_k U[b][k] W2[v][k]))
 // (U [M x r], W2 [V x r] bf16; the argmax key orders by value, then lowest index).  When out is
 // non-null the logits are also stored: out[b * ldo + v].
+// claim (optional): work-slot claim words (at least one per SM, zero before the first launch that
+// uses them) and epoch (nonzero, distinct for every launch sharing them): the CTAs then pick
+// their vocabulary tiles by the SM they run on, so that each W2 tile stays with one SM across
+// launches (see k_gemm_tc).
 cudaError_t gemm_tc_argmax(const __nv_bfloat16* U, const __nv_bfloat16* W2, int M, int V, int r,
                            const __nv_bfloat16* Lb, long long ldl, uint64_t* keys, float* out, long long ldo,
-                           int32_t* status, uint64_t limit, cudaStream_t st);
+                           int32_t* status, uint64_t limit, cudaStream_t st, uint32_t* claim = nullptr,
+                           uint32_t epoch = 0);
 
 // u16[n][k] = bf16(SiLU(P[n * ldp + k] + sum_j W1s[k][j] S[n][j])) for k < r, n < N, where the
 // fp32 state arrives as its two-term bf16 split S_hl [N x 2Hs] and W1s [r x Hs] has row stride ldw

@@ -22,6 +22,7 @@ struct Shape {
 struct Workspace {
   int32_t* status;     // fallback status word when the caller passes no status pointer
   uint32_t* sync;      // barrier counters of the persistent kernels (kSyncWords words)
+  uint32_t* claim;     // [kClaimWords] work-slot claims of SM-affine GEMM launches (zeroed per call)
   uint64_t* keys;      // [L][B]   greedy argmax keys per position
   uint64_t* acc_keys;  // [B*L]    target-logit argmax keys (accept length)
   float* P;            // [B*L][r] W1 . H for every position
@@ -37,6 +38,7 @@ struct Workspace {
   size_t bytes;
 };
 constexpr int kSyncWords = 64;
+constexpr int kClaimWords = 1024;
 // The fused greedy kernels spread the W1 state-block partial sums over this many copies of the
 // accumulator (fewer atomics per address); the reader adds the copies.
 constexpr int kAccReplicas = 4;

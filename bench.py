@@ -380,6 +380,27 @@ def cpu_baseline(seconds: float) -> dict:
                       f"{el:.1f} s", "ms_per_block": round(1e3 * el / (n * sh["B"]), 3)}
 
 
+def rank_workload(rank: int) -> dict:
+    """The headline workload of one replica: same shapes and weights, rows drawn from a
+    rank-specific input seed (the replicas draft different rows; nothing is exchanged)."""
+    return synth.workload(HEADLINE, input_seed=synth.WORKLOADS[HEADLINE]["input_seed"] + 1000 * rank)
+
+
+def max_over_ranks(total_ms: float, dist, device) -> float:
+    """The slowest replica's timed-region total (the job ends when the last replica does)."""
+    if dist is None:
+        return total_ms
+    import torch
+    t = torch.tensor([total_ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(B: int, world: int, steps: int, total_ms: float) -> float:
+    """Whole-job blocks/s: every replica drafts B rows per step."""
+    return B * world * steps / (total_ms * 1e-3)
+
+
 def run_ours(args):
     import torch
     rank = int(os.environ.get("RANK", "0"))
@@ -402,22 +423,18 @@ def run_ours(args):
     peaks = _peaks()
 
     # headline point: every rank drafts its own batch (replicas; rows differ per rank)
-    wl = synth.workload(HEADLINE, input_seed=synth.WORKLOADS[HEADLINE]["input_seed"] + 1000 * rank)
+    wl = rank_workload(rank)
     pt = Point(wl, device)
     clk = ClockSampler(local)
     clk.start()
     step_ms, greedy_ms, launches = time_steps(pt, args.steps, args.warmup, flush, stream, dist)
     clocks = clk.stop()
-    total_ms = sum(step_ms)
-    if dist is not None:
-        t = torch.tensor([total_ms], device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(sum(step_ms), dist, device)
     torch.cuda.synchronize()
     assert int(pt.status.item()) == 0, domino.status_string(int(pt.status.item()))
     sh = pt.sh
     B = sh["B"]
-    value = B * world * args.steps / (total_ms * 1e-3)
+    value = job_throughput(B, world, args.steps, total_ms)
 
     g_avg = statistics.mean(greedy_ms)
     gbytes = greedy_bytes(sh)

@@ -95,6 +95,17 @@ def greedy_flops(sh: dict) -> int:
     return 2 * B * (L * r * V + (L - 1) * 3 * Hs * (d + Hs) + L * r * (d + Hs))
 
 
+def tf_bytes(sh: dict) -> int:
+    """Algorithmic bytes of one teacher-forced call (logits out, no states): W_ih, W1 and W2 once
+    (all positions in one product each), W_hh once per GRU update, the given tokens' embedding
+    rows, and per row the base logits, hidden states, S0 and the fp32 logits written."""
+    B, L, d, Hs, r, V = (sh[k] for k in ("B", "L", "d", "Hs", "r", "V"))
+    e = 2 if sh["dtype"] == synth.BF16 else 4
+    weights = (3 * Hs * d + r * (d + Hs) + V * r + 6 * Hs) * e + (L - 1) * 3 * Hs * Hs * e
+    per_row = L * V * e + L * d * e + (L - 1) * d * e + Hs * 4 + L * 4 + L * V * 4
+    return weights + B * per_row
+
+
 def accept_bytes(B: int, L: int, V: int) -> int:
     return B * L * V * 4 + B * L * 4 + B * 4
 
@@ -295,6 +306,30 @@ def w2_kernel_us(pt: Point, flush, stream) -> float:
     t = buf.view(-1, 16).cpu().numpy()
     t = t[(t[:, 1] != 0) & (t[:, 15] != 0)]
     return float((t[:, 1].max() - t[:, 15].min()) / 1e3)
+
+
+def time_tf(pt: Point, steps: int, warmup: int, flush, stream) -> list:
+    """Teacher-forced calls (uniform given tokens, logits out), each after an L2 flush; per-call
+    device times in ms."""
+    torch = pt.torch
+    sh = pt.sh
+    tokens = torch.from_numpy(synth.teacher_tokens(sh, 7)).to(pt.lb.device)
+    logits = torch.empty((sh["B"], sh["L"], sh["V"]), dtype=torch.float32, device=pt.lb.device)
+    for _ in range(warmup):
+        flush.zero_()
+        pt.tf(stream, tokens, logits)
+    torch.cuda.synchronize()
+    times = []
+    with torch.cuda.stream(stream):
+        for _ in range(steps):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            pt.tf(stream, tokens, logits)
+            e1.record(stream)
+            e1.synchronize()
+            times.append(e0.elapsed_time(e1))
+    return times
 
 
 def l2_reread_gbs(nbytes: int, flush, stream, device) -> float:
@@ -524,6 +559,27 @@ def run_ours(args):
                 p.w.embed_proj = None
                 del p
                 torch.cuda.empty_cache()
+        # teacher forcing (B = 1 headline rows and the B = 32 workload) and the Qwen3-4B-shaped head
+        modes = {}
+        if not args.no_points:
+            for name, wl_tf in (("tf_b1", synth.workload(HEADLINE)), ("tf_b32", synth.workload("qwen3-8b-head-b32"))):
+                p = Point(wl_tf, device)
+                t_ms = statistics.mean(time_tf(p, max(3, args.steps // 2), args.warmup, flush, stream))
+                tb = tf_bytes(p.sh)
+                modes[name] = {"blocks_per_s": round(p.sh["B"] / (t_ms * 1e-3), 1), "ms_per_call": round(t_ms, 4),
+                               "algorithmic_bytes": tb, "hbm_frac": round(tb / (t_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
+                               "note": "teacher-forced logits for uniform given tokens, fp32 logits written"}
+                del p
+                torch.cuda.empty_cache()
+            p = Point(synth.workload("qwen3-4b-head-b1"), device)
+            s4, g4, _ = time_steps(p, max(3, args.steps // 2), args.warmup, flush, stream)
+            modes["qwen3-4b-b1"] = {"blocks_per_s": round(len(s4) / (sum(s4) * 1e-3), 1),
+                                    "us_per_block": round(1e3 * statistics.mean(s4), 3),
+                                    "greedy_ms": round(statistics.mean(g4), 4),
+                                    "hbm_frac": round(greedy_bytes(p.sh) / (statistics.mean(g4) * 1e-3) / 1e9
+                                                      / peaks["hbm_gbs"], 4)}
+            del p
+            torch.cuda.empty_cache()
         cpu = None if args.no_cpu_baseline else cpu_baseline(args.cpu_seconds)
         result = {
             "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -543,6 +599,7 @@ def run_ours(args):
             "gpu_launches": launches,
             "clocks": clocks,
             "points": points,
+            "modes": modes,
             "variants": variants,
         }
     if dist is not None:

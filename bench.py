@@ -608,6 +608,25 @@ def run_ours(args):
     return result
 
 
+def profile_driver_tf(n: int, batch: int = 1):
+    """A short, fixed sequence of teacher-forced calls (uniform given tokens, logits out) for an
+    external profiler."""
+    import torch
+    torch.cuda.set_device(0)
+    device = torch.device("cuda", 0)
+    wl = synth.workload(HEADLINE) if batch == 1 else synth.workload("qwen3-8b-head-sweep", B=batch)
+    pt = Point(wl, device)
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
+    tokens = torch.from_numpy(synth.teacher_tokens(pt.sh, 7)).to(device)
+    logits = torch.empty((pt.sh["B"], pt.sh["L"], pt.sh["V"]), dtype=torch.float32, device=device)
+    for _ in range(n):
+        flush.zero_()
+        pt.tf(stream, tokens, logits)
+    torch.cuda.synchronize()
+    assert int(pt.status.item()) == 0
+
+
 def profile_driver(n: int, batch: int = 1, trace: bool = False, proj: bool = False):
     """A short, fixed sequence of greedy calls for an external profiler (ncu -k ... -s ... -c ...).
     With `trace`, the last call records the fused kernel's phase clock stamps (CTA 0) and the
@@ -701,7 +720,11 @@ def main():
     ap.add_argument("--profile-batch", type=int, default=1, help="batch of the profiling driver")
     ap.add_argument("--trace", action="store_true", help="profiling driver: print the fused kernel's phase times")
     ap.add_argument("--proj", action="store_true", help="profiling driver: use the embedding projection table")
+    ap.add_argument("--profile-tf", action="store_true", help="profiling driver: teacher-forced calls instead")
     args = ap.parse_args()
+    if args.profile and args.profile_tf:
+        profile_driver_tf(args.profile, batch=args.profile_batch)
+        return
     if args.profile:
         profile_driver(args.profile, batch=args.profile_batch, trace=args.trace, proj=args.proj)
         return

@@ -379,6 +379,13 @@ int domino_teacher_forced(const domino_shape_t* shape, const domino_weights_t* w
   cudaError_t e = tc ? gemm_tc_store_f32_bn64((const bf*)hidden, (const bf*)w->W1, (int)BL, s.r, s.d, s.d + s.Hs,
                                               ws.P, s.r, st, spin_limit(), cs)
                      : launch_hproj(s, w->W1, hidden, (int)BL, ws.P, cs);
+  // Small batches whose GRU rows fit in TMEM: the whole recurrence in one fused kernel (one grid
+  // barrier per update), then the activations and logits of all positions as below.
+  const bool fused = tc && use_persistent_greedy(s) && tmem_plan_fits(s, persistent_grid(), w->embed_proj != nullptr);
+  if (fused) {
+    if (e == cudaSuccess)
+      e = launch_tf_recurrence_tmem(s, *w, S0, tokens, SB, ws, st, spin_limit(), persistent_grid(), cs);
+  } else {
   if (e == cudaSuccess) e = launch_copy_rows(S0, s.Hs, SB, row, s.B, s.Hs, cs);
   if (e == cudaSuccess && tc) e = launch_split_state(S0, s.Hs, s.B, s.Hs, ws.S_hl, cs);
   // The GRU input half for every given token at once (one GEMM over B*(L-1) gathered rows), unless
@@ -398,6 +405,7 @@ int domino_teacher_forced(const domino_shape_t* shape, const domino_weights_t* w
                      SB + (size_t)i * s.Hs, row, SB + (size_t)(i + 1) * s.Hs, row, nullptr, 0, s.B, st, cs,
                      w->embed_proj);
   }
+  }  // per-update recurrence
   // W2 product over all B*L positions at once: a tcgen05 GEMM with the L_base add fused into its
   // epilogue (activations rounded to bf16 for the tensor cores), or the CUDA-core kernel.
   const bool tc_w2 = s.dtype == DOMINO_DTYPE_BF16 && gemm_tc_supported(s.V, (int)BL, s.r, w->W2, ws.u16);

@@ -103,14 +103,14 @@ struct EpiLogits {  // logits[n][m] = D + Lb[n][m]   (m = vocabulary row, n = (r
   __device__ __forceinline__ void apply(State&, int m, int n0, const float (&v)[16], int N, const uint8_t*, int,
                                         int) const {
     if (m >= M) return;
+    // all loads before any store: the compiler cannot assume that logits and Lb do not alias,
+    // and interleaving them would serialise one memory round trip per column
+    float l[16];
 #pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      const int n = n0 + j;
-      if (n < N) {
-        const size_t at = (size_t)n * M + m;
-        logits[at] = v[j] + __bfloat162float(Lb[at]);
-      }
-    }
+    for (int j = 0; j < 16; ++j) l[j] = (n0 + j < N) ? __bfloat162float(__ldg(Lb + (size_t)(n0 + j) * M + m)) : 0.f;
+#pragma unroll
+    for (int j = 0; j < 16; ++j)
+      if (n0 + j < N) logits[(size_t)(n0 + j) * M + m] = v[j] + l[j];
   }
 };
 
@@ -229,11 +229,14 @@ struct EpiSiluU {
   __device__ __forceinline__ void apply(State&, int m, int n0, const float (&v)[16], int N, const uint8_t*, int,
                                         int) const {
     if (m >= M) return;
+    float pv[16];  // all loads before any store (see EpiLogits)
+#pragma unroll
+    for (int j = 0; j < 16; ++j) pv[j] = (n0 + j < N) ? __ldg(P + (size_t)(n0 + j) * ldp + m) : 0.f;
 #pragma unroll
     for (int j = 0; j < 16; ++j) {
       const int n = n0 + j;
       if (n < N) {
-        const float u = siluf_(P[(size_t)n * ldp + m] + v[j]);
+        const float u = siluf_(pv[j] + v[j]);
         u16[(size_t)n * M + m] = __float2bfloat16_rn(u);
         if (uf) uf[(size_t)n * M + m] = u;
       }

@@ -435,6 +435,8 @@ const char* persistent_plan(const Shape& s) {
          "positions separated by bounded grid barriers";
 }
 
+int persistent_grid() { return num_sms(); }
+
 cudaError_t launch_persistent_greedy(const Shape& s, const domino_weights_t& w, const void* base_logits,
                                      const void* hidden, const float* S0, int32_t* tokens_out, float* logits_out,
                                      float* states_out, const Workspace& ws, int32_t* status, uint64_t spin,

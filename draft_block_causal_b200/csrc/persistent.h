@@ -21,6 +21,14 @@ cudaError_t launch_greedy_tmem(const Shape& s, const domino_weights_t& w, const 
                                const float* S0, int32_t* tokens_out, float* logits_out, float* states_out,
                                const Workspace& ws, int32_t* status, uint64_t spin, int G, cudaStream_t st);
 
+// Teacher-forced GRU recurrence of the TMEM-resident kernel: states [B][L][Hs] (states[b][0] = S0)
+// for the given tokens [B][L]; out-of-range tokens set DOMINO_STATUS_BAD_TOKEN and read token 0.
+cudaError_t launch_tf_recurrence_tmem(const Shape& s, const domino_weights_t& w, const float* S0, const int32_t* tokens,
+                                      float* states, const Workspace& ws, int32_t* status, uint64_t spin, int G,
+                                      cudaStream_t st);
+// Grid of the fused kernels (one CTA per SM of the current device).
+int persistent_grid();
+
 cudaError_t launch_persistent_greedy(const Shape& s, const domino_weights_t& w, const void* base_logits,
                                      const void* hidden, const float* S0, int32_t* tokens_out, float* logits_out,
                                      float* states_out, const Workspace& ws, int32_t* status, uint64_t spin_limit,

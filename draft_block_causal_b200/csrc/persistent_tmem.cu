@@ -15,6 +15,9 @@
 //     current chunk is reduced) and its first chunk is issued between barrier arrival and wait.
 //  3. The W1 state-block partials are spread over kRep replicas of the accumulator, cutting the
 //     number of same-address atomics per replica from G to G/kRep.
+// Teacher-forced mode (tf_tokens set): the given tokens drive the GRU, so the kernel runs only the
+// L - 1 state updates (TMEM-resident rows, one grid barrier each) and writes every state; the
+// activations and logits of all positions then come from two batched tensor-core products.
 // Every wait is bounded; on a timeout the CTA frees its TMEM and returns.
 #include "common.cuh"
 #include "persistent.h"
@@ -50,6 +53,7 @@ struct TArgs {
   unsigned long long* trace;  // [ntrace] SM clock stamps, or null
   int ntrace;
   const float* Xp;  // [V][3Hs] input projection of the embedding table, or null
+  const int32_t* tf_tokens;  // [B][L] given tokens (teacher-forced mode), or null (greedy)
 };
 
 __device__ __forceinline__ unsigned ld_acquire_u32(const unsigned* p) {
@@ -329,13 +333,14 @@ __global__ void __launch_bounds__(kThreads2, 1) k_greedy_tmem(TArgs p) {
     }
     tmem_wait_st();
   }
-  for (int k = tid; k < maxu * kR2; k += kThreads2) {
+  const bool tf = p.tf_tokens != nullptr;
+  for (int k = tid; k < maxu * kR2 && !tf; k += kThreads2) {
     const int jj = k / kR2, kk = k % kR2;
     w1s_s[k] = (jj < nu) ? __bfloat162float(p.W1[(size_t)kk * ldw1 + d + j0 + jj]) : 0.f;
   }
   for (int k = tid; k < BMAX * 6 * maxu; k += kThreads2) gh_s[k] = 0.f;  // gh_s and gi_s
   // a_acc[i][rep][b][k] += W1[k, :d] . H[b, i]  for the rank rows k = c, c + G, ...
-  {
+  if (!tf) {
     const int nk = (kR2 - c + G - 1) / G;
     const int npos = B * L;
     const int nseg = d / 256;
@@ -370,7 +375,7 @@ __global__ void __launch_bounds__(kThreads2, 1) k_greedy_tmem(TArgs p) {
   }
   __syncthreads();
   // a_acc[0][rep][b] += W1[:, d + own units] . S0[b, own units];  states_out[b, 0] = S0[b]
-  for (int t = tid; t < BMAX * (kR2 / 4); t += kThreads2) {
+  for (int t = tid; t < BMAX * (kR2 / 4) && !tf; t += kThreads2) {
     const int b = t / (kR2 / 4), k4 = (t % (kR2 / 4)) * 4;
     if (b < B && nu > 0) {
       float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -388,7 +393,7 @@ __global__ void __launch_bounds__(kThreads2, 1) k_greedy_tmem(TArgs p) {
       p.states[(size_t)b * L * Hs + j0 + jj] = p.S0[(size_t)b * Hs + j0 + jj];
     }
   // L_base rows of position 0 towards L2
-  for (int t = tid; t < B * ((v1 - v0 + 63) / 64); t += kThreads2) {
+  for (int t = tid; t < B * ((v1 - v0 + 63) / 64) && !tf; t += kThreads2) {
     const int b = t / ((v1 - v0 + 63) / 64), ln = t % ((v1 - v0 + 63) / 64);
     if (v0 + ln * 64 < v1) prefetch_l2(p.Lb + (size_t)b * L * V + v0 + ln * 64);
   }
@@ -400,12 +405,31 @@ __global__ void __launch_bounds__(kThreads2, 1) k_greedy_tmem(TArgs p) {
 
   stamp(p.trace, p.ntrace, 1);
   grid_arrive(p, epoch);
-  if (warp < nch) w2_load<BMAX, ROWS>(p, v0, v1, warp, lane, 0, L, qa, lba);
+  if (!tf && warp < nch) w2_load<BMAX, ROWS>(p, v0, v1, warp, lane, 0, L, qa, lba);
   if (!grid_wait(p, epoch, flag_s)) { leave(); return; }
   stamp(p.trace, p.ntrace, 2);
 
   for (int i = 0; i < L; ++i) {
     const size_t lrow = (size_t)i * V;
+    if (tf) {  // ---- teacher-forced step: t_i given; W_hh . S_{i-1} for the own units ----
+      if (i == L - 1) break;
+      if (tid < B) {
+        int tok = p.tf_tokens[(size_t)tid * L + i];
+        if (tok < 0 || tok >= V) {
+          set_status(p.status, DOMINO_STATUS_BAD_TOKEN);
+          tok = 0;
+        }
+        tok_s[tid] = tok;
+      }
+      const float* Sprev = (i == 0) ? p.S0 : p.Sbuf + (size_t)((i - 1) & 1) * B * Hs;
+      for (int t = tid; t < B * Hs; t += kThreads2) {
+        const int b = t / Hs, j = t % Hs;
+        s_t[((size_t)b * 2 * cprh + j % (2 * cprh)) * 128 + j / (2 * cprh)] = __ldcg(Sprev + t);
+      }
+      __syncthreads();
+      if (nu > 0) tmem_rows_dot<BMAX, float>(tbase, colh, cprh, 3 * nu, s_t, B, gh_s, 3 * maxu, warp, lane);
+      stamp(p.trace, p.ntrace, 4 + 10 * i + 3);
+    } else {
     // u = SiLU(sum of the accumulator replicas); S_{i-1} into the lane-sliced layout
     for (int t = tid; t < BMAX * kR2; t += kThreads2) {
       const int b = t / kR2, k = t % kR2;
@@ -488,13 +512,15 @@ __global__ void __launch_bounds__(kThreads2, 1) k_greedy_tmem(TArgs p) {
     if (!grid_wait(p, epoch, flag_s)) { leave(); return; }
     stamp(p.trace, p.ntrace, tb + 3);
     if (i == L - 1) break;
+    }  // greedy step
+    const int tb = 4 + 10 * i;
 
     // t_i; gi = W_ih . embed[t_i] for the own units: gathered from the projection table, or
     // computed from TMEM with the embedding row staged in the lane-sliced layout; GRU cell -> S_i
     if (proj) {
       for (int t = tid; t < B * 3 * nu; t += kThreads2) {
         const int b = t / (3 * nu), R = t % (3 * nu), g = R / nu, jj = R % nu;
-        const int tok = min(max(key_index(__ldcg(p.keys + (size_t)i * B + b)), 0), V - 1);
+        const int tok = tf ? tok_s[b] : min(max(key_index(__ldcg(p.keys + (size_t)i * B + b)), 0), V - 1);
         gi_s[b * 3 * maxu + R] = __ldg(p.Xp + (size_t)tok * 3 * Hs + (size_t)g * Hs + j0 + jj);
       }
       __syncthreads();
@@ -502,7 +528,7 @@ __global__ void __launch_bounds__(kThreads2, 1) k_greedy_tmem(TArgs p) {
     } else {
       for (int t = tid; t < B * (d / 2); t += kThreads2) {
         const int b = t / (d / 2), w = t % (d / 2);
-        const int tok = min(max(key_index(__ldcg(p.keys + (size_t)i * B + b)), 0), V - 1);
+        const int tok = tf ? tok_s[b] : min(max(key_index(__ldcg(p.keys + (size_t)i * B + b)), 0), V - 1);
         x_t[((size_t)b * cpri + w % cpri) * 128 + w / cpri] =
             __ldg(reinterpret_cast<const uint32_t*>(p.embed + (size_t)tok * d) + w);
       }
@@ -533,7 +559,7 @@ __global__ void __launch_bounds__(kThreads2, 1) k_greedy_tmem(TArgs p) {
       if (p.states) p.states[((size_t)b * L + i + 1) * Hs + j] = hn;
     }
     __syncthreads();
-    for (int t = tid; t < BMAX * (kR2 / 4); t += kThreads2) {
+    for (int t = tid; t < BMAX * (kR2 / 4) && !tf; t += kThreads2) {
       const int b = t / (kR2 / 4), k4 = (t % (kR2 / 4)) * 4;
       if (b < B && nu > 0) {
         float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -547,11 +573,11 @@ __global__ void __launch_bounds__(kThreads2, 1) k_greedy_tmem(TArgs p) {
     }
     stamp(p.trace, p.ntrace, tb + 6);
     grid_arrive(p, epoch);
-    if (warp < nch) w2_load<BMAX, ROWS>(p, v0, v1, warp, lane, lrow + V, L, qa, lba);
+    if (!tf && warp < nch) w2_load<BMAX, ROWS>(p, v0, v1, warp, lane, lrow + V, L, qa, lba);
     if (!grid_wait(p, epoch, flag_s)) { leave(); return; }
     stamp(p.trace, p.ntrace, tb + 7);
   }
-  if (c == 0)
+  if (c == 0 && !tf)
     for (int t = tid; t < B * L; t += kThreads2) {
       const int b = t / L, i = t % L;
       p.tokens[t] = key_index(__ldcg(p.keys + (size_t)i * B + b));
@@ -590,10 +616,13 @@ bool tmem_plan_fits(const Shape& s, int G, bool proj) {
          smem_bytes_tmem(4, s.d, s.Hs, maxu) <= 200 * 1024;
 }
 
-cudaError_t launch_greedy_tmem(const Shape& s, const domino_weights_t& w, const void* base_logits, const void* hidden,
+namespace {
+cudaError_t launch_tmem_common(const Shape& s, const domino_weights_t& w, const void* base_logits, const void* hidden,
                                const float* S0, int32_t* tokens_out, float* logits_out, float* states_out,
-                               const Workspace& ws, int32_t* status, uint64_t spin, int G, cudaStream_t st) {
+                               const Workspace& ws, int32_t* status, uint64_t spin, int G, cudaStream_t st,
+                               const int32_t* tf_tokens) {
   TArgs a{};
+  a.tf_tokens = tf_tokens;
   a.embed = (const bf16*)w.embed; a.W_ih = (const bf16*)w.W_ih; a.W_hh = (const bf16*)w.W_hh;
   a.b_ih = (const bf16*)w.b_ih; a.b_hh = (const bf16*)w.b_hh; a.W1 = (const bf16*)w.W1; a.W2 = (const bf16*)w.W2;
   a.Lb = (const bf16*)base_logits; a.H = (const bf16*)hidden; a.S0 = S0;
@@ -613,6 +642,20 @@ cudaError_t launch_greedy_tmem(const Shape& s, const domino_weights_t& w, const 
   else if (bmax == 2) e = launch_tmem_t<2, 8>(a, G, smem, st);
   else e = launch_tmem_t<4, 4>(a, G, smem, st);
   return note_launch(e);
+}
+}  // namespace
+
+cudaError_t launch_greedy_tmem(const Shape& s, const domino_weights_t& w, const void* base_logits, const void* hidden,
+                               const float* S0, int32_t* tokens_out, float* logits_out, float* states_out,
+                               const Workspace& ws, int32_t* status, uint64_t spin, int G, cudaStream_t st) {
+  return launch_tmem_common(s, w, base_logits, hidden, S0, tokens_out, logits_out, states_out, ws, status, spin, G, st,
+                            nullptr);
+}
+
+cudaError_t launch_tf_recurrence_tmem(const Shape& s, const domino_weights_t& w, const float* S0, const int32_t* tokens,
+                                      float* states, const Workspace& ws, int32_t* status, uint64_t spin, int G,
+                                      cudaStream_t st) {
+  return launch_tmem_common(s, w, nullptr, nullptr, S0, nullptr, nullptr, states, ws, status, spin, G, st, tokens);
 }
 
 }  // namespace domino

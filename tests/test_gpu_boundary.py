@@ -167,3 +167,25 @@ def test_split_k_products_are_reproducible():
         assert torch.equal(lg, runs[0][1])
         assert torch.equal(st, runs[0][2])
     assert torch.equal(tf[1][0], tf[0][0]) and torch.equal(tf[1][1], tf[0][1])
+
+
+def test_fused_teacher_forcing_reports_bad_tokens():
+    """Teacher forcing at a TMEM-resident shape runs the fused recurrence: an out-of-range given
+    token sets DOMINO_STATUS_BAD_TOKEN there too, and valid tokens match the oracle."""
+    import oracle
+    data = _persistent_case(B=2, seed=330, Hs=512)
+    w, lb, h, S0 = G.device_inputs(data)
+    y = torch.randint(0, data["shape"]["V"], (2, 16), dtype=torch.int32, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    lg, st = domino.teacher_forced(w, lb, h, S0, y, states_out=True, status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    ref = oracle.head(data["shape"], data["weights"], data["base_logits"], data["hidden"], data["S0"],
+                      tokens=y.cpu().numpy())
+    err = np.abs(lg.cpu().numpy() - ref["logits"])
+    assert (err <= G.LOGIT_ATOL + G.LOGIT_RTOL * np.abs(ref["logits"])).all()
+    assert np.abs(st.cpu().numpy() - ref["states"]).max() <= G.STATE_ATOL
+    y[1, 3] = data["shape"]["V"] + 5
+    domino.teacher_forced(w, lb, h, S0, y, status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == domino.STATUS_BAD_TOKEN

@@ -278,9 +278,10 @@ int domino_draft_greedy(const domino_shape_t* shape, const domino_weights_t* w, 
   // work-slot claims and argmax keys are adjacent: one memset clears both
   cudaError_t e = cudaMemsetAsync(ws.claim, 0, (char*)(ws.keys + BL) - (char*)ws.claim, cs);
   if (e == cudaSuccess) {
-    if (tc)  // P[n][k] = sum_c H[n][c] W1[k][c]: H [B*L x d], the first d columns of W1 (row stride d + Hs)
-      e = gemm_tc_store_f32_bn64((const __nv_bfloat16*)hidden, (const __nv_bfloat16*)w->W1, (int)BL, s.r, s.d,
-                                 s.d + s.Hs, ws.P, s.r, st, spin_limit(), cs);
+    if (tc)  // P[n][k] = sum_c W1[k][c] H[n][c]: the first d columns of W1 (row stride d + Hs) against
+             // the B*L hidden rows, a skinny product (split over K when its tiles do not cover the SMs)
+      e = gemm_tc_store_f32_t((const __nv_bfloat16*)w->W1, (const __nv_bfloat16*)hidden, s.r, (int)BL, s.d, 0, ws.P,
+                              s.r, st, spin_limit(), cs, 0, s.d + s.Hs);
     else
       e = launch_hproj(s, w->W1, hidden, (int)BL, ws.P, cs);
   }
@@ -376,15 +377,29 @@ int domino_teacher_forced(const domino_shape_t* shape, const domino_weights_t* w
   using bf = __nv_bfloat16;
   const bool tc = s.dtype == DOMINO_DTYPE_BF16 && s.d % 64 == 0 && s.r % 64 == 0 && s.Hs % 64 == 0 &&
                   gemm_tc_supported((int)BL, s.r, s.d, hidden, w->W1);
-  cudaError_t e = tc ? gemm_tc_store_f32_bn64((const bf*)hidden, (const bf*)w->W1, (int)BL, s.r, s.d, s.d + s.Hs,
-                                              ws.P, s.r, st, spin_limit(), cs)
+  cudaError_t e = tc ? gemm_tc_store_f32_t((const bf*)w->W1, (const bf*)hidden, s.r, (int)BL, s.d, 0, ws.P, s.r, st,
+                                           spin_limit(), cs, 0, s.d + s.Hs)
                      : launch_hproj(s, w->W1, hidden, (int)BL, ws.P, cs);
   // Small batches whose GRU rows fit in TMEM: the whole recurrence in one fused kernel (one grid
   // barrier per update), then the activations and logits of all positions as below.
-  const bool fused = tc && use_persistent_greedy(s) && tmem_plan_fits(s, persistent_grid(), w->embed_proj != nullptr);
+  // The input half of every update is known up front: one gather + W_ih product over all B*(L-1)
+  // given tokens (unless the projection table holds it), so TMEM keeps only the W_hh rows.
+  // (With a single position no gates are precomputed and the kernel keeps W_ih rows as in greedy
+  // drafting, so that plan must fit then.)
+  const bool fused = tc && use_persistent_greedy(s) && tmem_plan_fits(s, persistent_grid(), true) &&
+                     (s.L > 1 || w->embed_proj || tmem_plan_fits(s, persistent_grid(), false));
   if (fused) {
+    const int NXf = s.B * (s.L - 1);
+    const float* gx = nullptr;
+    if (e == cudaSuccess && !w->embed_proj && NXf > 0) {
+      e = launch_gather_rows((const bf*)w->embed, nullptr, tokens, s.L - 1, s.L, NXf, s.d, s.V, ws.X, cs);
+      if (e == cudaSuccess)
+        e = gemm_tc_store_f32_t((const bf*)w->W_ih, ws.X, 3 * s.Hs, NXf, s.d, 0, ws.Gx, 3 * s.Hs, st, spin_limit(),
+                                cs, 1);
+      gx = ws.Gx;
+    }
     if (e == cudaSuccess)
-      e = launch_tf_recurrence_tmem(s, *w, S0, tokens, SB, ws, st, spin_limit(), persistent_grid(), cs);
+      e = launch_tf_recurrence_tmem(s, *w, S0, tokens, gx, SB, ws, st, spin_limit(), persistent_grid(), cs);
   } else {
   if (e == cudaSuccess) e = launch_copy_rows(S0, s.Hs, SB, row, s.B, s.Hs, cs);
   if (e == cudaSuccess && tc) e = launch_split_state(S0, s.Hs, s.B, s.Hs, ws.S_hl, cs);

@@ -1042,9 +1042,10 @@ cudaError_t gemm_tc_store_f32_bn64(const bf16* A, const bf16* Bm, int M, int N, 
 }
 
 cudaError_t gemm_tc_store_f32_t(const bf16* A, const bf16* Bm, int M, int N, int K, int a_kwrap, float* out,
-                                long long ldo, int32_t* status, uint64_t limit, cudaStream_t st, int a_stream) {
+                                long long ldo, int32_t* status, uint64_t limit, cudaStream_t st, int a_stream,
+                                long long lda) {
   EpiStore e{out, M, ldo, 1};
-  return launch_gemm_skinny(A, Bm, M, N, K, e, status, limit, st, 0, a_kwrap, nullptr, 0, 0, a_stream);
+  return launch_gemm_skinny(A, Bm, M, N, K, e, status, limit, st, (uint64_t)lda, a_kwrap, nullptr, 0, 0, a_stream);
 }
 
 cudaError_t gemm_tc_logits(const bf16* W2, const bf16* U, int V, int N, int r, const bf16* Lb, float* logits,

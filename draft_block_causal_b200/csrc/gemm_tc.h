@@ -57,9 +57,10 @@ cudaError_t gemm_tc_store_f32_bn64(const __nv_bfloat16* A, const __nv_bfloat16* 
 // (N = a batch of rows), stored transposed (n-major) so that per-row consumers read contiguously.
 // With a_kwrap = K/2 and Bm = [hi | lo] this applies A to a two-term bf16 split of an fp32 operand.
 // a_stream: A is read once per call (no reuse by later calls): its lines are evicted from L2 first.
+// lda: row stride of A in elements (0: K, or a_kwrap when set).
 cudaError_t gemm_tc_store_f32_t(const __nv_bfloat16* A, const __nv_bfloat16* Bm, int M, int N, int K, int a_kwrap,
                                 float* out, long long ldo, int32_t* status, uint64_t limit, cudaStream_t st,
-                                int a_stream = 0);
+                                int a_stream = 0, long long lda = 0);
 
 // One store-epilogue product with a forced plan (bn in {16, 32, 64, 128}, ks in 1..8) or the
 // automatic skinny plan (bn = ks = 0); out[m * ldo + n], or out[n * ldo + m] when trans.

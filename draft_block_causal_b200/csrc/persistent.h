@@ -23,9 +23,11 @@ cudaError_t launch_greedy_tmem(const Shape& s, const domino_weights_t& w, const 
 
 // Teacher-forced GRU recurrence of the TMEM-resident kernel: states [B][L][Hs] (states[b][0] = S0)
 // for the given tokens [B][L]; out-of-range tokens set DOMINO_STATUS_BAD_TOKEN and read token 0.
+// Gx (optional): [B][L-1][3Hs] fp32 W_ih . embed[y_i], computed up front; else the projection
+// table of the weights, else the TMEM-resident W_ih rows give the input half.
 cudaError_t launch_tf_recurrence_tmem(const Shape& s, const domino_weights_t& w, const float* S0, const int32_t* tokens,
-                                      float* states, const Workspace& ws, int32_t* status, uint64_t spin, int G,
-                                      cudaStream_t st);
+                                      const float* Gx, float* states, const Workspace& ws, int32_t* status,
+                                      uint64_t spin, int G, cudaStream_t st);
 // Grid of the fused kernels (one CTA per SM of the current device).
 int persistent_grid();
 

@@ -54,6 +54,7 @@ struct TArgs {
   int ntrace;
   const float* Xp;  // [V][3Hs] input projection of the embedding table, or null
   const int32_t* tf_tokens;  // [B][L] given tokens (teacher-forced mode), or null (greedy)
+  const float* Gx;           // teacher-forced mode: [B][L-1][3Hs] W_ih . embed[y_i] precomputed, or null
 };
 
 __device__ __forceinline__ unsigned ld_acquire_u32(const unsigned* p) {
@@ -265,8 +266,10 @@ __global__ void __launch_bounds__(kThreads2, 1) k_greedy_tmem(TArgs p) {
   const int nu = j1 - j0;
   const int ldw1 = d + Hs;
   const int cpri = d / 256, cprh = Hs / 256;       // TMEM columns per W_ih / W_hh row
-  const bool proj = p.Xp != nullptr;               // GRU input half gathered from the projection table
-  const int colh = proj ? 0 : 3 * nu * cpri;       // first W_hh column (W_ih rows are not kept with proj)
+  // GRU input half gathered from the projection table (per token) or from precomputed teacher-forced
+  // gates (per row and position): the W_ih rows are then not kept in TMEM
+  const bool proj = p.Xp != nullptr || p.Gx != nullptr;
+  const int colh = proj ? 0 : 3 * nu * cpri;       // first W_hh column
   const int rep = c % kRep;
 
   // shared memory
@@ -520,6 +523,10 @@ __global__ void __launch_bounds__(kThreads2, 1) k_greedy_tmem(TArgs p) {
     if (proj) {
       for (int t = tid; t < B * 3 * nu; t += kThreads2) {
         const int b = t / (3 * nu), R = t % (3 * nu), g = R / nu, jj = R % nu;
+        if (p.Gx) {  // teacher forcing: the gates of (row b, position i) were computed up front
+          gi_s[b * 3 * maxu + R] = __ldg(p.Gx + ((size_t)b * (L - 1) + i) * 3 * Hs + (size_t)g * Hs + j0 + jj);
+          continue;
+        }
         const int tok = tf ? tok_s[b] : min(max(key_index(__ldcg(p.keys + (size_t)i * B + b)), 0), V - 1);
         gi_s[b * 3 * maxu + R] = __ldg(p.Xp + (size_t)tok * 3 * Hs + (size_t)g * Hs + j0 + jj);
       }
@@ -620,9 +627,10 @@ namespace {
 cudaError_t launch_tmem_common(const Shape& s, const domino_weights_t& w, const void* base_logits, const void* hidden,
                                const float* S0, int32_t* tokens_out, float* logits_out, float* states_out,
                                const Workspace& ws, int32_t* status, uint64_t spin, int G, cudaStream_t st,
-                               const int32_t* tf_tokens) {
+                               const int32_t* tf_tokens, const float* Gx) {
   TArgs a{};
   a.tf_tokens = tf_tokens;
+  a.Gx = Gx;
   a.embed = (const bf16*)w.embed; a.W_ih = (const bf16*)w.W_ih; a.W_hh = (const bf16*)w.W_hh;
   a.b_ih = (const bf16*)w.b_ih; a.b_hh = (const bf16*)w.b_hh; a.W1 = (const bf16*)w.W1; a.W2 = (const bf16*)w.W2;
   a.Lb = (const bf16*)base_logits; a.H = (const bf16*)hidden; a.S0 = S0;
@@ -649,13 +657,13 @@ cudaError_t launch_greedy_tmem(const Shape& s, const domino_weights_t& w, const 
                                const float* S0, int32_t* tokens_out, float* logits_out, float* states_out,
                                const Workspace& ws, int32_t* status, uint64_t spin, int G, cudaStream_t st) {
   return launch_tmem_common(s, w, base_logits, hidden, S0, tokens_out, logits_out, states_out, ws, status, spin, G, st,
-                            nullptr);
+                            nullptr, nullptr);
 }
 
 cudaError_t launch_tf_recurrence_tmem(const Shape& s, const domino_weights_t& w, const float* S0, const int32_t* tokens,
-                                      float* states, const Workspace& ws, int32_t* status, uint64_t spin, int G,
-                                      cudaStream_t st) {
-  return launch_tmem_common(s, w, nullptr, nullptr, S0, nullptr, nullptr, states, ws, status, spin, G, st, tokens);
+                                      const float* Gx, float* states, const Workspace& ws, int32_t* status,
+                                      uint64_t spin, int G, cudaStream_t st) {
+  return launch_tmem_common(s, w, nullptr, nullptr, S0, nullptr, nullptr, states, ws, status, spin, G, st, tokens, Gx);
 }
 
 }  // namespace domino

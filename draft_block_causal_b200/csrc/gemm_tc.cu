@@ -114,6 +114,47 @@ struct EpiLogits {  // logits[n][m] = D + Lb[n][m]   (m = vocabulary row, n = (r
   }
 };
 
+// Teacher-forced logits, row-major: m = row (b, i) < M, n = vocabulary column < N:
+//   logits[m * ld + n] = D + Lb[m * ld + n]
+// Each thread owns 16 consecutive columns of one row: two 16-byte loads and four 16-byte stores
+// (rows are 16-byte aligned since V % 8 == 0; n0 is a multiple of 16).
+struct EpiLogitsRow {
+  static constexpr bool kSide = false;
+  static constexpr bool kARes = false;
+  static constexpr bool kSideL2 = false;
+  static constexpr int kGroups = 1;
+  using State = NoState;
+  const bf16* Lb;
+  float* logits;
+  int M;
+  long long ld;
+  __device__ __forceinline__ void init(State&) const {}
+  __device__ __forceinline__ void finish(State&, int) const {}
+  __device__ __forceinline__ void apply(State&, int m, int n0, const float (&v)[16], int N, const uint8_t*, int,
+                                        int) const {
+    if (m >= M) return;
+    const bf16* lr = Lb + (size_t)m * ld + n0;
+    float* o = logits + (size_t)m * ld + n0;
+    if (n0 + 16 <= N) {
+      float a[8], b[8];
+      widen(__ldg(reinterpret_cast<const uint4*>(lr)), a);
+      widen(__ldg(reinterpret_cast<const uint4*>(lr) + 1), b);
+      float4* o4 = reinterpret_cast<float4*>(o);
+      o4[0] = make_float4(v[0] + a[0], v[1] + a[1], v[2] + a[2], v[3] + a[3]);
+      o4[1] = make_float4(v[4] + a[4], v[5] + a[5], v[6] + a[6], v[7] + a[7]);
+      o4[2] = make_float4(v[8] + b[0], v[9] + b[1], v[10] + b[2], v[11] + b[3]);
+      o4[3] = make_float4(v[12] + b[4], v[13] + b[5], v[14] + b[6], v[15] + b[7]);
+    } else {
+      float l[16];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) l[j] = (n0 + j < N) ? __bfloat162float(lr[j]) : 0.f;
+#pragma unroll
+      for (int j = 0; j < 16; ++j)
+        if (n0 + j < N) o[j] = v[j] + l[j];
+    }
+  }
+};
+
 // Greedy step, batch-major: m = batch row b (< M), n = vocabulary row v.
 //   z = D + Lb[b][v] (Lb row stride ldl); per 16-column group the maximum (a tree of 15 max
 //   operations) is compared with the running best, and only a group that beats it (strict >, so
@@ -1050,6 +1091,10 @@ cudaError_t gemm_tc_store_f32_t(const bf16* A, const bf16* Bm, int M, int N, int
 
 cudaError_t gemm_tc_logits(const bf16* W2, const bf16* U, int V, int N, int r, const bf16* Lb, float* logits,
                            int32_t* status, uint64_t limit, cudaStream_t st) {
+  if (N >= 64) {  // enough rows for the row-major orientation: vector loads and stores in the epilogue
+    EpiLogitsRow e{Lb, logits, N, (long long)V};
+    return launch_gemm<256>(U, W2, N, V, r, e, status, limit, st, 0, 0, 0, nullptr, 0, nullptr, 0, 0, 1, 0, 2);
+  }
   EpiLogits e{Lb, logits, V};
   return launch_gemm_bn(W2, U, V, N, r, e, status, limit, st);
 }

@@ -409,7 +409,8 @@ int domino_teacher_forced(const domino_shape_t* shape, const domino_weights_t* w
   if (e == cudaSuccess && tc && !w->embed_proj && NX > 0) {
     e = launch_gather_rows((const bf*)w->embed, nullptr, tokens, s.L - 1, s.L, NX, s.d, s.V, ws.X, cs);
     if (e == cudaSuccess)
-      e = gemm_tc_store_f32((const bf*)w->W_ih, ws.X, 3 * s.Hs, NX, s.d, ws.Gx, 3 * s.Hs, st, spin_limit(), cs, 1);
+      e = gemm_tc_store_f32_t((const bf*)w->W_ih, ws.X, 3 * s.Hs, NX, s.d, 0, ws.Gx, 3 * s.Hs, st, spin_limit(), cs,
+                              1);
   }
   for (int i = 0; i + 1 < s.L && e == cudaSuccess; ++i) {
     if (tc)

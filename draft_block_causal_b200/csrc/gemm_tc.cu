@@ -122,7 +122,7 @@ struct EpiLogitsRow {
   static constexpr bool kSide = false;
   static constexpr bool kARes = false;
   static constexpr bool kSideL2 = false;
-  static constexpr int kGroups = 1;
+  static constexpr int kGroups = 2;  // the epilogue is the longest phase of a tile: two warps per lane quadrant
   using State = NoState;
   const bf16* Lb;
   float* logits;

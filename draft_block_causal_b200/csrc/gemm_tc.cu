@@ -516,8 +516,8 @@ __global__ void __launch_bounds__(EpiWarps<Epi>::kThreads, 1)
             const int m2 = (tile2 / n_tiles) * kBM, n2 = (tile2 % n_tiles) * BN;
             if constexpr (Epi::kARes)
               for (int kb = 0; kb < kblocks; ++kb) tma_prefetch_l2(&tmB, kb * kBK, n2);
-            if constexpr (Epi::kSide)
-              for (int bx = 0; bx < BN / 64; ++bx) tma_prefetch_l2_hint(&tmS, n2 + bx * 64, m2, pol_first);
+            if constexpr (Epi::kSide)  // normal priority: the lines must survive until the side load
+              for (int bx = 0; bx < BN / 64; ++bx) tma_prefetch_l2(&tmS, n2 + bx * 64, m2);
           }
         }
         for (int kb = kb0; kb < kb1; kb += C::kKBS, ++it) {

@@ -4,28 +4,36 @@
 //
 // One CTA per SM walks output tiles of 128 x BN.  Warp roles:
 //   warp 0, one thread : TMA producer -- 128x64 A tile + BNx64 B tile per k-block into a ring of
-//                        S shared-memory stages (128-byte swizzle), signalled on full[s]
+//                        S shared-memory stages (128-byte swizzle), signalled on full[s]; with a
+//                        resident A (K <= 256, one 128-row band) only B streams, two k-blocks a stage
 //   warp 1, one thread : MMA issuer   -- four tcgen05.mma (K = 16) per k-block into one of two TMEM
 //                        accumulators; tcgen05.commit frees the stage (empty[s]) and, after the
 //                        last k-block, publishes the accumulator (acc_full[a])
-//   warps 2..5         : epilogue     -- tcgen05.ld of the accumulator (warp w reads TMEM lanes
-//                        32*(w%4).., i.e. output rows), then the epilogue functor; acc_empty[a]
+//   warps 2 ..         : epilogue     -- 4 or 8 warps (EpiWarps); warp w reads TMEM lanes
+//                        32*(w%4).. (output rows) and, with 8 warps, half of the columns; then the
+//                        epilogue functor; acc_empty[a]
 // Split-K: when the output has too few tiles to occupy the SMs, each tile's K range is cut into
 // ksplit pieces computed by the ksplit CTAs of one thread-block cluster (one tile per cluster, one
-// piece per CTA).  Each CTA parks its fp32 accumulator in its own shared memory; after a cluster
-// barrier every CTA takes 1/ksplit of the tile, adds the ksplit partials read from its peers'
-// shared memory in piece order (fixed, so results do not depend on scheduling) and runs the
-// epilogue functor on them; a second cluster barrier keeps every CTA's shared memory alive until
-// its peers have read it.
+// piece per CTA).  Each CTA stores its partial of every 16-column unit of the tile straight into the
+// shared memory of the cluster CTA that owns the unit (st.shared::cluster); after one cluster
+// barrier each owner adds the ksplit pieces in piece order (fixed, so results do not depend on
+// scheduling) and runs the epilogue functor.  An earlier cluster barrier, arrived at start and
+// awaited before the first remote store, guarantees that every CTA of the cluster is running.
+// Launches use programmatic stream serialization: a CTA triggers its dependents after set-up and
+// waits on the previous grid before touching produced memory; the producer prefetches weight tiles
+// into L2 before that wait.  A persistent launch with one CTA per SM may take its work slots by the
+// SM it runs on (claim_slot), so that each tile keeps the same SM at every launch.
 // Every mbarrier wait is bounded.  A role that gives up raises a CTA-wide abort flag; the others
 // stop at their next wait, the producer waits for its copies still in flight, TMEM is freed and
 // DOMINO_STATUS_DEVICE_TIMEOUT is reported.
 //
-// Uses in this library:
-//   - the W2 product of teacher forcing: A = W2 [V x r], B = u [B*L x r] (bf16), epilogue adds
-//     L_base and writes fp32 logits -- the logit-space residual of the Domino head equation;
-//   - the input projection of the embedding table: A = embed [V x d], B = W_ih [3Hs x d],
-//     epilogue stores fp32 [V x 3Hs] (the GRU's input half for every token at once).
+// Uses in this library (the Domino head equation, review page section 二):
+//   - the W2 product of greedy drafting, batch-major with L_base and the argmax in the epilogue
+//     (EpiArgmaxT), and of teacher forcing with L_base added (EpiLogitsRow / EpiLogits);
+//   - the GRU products on the tensor cores: W_ih . embedding rows and W_hh . state (EpiStore,
+//     transposed), W_hh stacked with W1's state block giving gh and the next activations
+//     (EpiGruU), the activations alone (EpiSiluU), and the H-projection W1[:, :d] . H (EpiStore);
+//   - the input projection of the embedding table (embed . W_ih^T, EpiStore).
 #include "common.cuh"
 #include "gemm_tc.h"
 #include "launch.cuh"
@@ -1074,12 +1082,6 @@ cudaError_t gemm_tc_silu_u(const bf16* W1s, long long ldw, const bf16* S_hl, int
                            long long ldp, bf16* u16, float* uf, int32_t* status, uint64_t limit, cudaStream_t st) {
   EpiSiluU e{P, ldp, u16, uf, r};
   return launch_gemm_skinny(W1s, S_hl, r, N, 2 * Hs, e, status, limit, st, (uint64_t)ldw, Hs);
-}
-
-cudaError_t gemm_tc_store_f32_bn64(const bf16* A, const bf16* Bm, int M, int N, int K, long long ldb, float* out,
-                                  long long ldo, int32_t* status, uint64_t limit, cudaStream_t st) {
-  EpiStore e{out, M, ldo, 0};
-  return launch_gemm<64>(A, Bm, M, N, K, e, status, limit, st, 0, (uint64_t)ldb, 0, nullptr, 0, nullptr, 0, 0, 1, 0, 3);
 }
 
 cudaError_t gemm_tc_store_f32_t(const bf16* A, const bf16* Bm, int M, int N, int K, int a_kwrap, float* out,

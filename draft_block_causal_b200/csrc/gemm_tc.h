@@ -48,11 +48,6 @@ cudaError_t gemm_tc_gru_u(const __nv_bfloat16* W_hh, const __nv_bfloat16* W1s, l
                           const __nv_bfloat16* S_hl, int Hs, int r, int N, float* Gh, const float* P, long long ldp,
                           __nv_bfloat16* u16, int32_t* status, uint64_t limit, cudaStream_t st);
 
-// out[m * ldo + n] = sum_k A[m][k] Bm[n*ldb + k], with 64-wide output tiles (more CTAs for small N)
-cudaError_t gemm_tc_store_f32_bn64(const __nv_bfloat16* A, const __nv_bfloat16* Bm, int M, int N, int K,
-                                  long long ldb, float* out, long long ldo, int32_t* status, uint64_t limit,
-                                  cudaStream_t st);
-
 // out[n * ldo + m] = sum_k A[m][k mod a_kwrap] Bm[n][k] (a_kwrap = 0: no wrap) for a skinny Bm
 // (N = a batch of rows), stored transposed (n-major) so that per-row consumers read contiguously.
 // With a_kwrap = K/2 and Bm = [hi | lo] this applies A to a two-term bf16 split of an fp32 operand.

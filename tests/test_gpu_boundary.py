@@ -189,3 +189,25 @@ def test_fused_teacher_forcing_reports_bad_tokens():
     domino.teacher_forced(w, lb, h, S0, y, status=status)
     torch.cuda.synchronize()
     assert int(status.item()) == domino.STATUS_BAD_TOKEN
+
+
+def test_batched_teacher_forcing_reports_bad_tokens():
+    """B = 8 (beyond the TMEM kernel): the batched tensor-core recurrence gives the oracle's logits
+    and states, and an out-of-range given token sets DOMINO_STATUS_BAD_TOKEN."""
+    import oracle
+    data = _persistent_case(B=8, seed=340, Hs=256)
+    w, lb, h, S0 = G.device_inputs(data)
+    y = torch.randint(0, data["shape"]["V"], (8, 16), dtype=torch.int32, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    lg, st = domino.teacher_forced(w, lb, h, S0, y, states_out=True, status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    ref = oracle.head(data["shape"], data["weights"], data["base_logits"], data["hidden"], data["S0"],
+                      tokens=y.cpu().numpy())
+    err = np.abs(lg.cpu().numpy() - ref["logits"])
+    assert (err <= G.LOGIT_ATOL + G.LOGIT_RTOL * np.abs(ref["logits"])).all()
+    assert np.abs(st.cpu().numpy() - ref["states"]).max() <= G.STATE_ATOL
+    y[5, 7] = -3
+    domino.teacher_forced(w, lb, h, S0, y, status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == domino.STATUS_BAD_TOKEN

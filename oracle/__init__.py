@@ -47,20 +47,24 @@ def build(force: bool = False) -> str:
 _lib = None
 
 
+def configure(lib: ctypes.CDLL) -> ctypes.CDLL:
+    """Declare the C entry points' argument types on a loaded oracle library."""
+    vp = ctypes.c_void_p
+    lib.oracle_head.argtypes = [ctypes.POINTER(_Shape)] + [vp] * 10 + [vp, vp, vp, vp, vp, ctypes.c_int]
+    lib.oracle_head.restype = ctypes.c_int
+    lib.oracle_accept_len.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, vp, vp, vp]
+    lib.oracle_accept_len.restype = ctypes.c_int
+    lib.oracle_gru_step.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int] + [vp] * 7
+    lib.oracle_gru_step.restype = None
+    lib.oracle_max_threads.argtypes = []
+    lib.oracle_max_threads.restype = ctypes.c_int
+    return lib
+
+
 def _load():
     global _lib
     if _lib is None:
-        lib = ctypes.CDLL(build())
-        vp, i32p, f64p, f32p = ctypes.c_void_p, ctypes.POINTER(ctypes.c_int32), ctypes.c_void_p, ctypes.c_void_p
-        lib.oracle_head.argtypes = [ctypes.POINTER(_Shape)] + [vp] * 10 + [vp, vp, vp, vp, vp, ctypes.c_int]
-        lib.oracle_head.restype = ctypes.c_int
-        lib.oracle_accept_len.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, vp, vp, vp]
-        lib.oracle_accept_len.restype = ctypes.c_int
-        lib.oracle_gru_step.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int] + [vp] * 7
-        lib.oracle_gru_step.restype = None
-        lib.oracle_max_threads.argtypes = []
-        lib.oracle_max_threads.restype = ctypes.c_int
-        _lib = lib
+        _lib = configure(ctypes.CDLL(build()))
     return _lib
 
 

@@ -171,7 +171,8 @@ DOMINO_API int domino_draft_greedy(const domino_shape_t* shape, const domino_wei
  * given tokens instead of its own predictions).  Same equations as greedy drafting with
  * t_i := tokens[b, i]; no argmax is taken.
  * Inputs:  as domino_draft_greedy plus tokens [B, L] int32 (each in [0, V); an out-of-range
- *          token sets DOMINO_STATUS_BAD_TOKEN and its row's later outputs are unspecified).
+ *          token sets DOMINO_STATUS_BAD_TOKEN and its row's later outputs are unspecified;
+ *          tokens[b, L-1] feeds no GRU update and is not read).
  * Outputs: logits_out [B, L, V] fp32 (required); states_out [B, L, Hs] fp32 or NULL.
  * Returns DOMINO_OK or a negative DOMINO_ERR_* code. */
 DOMINO_API int domino_teacher_forced(const domino_shape_t* shape, const domino_weights_t* weights,

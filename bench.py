@@ -446,7 +446,7 @@ def run_ours(args):
         import torch.distributed as dist_mod
         dist = dist_mod
         torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
                                 device_id=torch.device("cuda", local))
     else:
         torch.cuda.set_device(local)
@@ -496,35 +496,39 @@ def run_ours(args):
                    "frac": round(t_bound_ms / g_avg, 4)}
         e2e_ms, h2d, d2h = time_e2e(pt, max(3, args.steps // 2), 2, flush, stream)
         e2e_val = B / (statistics.mean(e2e_ms) * 1e-3)
+        # The extra measurements (variants, batch points, modes, CPU baseline) belong to the
+        # single-GPU run; with N > 1 the other ranks would only wait for them at the final barrier.
+        extras = world == 1
         # variant: the same workload with the GRU input half gathered from the projection table
         variants = {}
-        pt.w.embed_proj = pt.domino.project_embeddings(pt.w)
-        torch.cuda.synchronize()
-        v_step, v_greedy, _ = time_steps(pt, args.steps, args.warmup, flush, stream)
-        pt.w.embed_proj = None
-        vg = statistics.mean(v_greedy)
-        vb = greedy_bytes_proj(sh)
-        variants["embed_proj"] = {
-            "blocks_per_s": round(B * len(v_step) / (sum(v_step) * 1e-3), 2),
-            "us_per_block": round(1e3 * statistics.mean(v_step) / B, 3),
-            "greedy_ms": round(vg, 4),
-            "roofline": {"bound": "hbm", "achieved": round(vb / (vg * 1e-3) / 1e9, 1), "peak": peaks["hbm_gbs"],
-                         "unit": "GB/s", "frac": round(vb / (vg * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
-                         "algorithmic_bytes": vb},
-            "note": "GRU input half gathered from embed . W_ih^T (prepared once per weight set, untimed)",
-        }
-        warm = time_steps_persisting(pt, args.steps, args.warmup, flush, stream)
-        if warm is not None:
-            w_step, w_greedy, _ = warm
-            variants["l2_persisting"] = {
-                "blocks_per_s": round(B * len(w_step) / (sum(w_step) * 1e-3), 2),
-                "us_per_block": round(1e3 * statistics.mean(w_step) / B, 3),
-                "greedy_ms": round(statistics.mean(w_greedy), 4),
-                "note": "warm regime: weights packed into one arena under an L2 persisting access-policy "
-                        "window (domino_set_l2_persistence); L2 still flushed before every step",
+        if extras:
+            pt.w.embed_proj = pt.domino.project_embeddings(pt.w)
+            torch.cuda.synchronize()
+            v_step, v_greedy, _ = time_steps(pt, args.steps, args.warmup, flush, stream)
+            pt.w.embed_proj = None
+            vg = statistics.mean(v_greedy)
+            vb = greedy_bytes_proj(sh)
+            variants["embed_proj"] = {
+                "blocks_per_s": round(B * len(v_step) / (sum(v_step) * 1e-3), 2),
+                "us_per_block": round(1e3 * statistics.mean(v_step) / B, 3),
+                "greedy_ms": round(vg, 4),
+                "roofline": {"bound": "hbm", "achieved": round(vb / (vg * 1e-3) / 1e9, 1), "peak": peaks["hbm_gbs"],
+                             "unit": "GB/s", "frac": round(vb / (vg * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
+                             "algorithmic_bytes": vb},
+                "note": "GRU input half gathered from embed . W_ih^T (prepared once per weight set, untimed)",
             }
+            warm = time_steps_persisting(pt, args.steps, args.warmup, flush, stream)
+            if warm is not None:
+                w_step, w_greedy, _ = warm
+                variants["l2_persisting"] = {
+                    "blocks_per_s": round(B * len(w_step) / (sum(w_step) * 1e-3), 2),
+                    "us_per_block": round(1e3 * statistics.mean(w_step) / B, 3),
+                    "greedy_ms": round(statistics.mean(w_greedy), 4),
+                    "note": "warm regime: weights packed into one arena under an L2 persisting access-policy "
+                            "window (domino_set_l2_persistence); L2 still flushed before every step",
+                }
         points = {}
-        if not args.no_points:
+        if extras and not args.no_points:
             del pt
             torch.cuda.empty_cache()
             for pb in (32, 128):
@@ -561,7 +565,7 @@ def run_ours(args):
                 torch.cuda.empty_cache()
         # teacher forcing (B = 1 headline rows and the B = 32 workload) and the Qwen3-4B-shaped head
         modes = {}
-        if not args.no_points:
+        if extras and not args.no_points:
             for name, wl_tf in (("tf_b1", synth.workload(HEADLINE)), ("tf_b32", synth.workload("qwen3-8b-head-b32"))):
                 p = Point(wl_tf, device)
                 t_ms = statistics.mean(time_tf(p, max(3, args.steps // 2), args.warmup, flush, stream))
@@ -580,7 +584,7 @@ def run_ours(args):
                                                       / peaks["hbm_gbs"], 4)}
             del p
             torch.cuda.empty_cache()
-        cpu = None if args.no_cpu_baseline else cpu_baseline(args.cpu_seconds)
+        cpu = None if (args.no_cpu_baseline or not extras) else cpu_baseline(args.cpu_seconds)
         result = {
             "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 4), "higher_is_better": True,

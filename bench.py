@@ -95,14 +95,15 @@ def greedy_flops(sh: dict) -> int:
     return 2 * B * (L * r * V + (L - 1) * 3 * Hs * (d + Hs) + L * r * (d + Hs))
 
 
-def tf_bytes(sh: dict) -> int:
+def tf_bytes(sh: dict, logit_bytes: int = 4) -> int:
     """Algorithmic bytes of one teacher-forced call (logits out, no states): W_ih, W1 and W2 once
     (all positions in one product each), W_hh once per GRU update, the given tokens' embedding
-    rows, and per row the base logits, hidden states, S0 and the fp32 logits written."""
+    rows, and per row the base logits, hidden states, S0 and the logits written (4 bytes each, or 2
+    for bf16 logits)."""
     B, L, d, Hs, r, V = (sh[k] for k in ("B", "L", "d", "Hs", "r", "V"))
     e = 2 if sh["dtype"] == synth.BF16 else 4
     weights = (3 * Hs * d + r * (d + Hs) + V * r + 6 * Hs) * e + (L - 1) * 3 * Hs * Hs * e
-    per_row = L * V * e + L * d * e + (L - 1) * d * e + Hs * 4 + L * 4 + L * V * 4
+    per_row = L * V * e + L * d * e + (L - 1) * d * e + Hs * 4 + L * 4 + L * V * logit_bytes
     return weights + B * per_row
 
 
@@ -308,13 +309,14 @@ def w2_kernel_us(pt: Point, flush, stream) -> float:
     return float((t[:, 1].max() - t[:, 15].min()) / 1e3)
 
 
-def time_tf(pt: Point, steps: int, warmup: int, flush, stream) -> list:
+def time_tf(pt: Point, steps: int, warmup: int, flush, stream, bf16_logits: bool = False) -> list:
     """Teacher-forced calls (uniform given tokens, logits out), each after an L2 flush; per-call
     device times in ms."""
     torch = pt.torch
     sh = pt.sh
     tokens = torch.from_numpy(synth.teacher_tokens(sh, 7)).to(pt.lb.device)
-    logits = torch.empty((sh["B"], sh["L"], sh["V"]), dtype=torch.float32, device=pt.lb.device)
+    logits = torch.empty((sh["B"], sh["L"], sh["V"]), dtype=torch.bfloat16 if bf16_logits else torch.float32,
+                         device=pt.lb.device)
     for _ in range(warmup):
         flush.zero_()
         pt.tf(stream, tokens, logits)
@@ -573,6 +575,14 @@ def run_ours(args):
                 modes[name] = {"blocks_per_s": round(p.sh["B"] / (t_ms * 1e-3), 1), "ms_per_call": round(t_ms, 4),
                                "algorithmic_bytes": tb, "hbm_frac": round(tb / (t_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
                                "note": "teacher-forced logits for uniform given tokens, fp32 logits written"}
+                if name == "tf_b32":  # the same with bf16 logits (half the bytes of the largest output)
+                    t16 = statistics.mean(time_tf(p, max(3, args.steps // 2), args.warmup, flush, stream, True))
+                    tb16 = tf_bytes(p.sh, 2)
+                    modes["tf_b32_bf16_logits"] = {
+                        "blocks_per_s": round(p.sh["B"] / (t16 * 1e-3), 1), "ms_per_call": round(t16, 4),
+                        "algorithmic_bytes": tb16,
+                        "hbm_frac": round(tb16 / (t16 * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
+                        "note": "as tf_b32 with bf16 logits (domino_teacher_forced_ex)"}
                 del p
                 torch.cuda.empty_cache()
             p = Point(synth.workload("qwen3-4b-head-b1"), device)

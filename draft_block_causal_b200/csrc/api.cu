@@ -352,10 +352,15 @@ int domino_draft_greedy(const domino_shape_t* shape, const domino_weights_t* w, 
   return cuda_rc(e);
 }
 
-int domino_teacher_forced(const domino_shape_t* shape, const domino_weights_t* w, const void* base_logits,
-                          const void* hidden, const float* S0, const int32_t* tokens, float* logits_out,
-                          float* states_out, void* workspace, size_t workspace_bytes, int32_t* status_dev,
-                          domino_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// Teacher forcing with fp32 or bf16 logits (logits_dtype: DOMINO_DTYPE_F32 or DOMINO_DTYPE_BF16).
+int teacher_forced_impl(const domino_shape_t* shape, const domino_weights_t* w, const void* base_logits,
+                        const void* hidden, const float* S0, const int32_t* tokens, void* logits_out,
+                        int logits_dtype, float* states_out, void* workspace, size_t workspace_bytes,
+                        int32_t* status_dev, domino_stream_t stream) {
   int rc = check_shape(shape);
   if (rc != DOMINO_OK) return rc;
   if ((rc = check_weights(w)) != DOMINO_OK) return rc;
@@ -372,6 +377,9 @@ int domino_teacher_forced(const domino_shape_t* shape, const domino_weights_t* w
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
 
   const size_t BL = (size_t)s.B * s.L;
+  // bf16 logits come from the tensor-core W2 product only
+  const bool tc_w2 = s.dtype == DOMINO_DTYPE_BF16 && gemm_tc_supported(s.V, (int)BL, s.r, w->W2, ws.u16);
+  if (logits_dtype == DOMINO_DTYPE_BF16 && !tc_w2) return DOMINO_ERR_UNSUPPORTED;
   float* SB = states_out ? states_out : ws.states;  // [B][L][Hs]
   const size_t row = (size_t)s.L * s.Hs;
   using bf = __nv_bfloat16;
@@ -424,7 +432,6 @@ int domino_teacher_forced(const domino_shape_t* shape, const domino_weights_t* w
   }  // per-update recurrence
   // W2 product over all B*L positions at once: a tcgen05 GEMM with the L_base add fused into its
   // epilogue (activations rounded to bf16 for the tensor cores), or the CUDA-core kernel.
-  const bool tc_w2 = s.dtype == DOMINO_DTYPE_BF16 && gemm_tc_supported(s.V, (int)BL, s.r, w->W2, ws.u16);
   if (e == cudaSuccess && tc && tc_w2) {  // u for every position: one GEMM on the split of all states
     e = launch_split_state(SB, s.Hs, (int)BL, s.Hs, ws.S_hl, cs);
     if (e == cudaSuccess)
@@ -436,11 +443,32 @@ int domino_teacher_forced(const domino_shape_t* shape, const domino_weights_t* w
   if (e == cudaSuccess) {
     if (tc_w2)
       e = gemm_tc_logits((const __nv_bfloat16*)w->W2, ws.u16, s.V, (int)BL, s.r, (const __nv_bfloat16*)base_logits,
-                         logits_out, st, spin_limit(), cs);
+                         logits_out, logits_dtype == DOMINO_DTYPE_BF16, st, spin_limit(), cs);
     else
-      e = launch_w2(s, w->W2, ws.u, (int)BL, base_logits, 1, 0, nullptr, logits_out, cs);
+      e = launch_w2(s, w->W2, ws.u, (int)BL, base_logits, 1, 0, nullptr, static_cast<float*>(logits_out), cs);
   }
   return cuda_rc(e);
+}
+
+}  // namespace
+
+extern "C" {
+
+int domino_teacher_forced(const domino_shape_t* shape, const domino_weights_t* w, const void* base_logits,
+                          const void* hidden, const float* S0, const int32_t* tokens, float* logits_out,
+                          float* states_out, void* workspace, size_t workspace_bytes, int32_t* status_dev,
+                          domino_stream_t stream) {
+  return teacher_forced_impl(shape, w, base_logits, hidden, S0, tokens, logits_out, DOMINO_DTYPE_F32, states_out,
+                             workspace, workspace_bytes, status_dev, stream);
+}
+
+int domino_teacher_forced_ex(const domino_shape_t* shape, const domino_weights_t* w, const void* base_logits,
+                             const void* hidden, const float* S0, const int32_t* tokens, void* logits_out,
+                             int32_t logits_dtype, float* states_out, void* workspace, size_t workspace_bytes,
+                             int32_t* status_dev, domino_stream_t stream) {
+  if (logits_dtype != DOMINO_DTYPE_F32 && logits_dtype != DOMINO_DTYPE_BF16) return DOMINO_ERR_INVALID_ARGUMENT;
+  return teacher_forced_impl(shape, w, base_logits, hidden, S0, tokens, logits_out, logits_dtype, states_out,
+                             workspace, workspace_bytes, status_dev, stream);
 }
 
 int domino_accept_len(int32_t B, int32_t L, int32_t V, const int32_t* draft_tokens, const float* target_logits,

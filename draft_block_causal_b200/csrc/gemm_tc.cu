@@ -41,6 +41,7 @@
 
 #include <atomic>
 #include <mutex>
+#include <type_traits>
 
 namespace domino {
 
@@ -50,8 +51,15 @@ constexpr int kBM = 128, kBK = 64;
 // Warps 0 and 1 produce and issue; 4 * kGroups epilogue warps follow (two warps per TMEM lane
 // quadrant, each on half of the tile's columns, for the argmax epilogue whose per-tile work is the
 // longest; one per quadrant otherwise).
+// An epilogue may state its group count (kGroups); otherwise the side-tile epilogues take two.
+template <class Epi, class = void> struct GroupsOf {
+  static constexpr int value = Epi::kSide ? 2 : 1;
+};
+template <class Epi> struct GroupsOf<Epi, std::void_t<decltype(Epi::kGroups)>> {
+  static constexpr int value = Epi::kGroups;
+};
 template <class Epi> struct EpiWarps {
-  static constexpr int kGroups = Epi::kSide ? 2 : 1;
+  static constexpr int kGroups = GroupsOf<Epi>::value;
   static constexpr int kThreads = 64 + 128 * kGroups;
 };
 constexpr uint32_t kABytes = kBM * kBK * 2;
@@ -99,12 +107,17 @@ struct EpiStore {  // out[m * ldo + n] = D, or out[n * ldo + m] = D when trans
     }
   }
 };
-struct EpiLogits {  // logits[n][m] = D + Lb[n][m]   (m = vocabulary row, n = (row, position))
+// Output element conversion of the logits epilogues (fp32, or bf16 rounded to nearest even).
+__device__ __forceinline__ void put(float* p, float v) { *p = v; }
+__device__ __forceinline__ void put(bf16* p, float v) { *p = __float2bfloat16_rn(v); }
+
+template <typename OutT>
+struct EpiLogitsT {  // logits[n][m] = D + Lb[n][m]   (m = vocabulary row, n = (row, position))
   static constexpr bool kSide = false;
   static constexpr bool kARes = false;
   using State = NoState;
   const bf16* Lb;
-  float* logits;
+  OutT* logits;
   int M;
   __device__ __forceinline__ void init(State&) const {}
   __device__ __forceinline__ void finish(State&, int) const {}
@@ -118,22 +131,22 @@ struct EpiLogits {  // logits[n][m] = D + Lb[n][m]   (m = vocabulary row, n = (r
     for (int j = 0; j < 16; ++j) l[j] = (n0 + j < N) ? __bfloat162float(__ldg(Lb + (size_t)(n0 + j) * M + m)) : 0.f;
 #pragma unroll
     for (int j = 0; j < 16; ++j)
-      if (n0 + j < N) logits[(size_t)(n0 + j) * M + m] = v[j] + l[j];
+      if (n0 + j < N) put(logits + (size_t)(n0 + j) * M + m, v[j] + l[j]);
   }
 };
 
 // Teacher-forced logits, row-major: m = row (b, i) < M, n = vocabulary column < N:
 //   logits[m * ld + n] = D + Lb[m * ld + n]
-// Each thread owns 16 consecutive columns of one row: two 16-byte loads and four 16-byte stores
-// (rows are 16-byte aligned since V % 8 == 0; n0 is a multiple of 16).
-struct EpiLogitsRow {
+// Each thread owns 16 consecutive columns of one row: two 16-byte loads and four (fp32) or two
+// (bf16) 16-byte stores (rows are 16-byte aligned since V % 8 == 0; n0 is a multiple of 16).
+template <typename OutT>
+struct EpiLogitsRowT {
   static constexpr bool kSide = false;
   static constexpr bool kARes = false;
-  static constexpr bool kSideL2 = false;
   static constexpr int kGroups = 2;  // the epilogue is the longest phase of a tile: two warps per lane quadrant
   using State = NoState;
   const bf16* Lb;
-  float* logits;
+  OutT* logits;
   int M;
   long long ld;
   __device__ __forceinline__ void init(State&) const {}
@@ -142,23 +155,35 @@ struct EpiLogitsRow {
                                         int) const {
     if (m >= M) return;
     const bf16* lr = Lb + (size_t)m * ld + n0;
-    float* o = logits + (size_t)m * ld + n0;
+    OutT* o = logits + (size_t)m * ld + n0;
     if (n0 + 16 <= N) {
-      float a[8], b[8];
+      float a[8], b[8], z[16];
       widen(__ldg(reinterpret_cast<const uint4*>(lr)), a);
       widen(__ldg(reinterpret_cast<const uint4*>(lr) + 1), b);
-      float4* o4 = reinterpret_cast<float4*>(o);
-      o4[0] = make_float4(v[0] + a[0], v[1] + a[1], v[2] + a[2], v[3] + a[3]);
-      o4[1] = make_float4(v[4] + a[4], v[5] + a[5], v[6] + a[6], v[7] + a[7]);
-      o4[2] = make_float4(v[8] + b[0], v[9] + b[1], v[10] + b[2], v[11] + b[3]);
-      o4[3] = make_float4(v[12] + b[4], v[13] + b[5], v[14] + b[6], v[15] + b[7]);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) { z[j] = v[j] + a[j]; z[8 + j] = v[8 + j] + b[j]; }
+      if constexpr (std::is_same<OutT, float>::value) {
+        float4* o4 = reinterpret_cast<float4*>(o);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) o4[q] = make_float4(z[4 * q], z[4 * q + 1], z[4 * q + 2], z[4 * q + 3]);
+      } else {
+        uint32_t w[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const __nv_bfloat162 pr = __floats2bfloat162_rn(z[2 * q], z[2 * q + 1]);
+          w[q] = *reinterpret_cast<const uint32_t*>(&pr);
+        }
+        uint4* o4 = reinterpret_cast<uint4*>(o);
+        o4[0] = make_uint4(w[0], w[1], w[2], w[3]);
+        o4[1] = make_uint4(w[4], w[5], w[6], w[7]);
+      }
     } else {
       float l[16];
 #pragma unroll
       for (int j = 0; j < 16; ++j) l[j] = (n0 + j < N) ? __bfloat162float(lr[j]) : 0.f;
 #pragma unroll
       for (int j = 0; j < 16; ++j)
-        if (n0 + j < N) o[j] = v[j] + l[j];
+        if (n0 + j < N) put(o + j, v[j] + l[j]);
     }
   }
 };
@@ -1091,14 +1116,21 @@ cudaError_t gemm_tc_store_f32_t(const bf16* A, const bf16* Bm, int M, int N, int
   return launch_gemm_skinny(A, Bm, M, N, K, e, status, limit, st, (uint64_t)lda, a_kwrap, nullptr, 0, 0, a_stream);
 }
 
-cudaError_t gemm_tc_logits(const bf16* W2, const bf16* U, int V, int N, int r, const bf16* Lb, float* logits,
-                           int32_t* status, uint64_t limit, cudaStream_t st) {
+template <typename OutT>
+cudaError_t logits_t(const bf16* W2, const bf16* U, int V, int N, int r, const bf16* Lb, OutT* logits, int32_t* status,
+                     uint64_t limit, cudaStream_t st) {
   if (N >= 64) {  // enough rows for the row-major orientation: vector loads and stores in the epilogue
-    EpiLogitsRow e{Lb, logits, N, (long long)V};
+    EpiLogitsRowT<OutT> e{Lb, logits, N, (long long)V};
     return launch_gemm<256>(U, W2, N, V, r, e, status, limit, st, 0, 0, 0, nullptr, 0, nullptr, 0, 0, 1, 0, 2);
   }
-  EpiLogits e{Lb, logits, V};
+  EpiLogitsT<OutT> e{Lb, logits, V};
   return launch_gemm_bn(W2, U, V, N, r, e, status, limit, st);
+}
+
+cudaError_t gemm_tc_logits(const bf16* W2, const bf16* U, int V, int N, int r, const bf16* Lb, void* logits,
+                           int out_bf16, int32_t* status, uint64_t limit, cudaStream_t st) {
+  return out_bf16 ? logits_t(W2, U, V, N, r, Lb, static_cast<bf16*>(logits), status, limit, st)
+                  : logits_t(W2, U, V, N, r, Lb, static_cast<float*>(logits), status, limit, st);
 }
 
 }  // namespace domino

@@ -65,8 +65,10 @@ cudaError_t gemm_tc_debug(const __nv_bfloat16* A, const __nv_bfloat16* Bm, int M
 // The automatic skinny plan for an M x N x K product (tile width bn, K split ks).
 void gemm_tc_skinny_plan(int M, int N, int K, int* bn, int* ks);
 
-// logits[n][v] = Lb[n][v] + sum_k W2[v][k] U[n][k]   (W2 [V x r], U [N x r], Lb [N x V] bf16)
+// logits[n][v] = Lb[n][v] + sum_k W2[v][k] U[n][k]   (W2 [V x r], U [N x r], Lb [N x V] bf16); logits
+// fp32, or bf16 (round to nearest even) when out_bf16
 cudaError_t gemm_tc_logits(const __nv_bfloat16* W2, const __nv_bfloat16* U, int V, int N, int r,
-                           const __nv_bfloat16* Lb, float* logits, int32_t* status, uint64_t limit, cudaStream_t st);
+                           const __nv_bfloat16* Lb, void* logits, int out_bf16, int32_t* status, uint64_t limit,
+                           cudaStream_t st);
 
 }  // namespace domino

@@ -38,7 +38,7 @@ EXPORTS = ("domino_workspace_bytes", "domino_draft_greedy", "domino_teacher_forc
            "domino_greedy_plan", "domino_draft_greedy_noalloc", "domino_debug_set_trace",
            "domino_embed_proj_bytes", "domino_project_embeddings", "domino_arena_bytes",
            "domino_pack_weights", "domino_set_l2_persistence", "domino_debug_gemm",
-           "domino_debug_read_passes")
+           "domino_debug_read_passes", "domino_teacher_forced_ex")
 
 
 class DominoError(RuntimeError):
@@ -106,6 +106,9 @@ def lib(path: str = LIB_PATH) -> ctypes.CDLL:
         L.domino_set_l2_persistence.restype = ctypes.c_int
         L.domino_debug_gemm.argtypes = [vp, vp, i32, i32, i32, i32, vp, ctypes.c_int64, i32, i32, i32, vp, vp]
         L.domino_debug_gemm.restype = ctypes.c_int
+        L.domino_teacher_forced_ex.argtypes = [ctypes.POINTER(Shape), ctypes.POINTER(Weights), vp, vp, vp, vp, vp,
+                                               i32, vp, vp, sz, vp, vp]
+        L.domino_teacher_forced_ex.restype = ctypes.c_int
         L.domino_debug_read_passes.argtypes = [vp, sz, i32, vp]
         L.domino_debug_read_passes.restype = ctypes.c_int
         _lib = L
@@ -349,12 +352,15 @@ def draft_greedy_noalloc(w: HeadWeights, base_logits, hidden, S0, tokens_out=Non
 
 
 def teacher_forced(w: HeadWeights, base_logits, hidden, S0, tokens, logits_out=None, states_out=None,
-                   workspace=None, status=None, stream=None):
-    """Teacher-forced logits (``domino_teacher_forced``); returns (logits, states or None)."""
+                   workspace=None, status=None, stream=None, logits_dtype=torch.float32):
+    """Teacher-forced logits (``domino_teacher_forced``, or ``domino_teacher_forced_ex`` for bf16
+    logits: ``logits_dtype=torch.bfloat16``); returns (logits, states or None)."""
     B, L, V = base_logits.shape
     dev = base_logits.device
     if logits_out is None:
-        logits_out = torch.empty((B, L, V), dtype=torch.float32, device=dev)
+        logits_out = torch.empty((B, L, V), dtype=logits_dtype, device=dev)
+    if logits_out.dtype not in (torch.float32, torch.bfloat16):
+        raise ValueError("logits_out must be float32 or bfloat16")
     if states_out is True:
         states_out = torch.empty((B, L, w.W_hh.shape[1]), dtype=torch.float32, device=dev)
     if states_out is False:
@@ -363,10 +369,16 @@ def teacher_forced(w: HeadWeights, base_logits, hidden, S0, tokens, logits_out=N
     if workspace is None:
         workspace = alloc_workspace(workspace_bytes(w, B, L), dev)
     ws = w.c_struct()
-    rc = lib().domino_teacher_forced(ctypes.byref(sh), ctypes.byref(ws), _ptr(base_logits), _ptr(hidden), _ptr(S0),
-                                     _ptr(tokens), _ptr(logits_out), _ptr(states_out), _ptr(workspace),
-                                     workspace.numel(), _ptr(status), _stream(stream))
-    _check(rc, "domino_teacher_forced")
+    if logits_out.dtype == torch.float32:
+        rc = lib().domino_teacher_forced(ctypes.byref(sh), ctypes.byref(ws), _ptr(base_logits), _ptr(hidden),
+                                         _ptr(S0), _ptr(tokens), _ptr(logits_out), _ptr(states_out),
+                                         _ptr(workspace), workspace.numel(), _ptr(status), _stream(stream))
+        _check(rc, "domino_teacher_forced")
+    else:
+        rc = lib().domino_teacher_forced_ex(ctypes.byref(sh), ctypes.byref(ws), _ptr(base_logits), _ptr(hidden),
+                                            _ptr(S0), _ptr(tokens), _ptr(logits_out), DTYPE_BF16, _ptr(states_out),
+                                            _ptr(workspace), workspace.numel(), _ptr(status), _stream(stream))
+        _check(rc, "domino_teacher_forced_ex")
     return logits_out, states_out
 
 

@@ -141,3 +141,19 @@ def test_read_passes_argument_checks(L):
     assert L.domino_debug_read_passes(ctypes.c_void_p(0x10004), 1 << 20, 1, None) == domino.ERR_INVALID_ARGUMENT
     assert L.domino_debug_read_passes(ctypes.c_void_p(0x10000), 1 << 20, 0, None) == domino.ERR_INVALID_ARGUMENT
     assert L.domino_debug_read_passes(ctypes.c_void_p(0x10000), 8, 1, None) == domino.ERR_INVALID_ARGUMENT
+
+
+def test_teacher_forced_ex_rejects_a_bad_logits_dtype(L):
+    sh = _shape()
+    fake = ctypes.c_void_p(0x10000)
+    w = domino.Weights(*([0x10000] * 7))
+    n = L.domino_workspace_bytes(ctypes.byref(sh))
+    for bad in (-1, 2, 7):
+        assert L.domino_teacher_forced_ex(ctypes.byref(sh), ctypes.byref(w), fake, fake, fake, fake, fake,
+                                          ctypes.c_int32(bad), None, fake, n, None,
+                                          None) == domino.ERR_INVALID_ARGUMENT
+    # bf16 logits with fp32 storage: unsupported, refused on the host
+    sh32 = _shape(dtype=0)
+    n32 = L.domino_workspace_bytes(ctypes.byref(sh32))
+    assert L.domino_teacher_forced_ex(ctypes.byref(sh32), ctypes.byref(w), fake, fake, fake, fake, fake,
+                                      ctypes.c_int32(1), None, fake, n32, None, None) == domino.ERR_UNSUPPORTED

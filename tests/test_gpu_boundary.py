@@ -211,3 +211,17 @@ def test_batched_teacher_forcing_reports_bad_tokens():
     domino.teacher_forced(w, lb, h, S0, y, status=status)
     torch.cuda.synchronize()
     assert int(status.item()) == domino.STATUS_BAD_TOKEN
+
+
+@pytest.mark.parametrize("B", [1, 8], ids=["vocabulary-major", "row-major"])
+def test_bf16_teacher_forced_logits_are_the_fp32_ones_rounded(B):
+    """domino_teacher_forced_ex with bf16 logits writes exactly the fp32 logits of the same call
+    rounded to nearest even (both logits epilogues: B*L < 64 and >= 64)."""
+    data = _persistent_case(B=B, seed=350 + B, Hs=256)
+    w, lb, h, S0 = G.device_inputs(data)
+    y = torch.randint(0, data["shape"]["V"], (B, 16), dtype=torch.int32, device="cuda")
+    lg32, _ = domino.teacher_forced(w, lb, h, S0, y)
+    lg16, _ = domino.teacher_forced(w, lb, h, S0, y, logits_dtype=torch.bfloat16)
+    torch.cuda.synchronize()
+    assert lg16.dtype == torch.bfloat16
+    assert torch.equal(lg16, lg32.to(torch.bfloat16))

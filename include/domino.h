@@ -96,18 +96,6 @@ typedef struct {
   const float* embed_proj;
 } domino_weights_t;
 
-/* domino_teacher_forced with a choice of logits storage: logits_dtype DOMINO_DTYPE_F32 (logits_out
- * is float [B, L, V], as domino_teacher_forced) or DOMINO_DTYPE_BF16 (logits_out is bf16 [B, L, V],
- * each value the fp32 logit rounded to nearest even: half the bytes of the largest output).
- * bf16 logits need bf16 storage (shape->dtype) and the tensor-core W2 product, else
- * DOMINO_ERR_UNSUPPORTED; another logits_dtype gives DOMINO_ERR_INVALID_ARGUMENT.  Nothing is
- * launched when a negative code is returned. */
-DOMINO_API int domino_teacher_forced_ex(const domino_shape_t* shape, const domino_weights_t* weights,
-                                        const void* base_logits, const void* hidden, const float* S0,
-                                        const int32_t* tokens, void* logits_out, int32_t logits_dtype,
-                                        float* states_out, void* workspace, size_t workspace_bytes,
-                                        int32_t* status_dev, domino_stream_t stream);
-
 /* Bytes of the optional input-projection table (V * 3Hs * 4), or 0 for an invalid shape. */
 DOMINO_API size_t domino_embed_proj_bytes(const domino_shape_t* shape);
 
@@ -192,6 +180,18 @@ DOMINO_API int domino_teacher_forced(const domino_shape_t* shape, const domino_w
                           const int32_t* tokens, float* logits_out, float* states_out,
                           void* workspace, size_t workspace_bytes, int32_t* status_dev,
                           domino_stream_t stream);
+
+/* domino_teacher_forced with a choice of logits storage: logits_dtype DOMINO_DTYPE_F32 (logits_out
+ * is float [B, L, V], as domino_teacher_forced) or DOMINO_DTYPE_BF16 (logits_out is bf16 [B, L, V],
+ * each value the fp32 logit rounded to nearest even: half the bytes of the largest output).
+ * bf16 logits need bf16 storage (shape->dtype) and the tensor-core W2 product, else
+ * DOMINO_ERR_UNSUPPORTED; another logits_dtype gives DOMINO_ERR_INVALID_ARGUMENT.  Nothing is
+ * launched when a negative code is returned. */
+DOMINO_API int domino_teacher_forced_ex(const domino_shape_t* shape, const domino_weights_t* weights,
+                                        const void* base_logits, const void* hidden, const float* S0,
+                                        const int32_t* tokens, void* logits_out, int32_t logits_dtype,
+                                        float* states_out, void* workspace, size_t workspace_bytes,
+                                        int32_t* status_dev, domino_stream_t stream);
 
 /* Greedy accept length (the accept-length metric of the review page, section 四; the target
  * verifies the whole block in one pass and keeps the longest agreeing prefix, sections 一 and

@@ -1,7 +1,7 @@
 /*
  * domino_oracle.c -- fp64 CPU oracle of the Domino head.  TEST INFRASTRUCTURE ONLY.
  *
- * This file is the checker, not the product.  Only the tests, the package's smoke() and
+ * This file is test infrastructure, not the product.  Only the tests, the package's smoke() and
  * bench.py's CPU-baseline leg may load it.  It shares no code, header, table or helper with
  * the CUDA library; the two meet only through the seeded input arrays.
  *

@@ -1,6 +1,6 @@
-"""The bench's roofline arithmetic on CPU, against the figures the survey of the method derives
-for the Qwen3-8B-shaped head (16-token block, Hs = 1024, r = 256, V = 151936): algorithmic bytes
-of a greedy call with no reuse, unique (first-touch) bytes, and FLOPs per call."""
+"""The bench's roofline arithmetic on CPU, against figures worked out by hand from the
+Qwen3-8B-shaped head (16-token block, Hs = 1024, r = 256, V = 151936): algorithmic bytes of a
+greedy call with no reuse, unique (first-touch) bytes, and FLOPs per call."""
 import os
 import sys
 

@@ -157,3 +157,54 @@ def test_teacher_forced_ex_rejects_a_bad_logits_dtype(L):
     n32 = L.domino_workspace_bytes(ctypes.byref(sh32))
     assert L.domino_teacher_forced_ex(ctypes.byref(sh32), ctypes.byref(w), fake, fake, fake, fake, fake,
                                       ctypes.c_int32(1), None, fake, n32, None, None) == domino.ERR_UNSUPPORTED
+
+
+def test_noalloc_limits_are_checked_on_the_host(L):
+    w = domino.Weights(*([0x10000] * 7))
+    p = ctypes.c_void_p(0x10000)  # never dereferenced: every case fails before any launch
+    # B = 4 rows of 64 positions need more than the 1 MiB scratch array
+    big = domino.Shape(4, 64, 512, 256, 256, 12000, 1)
+    assert L.domino_draft_greedy_noalloc(ctypes.byref(big), ctypes.byref(w), p, p, p, p, None, None, None,
+                                         None) == domino.ERR_SCRATCH_LIMIT
+    # shapes the fused small-batch kernel does not take: a larger batch, fp32 storage, another rank
+    for bad in (domino.Shape(8, 16, 512, 256, 256, 12000, 1), domino.Shape(1, 16, 512, 256, 256, 12000, 0),
+                domino.Shape(1, 16, 512, 256, 128, 12000, 1)):
+        assert L.domino_draft_greedy_noalloc(ctypes.byref(bad), ctypes.byref(w), p, p, p, p, None, None, None,
+                                             None) == domino.ERR_UNSUPPORTED
+    ok = domino.Shape(1, 16, 512, 256, 256, 12000, 1)
+    assert L.domino_draft_greedy_noalloc(ctypes.byref(ok), None, p, p, p, p, None, None, None,
+                                         None) == domino.ERR_INVALID_ARGUMENT
+    assert L.domino_draft_greedy_noalloc(ctypes.byref(ok), ctypes.byref(w), p, p, p, None, None, None, None,
+                                         None) == domino.ERR_INVALID_ARGUMENT  # tokens_out is required
+
+
+def test_projection_and_debug_entry_points_check_their_arguments(L):
+    sh = _shape()
+    w = domino.Weights(*([0x10000] * 7))
+    assert L.domino_embed_proj_bytes(ctypes.byref(sh)) == 151936 * 3 * 1024 * 4
+    assert L.domino_embed_proj_bytes(ctypes.byref(_shape(V=999))) == 0
+    # the table pointer is required and must be 16-byte aligned
+    assert L.domino_project_embeddings(ctypes.byref(sh), ctypes.byref(w), None, None,
+                                       None) == domino.ERR_INVALID_ARGUMENT
+    assert L.domino_project_embeddings(ctypes.byref(sh), ctypes.byref(w), ctypes.c_void_p(0x10004), None,
+                                       None) == domino.ERR_INVALID_ARGUMENT
+    a = ctypes.c_void_p(0x10000)
+    i64 = ctypes.c_int64
+    # K must be a positive multiple of 64, the wrap a divisor of K and a multiple of 64
+    for M, N, K, wrap in ((128, 16, 100, 0), (128, 16, 0, 0), (128, 16, 256, 96), (128, 16, 192, 128), (0, 16, 64, 0)):
+        assert L.domino_debug_gemm(a, a, M, N, K, wrap, a, i64(128), 0, 0, 0, None,
+                                   None) == domino.ERR_INVALID_ARGUMENT, (M, N, K, wrap)
+    # output stride shorter than a row, misaligned output, unknown tile width or split
+    assert L.domino_debug_gemm(a, a, 128, 16, 64, 0, a, i64(8), 0, 0, 0, None, None) == domino.ERR_INVALID_ARGUMENT
+    assert L.domino_debug_gemm(a, a, 128, 16, 64, 0, ctypes.c_void_p(0x10008), i64(16), 0, 0, 0, None,
+                               None) == domino.ERR_INVALID_ARGUMENT
+    for bn, ks in ((48, 1), (64, 0), (64, 9), (0, 2)):
+        assert L.domino_debug_gemm(a, a, 128, 16, 64, 0, a, i64(16), 0, bn, ks, None,
+                                   None) == domino.ERR_INVALID_ARGUMENT, (bn, ks)
+    # the trace hook wants an 8-byte aligned buffer and a positive length; NULL turns it off
+    assert L.domino_debug_set_trace(ctypes.c_void_p(0x10004), 16) == domino.ERR_INVALID_ARGUMENT
+    assert L.domino_debug_set_trace(ctypes.c_void_p(0x10000), 0) == domino.ERR_INVALID_ARGUMENT
+    assert L.domino_debug_set_trace(None, 0) == domino.OK
+    # the plan text of an invalid shape, and the CUDA-core kernels of fp32 storage
+    assert L.domino_greedy_plan(ctypes.byref(_shape(B=0))) == b"invalid shape"
+    assert b"k_w2" in L.domino_greedy_plan(ctypes.byref(_shape(dtype=0)))

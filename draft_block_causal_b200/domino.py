@@ -156,9 +156,54 @@ def _ptr(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
-def _stream(stream):
-    s = torch.cuda.current_stream() if stream is None else stream
+def _stream(stream, device):
+    """The caller's stream (default: the current stream of `device`), which must belong to `device`."""
+    if device.type != "cuda":
+        raise ValueError(f"the call's tensors must be on a CUDA device, not {device}")
+    s = torch.cuda.current_stream(device) if stream is None else stream
+    if s.device != device:
+        raise ValueError(f"stream is on {s.device}, the call's tensors on {device}")
     return ctypes.c_void_p(s.cuda_stream)
+
+
+def _launch(device, fn, *args):
+    """Call a library entry point with `device` current: the library queries and launches on the
+    current device, which must be the one that holds the call's memory."""
+    if torch.cuda.current_device() == device.index:
+        return fn(*args)
+    with torch.cuda.device(device):
+        return fn(*args)
+
+
+def _expect(t, name: str, shape, dtype, device) -> None:
+    """The library sees only a pointer: check here that a tensor has the exact shape, dtype,
+    contiguity and device the call reads or writes, so that no kernel touches memory outside it."""
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor, got {type(t).__name__}")
+    if t.shape != shape:  # torch.Size compares equal to a tuple of ints
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(int(x) for x in shape)}")
+    if t.dtype is not dtype and not (isinstance(dtype, tuple) and t.dtype in dtype):
+        dts = dtype if isinstance(dtype, tuple) else (dtype,)
+        raise ValueError(f"{name} has dtype {t.dtype}, expected {' or '.join(str(d) for d in dts)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+
+
+def _expect_status(status, device) -> None:
+    if status is not None:
+        if not isinstance(status, torch.Tensor) or status.dtype != torch.int32 or status.numel() < 1:
+            raise ValueError("status must be an int32 tensor with at least one element")
+        if status.device != device:
+            raise ValueError(f"status is on {status.device}, expected {device}")
+
+
+def _expect_workspace(ws, device) -> None:
+    if not isinstance(ws, torch.Tensor) or ws.dtype != torch.uint8 or ws.dim() != 1 or not ws.is_contiguous():
+        raise ValueError("workspace must be a contiguous 1-D uint8 tensor (see alloc_workspace)")
+    if ws.device != device:
+        raise ValueError(f"workspace is on {ws.device}, expected {device}")
 
 
 @dataclass
@@ -190,16 +235,54 @@ class HeadWeights:
         r = self.W2.shape[1]
         return d, Hs, r, V
 
+    def check(self) -> None:
+        """Every weight has the shape the dimensions of embed, W_hh and W2 imply, the storage type
+        of W2, and the device of W2."""
+        d, Hs, r, V = self.dims()
+        dev = self.W2.device
+        want = {"embed": (V, d), "W_ih": (3 * Hs, d), "W_hh": (3 * Hs, Hs), "b_ih": (3 * Hs,), "b_hh": (3 * Hs,),
+                "W1": (r, d + Hs), "W2": (V, r)}
+        for n, shp in want.items():
+            _expect(getattr(self, n), f"weight {n}", shp, self.W2.dtype, dev)
+        if self.embed_proj is not None:
+            _expect(self.embed_proj, "embed_proj", (V, 3 * Hs), torch.float32, dev)
+
+    def __post_init__(self):
+        self.check()
+        object.__setattr__(self, "_checked", True)
+
+    def __setattr__(self, name, value):
+        # a replaced weight is checked against the others at once (every call relies on it); a
+        # rejected one leaves the previous value in place
+        old = self.__dict__.get(name)
+        object.__setattr__(self, name, value)
+        if self.__dict__.get("_checked"):
+            try:
+                self.check()
+            except Exception:
+                object.__setattr__(self, name, old)
+                raise
+
     def c_struct(self) -> Weights:
         for n in ("embed", "W_ih", "W_hh", "b_ih", "b_hh", "W1", "W2"):
-            t = getattr(self, n)
-            if not t.is_contiguous() or t.dtype != self.W2.dtype or not t.is_cuda:
-                raise ValueError(f"weight {n} must be a contiguous CUDA tensor of dtype {self.W2.dtype}")
+            if not getattr(self, n).is_cuda:
+                raise ValueError(f"weight {n} must be a CUDA tensor")
         xp = self.embed_proj
-        if xp is not None and (xp.dtype != torch.float32 or not xp.is_contiguous() or not xp.is_cuda):
-            raise ValueError("embed_proj must be a contiguous CUDA float32 tensor [V, 3Hs]")
         ptrs = [self.__dict__[n].data_ptr() for n in ("embed", "W_ih", "W_hh", "b_ih", "b_hh", "W1", "W2")]
         return Weights(*ptrs, xp.data_ptr() if xp is not None else None)
+
+
+def _check_head_inputs(w: HeadWeights, base_logits, hidden, S0):
+    """The inputs every head call reads; returns (B, L, device)."""
+    d, Hs, r, V = w.dims()
+    dev = w.W2.device
+    if not isinstance(base_logits, torch.Tensor) or base_logits.dim() != 3:
+        raise ValueError("base_logits must be a [B, L, V] tensor")
+    B, L = int(base_logits.shape[0]), int(base_logits.shape[1])
+    _expect(base_logits, "base_logits", (B, L, V), w.W2.dtype, dev)
+    _expect(hidden, "hidden", (B, L, d), w.W2.dtype, dev)
+    _expect(S0, "S0", (B, Hs), torch.float32, dev)
+    return B, L, dev
 
 
 def make_shape(w: HeadWeights, B: int, L: int) -> Shape:
@@ -220,9 +303,13 @@ def project_embeddings(w: HeadWeights, out=None, status=None, stream=None) -> to
     d, Hs, r, V = w.dims()
     if out is None:
         out = torch.empty((V, 3 * Hs), dtype=torch.float32, device=w.W2.device)
+    _expect(out, "out", (V, 3 * Hs), torch.float32, w.W2.device)
+    _expect_status(status, w.W2.device)
     sh = make_shape(w, 1, 1)
     ws = w.c_struct()
-    rc = lib().domino_project_embeddings(ctypes.byref(sh), ctypes.byref(ws), _ptr(out), _ptr(status), _stream(stream))
+    dev = w.W2.device
+    rc = _launch(dev, lib().domino_project_embeddings, ctypes.byref(sh), ctypes.byref(ws), _ptr(out), _ptr(status),
+                 _stream(stream, dev))
     _check(rc, "domino_project_embeddings")
     return out
 
@@ -242,8 +329,8 @@ def pack_weights(w: HeadWeights, stream=None) -> HeadWeights:
     sh = make_shape(w, 1, 1)
     src = w.c_struct()
     out = Weights()
-    rc = lib().domino_pack_weights(ctypes.byref(sh), ctypes.byref(src), ctypes.c_void_p(arena.data_ptr()),
-                                   nbytes, ctypes.byref(out), _stream(stream))
+    rc = _launch(w.W2.device, lib().domino_pack_weights, ctypes.byref(sh), ctypes.byref(src),
+                 ctypes.c_void_p(arena.data_ptr()), nbytes, ctypes.byref(out), _stream(stream, w.W2.device))
     _check(rc, "domino_pack_weights")
     dt = w.W2.dtype
     es = torch.empty((), dtype=dt).element_size()
@@ -262,7 +349,8 @@ def set_l2_persistence(w: HeadWeights, stream, hit_ratio: float = 1.0) -> None:
     ``hit_ratio=0`` clears it and restores the context's persisting-L2 set-aside."""
     sh = make_shape(w, 1, 1)
     ws = w.c_struct()
-    rc = lib().domino_set_l2_persistence(ctypes.byref(sh), ctypes.byref(ws), _stream(stream), float(hit_ratio))
+    rc = _launch(w.W2.device, lib().domino_set_l2_persistence, ctypes.byref(sh), ctypes.byref(ws),
+                 _stream(stream, w.W2.device), float(hit_ratio))
     _check(rc, "domino_set_l2_persistence")
 
 
@@ -270,17 +358,22 @@ def debug_gemm(A, B, out=None, trans=False, a_kwrap=0, bn=0, ks=0, status=None, 
     """The tensor-core GEMM engine on its own (domino_debug_gemm): fp32 A[:, k mod K'] . B^T for bf16
     A [M, K'] and B [N, K]; [M, N], or [N, M] when ``trans``.  bn/ks force a plan (0, 0: automatic)."""
     M, N, K = A.shape[0], B.shape[0], B.shape[1]
+    _expect(A, "A", (M, int(a_kwrap) or K), torch.bfloat16, A.device)
+    _expect(B, "B", (N, K), torch.bfloat16, A.device)
     if out is None:
         out = torch.empty((N, M) if trans else (M, N), dtype=torch.float32, device=A.device)
-    rc = lib().domino_debug_gemm(_ptr(A), _ptr(B), M, N, K, int(a_kwrap), _ptr(out), out.shape[1], int(bool(trans)),
-                                 int(bn), int(ks), _ptr(status), _stream(stream))
+    _expect(out, "out", (N, M) if trans else (M, N), torch.float32, A.device)
+    _expect_status(status, A.device)
+    rc = _launch(A.device, lib().domino_debug_gemm, _ptr(A), _ptr(B), M, N, K, int(a_kwrap), _ptr(out), out.shape[1],
+                 int(bool(trans)), int(bn), int(ks), _ptr(status), _stream(stream, A.device))
     _check(rc, "domino_debug_gemm")
     return out
 
 
 def debug_read_passes(buf, passes: int, stream=None) -> None:
     """Re-read a device buffer `passes` times in one launch (domino_debug_read_passes)."""
-    rc = lib().domino_debug_read_passes(_ptr(buf), buf.numel() * buf.element_size(), int(passes), _stream(stream))
+    rc = _launch(buf.device, lib().domino_debug_read_passes, _ptr(buf), buf.numel() * buf.element_size(), int(passes),
+                 _stream(stream, buf.device))
     _check(rc, "domino_debug_read_passes")
 
 
@@ -293,6 +386,14 @@ def alloc_workspace(nbytes: int, device=None) -> torch.Tensor:
     return torch.empty(int(nbytes), dtype=torch.uint8, device=device or "cuda")
 
 
+def _check_greedy_outputs(tokens_out, logits_out, states_out, B, L, Hs, V, dev) -> None:
+    _expect(tokens_out, "tokens_out", (B, L), torch.int32, dev)
+    if logits_out is not None:
+        _expect(logits_out, "logits_out", (B, L, V), torch.float32, dev)
+    if states_out is not None:
+        _expect(states_out, "states_out", (B, L, Hs), torch.float32, dev)
+
+
 def draft_greedy(w: HeadWeights, base_logits, hidden, S0, tokens_out=None, logits_out=None, states_out=None,
                  workspace=None, status=None, stream=None):
     """Greedy drafting (``domino_draft_greedy``); returns (tokens, logits or None, states or None).
@@ -300,25 +401,28 @@ def draft_greedy(w: HeadWeights, base_logits, hidden, S0, tokens_out=None, logit
     base_logits [B, L, V] and hidden [B, L, d] in the weights' storage type, S0 [B, Hs] fp32.
     Pass ``logits_out=True`` / ``states_out=True`` to have them allocated, or tensors to fill.
     """
-    B, L, V = base_logits.shape
-    dev = base_logits.device
+    B, L, dev = _check_head_inputs(w, base_logits, hidden, S0)
+    d, Hs, r, V = w.dims()
     if tokens_out is None:
         tokens_out = torch.empty((B, L), dtype=torch.int32, device=dev)
     if logits_out is True:
         logits_out = torch.empty((B, L, V), dtype=torch.float32, device=dev)
     if states_out is True:
-        states_out = torch.empty((B, L, w.W_hh.shape[1]), dtype=torch.float32, device=dev)
+        states_out = torch.empty((B, L, Hs), dtype=torch.float32, device=dev)
     if logits_out is False:
         logits_out = None
     if states_out is False:
         states_out = None
+    _check_greedy_outputs(tokens_out, logits_out, states_out, B, L, Hs, V, dev)
+    _expect_status(status, dev)
     sh = make_shape(w, B, L)
     if workspace is None:
         workspace = alloc_workspace(workspace_bytes(w, B, L), dev)
+    _expect_workspace(workspace, dev)
     ws = w.c_struct()
-    rc = lib().domino_draft_greedy(ctypes.byref(sh), ctypes.byref(ws), _ptr(base_logits), _ptr(hidden), _ptr(S0),
-                                   _ptr(tokens_out), _ptr(logits_out), _ptr(states_out), _ptr(workspace),
-                                   workspace.numel(), _ptr(status), _stream(stream))
+    rc = _launch(dev, lib().domino_draft_greedy, ctypes.byref(sh), ctypes.byref(ws), _ptr(base_logits), _ptr(hidden),
+                 _ptr(S0), _ptr(tokens_out), _ptr(logits_out), _ptr(states_out), _ptr(workspace), workspace.numel(),
+                 _ptr(status), _stream(stream, dev))
     _check(rc, "domino_draft_greedy")
     return tokens_out, logits_out, states_out
 
@@ -332,21 +436,23 @@ def draft_greedy_noalloc(w: HeadWeights, base_logits, hidden, S0, tokens_out=Non
     that array and race -- keep them on one stream.  Pass preallocated output tensors to keep the
     whole call free of allocations; ``logits_out=True`` / ``states_out=True`` allocate them here.
     """
-    B, L, V = base_logits.shape
-    dev = base_logits.device
+    B, L, dev = _check_head_inputs(w, base_logits, hidden, S0)
+    d, Hs, r, V = w.dims()
     if tokens_out is None:
         tokens_out = torch.empty((B, L), dtype=torch.int32, device=dev)
     if logits_out is True:
         logits_out = torch.empty((B, L, V), dtype=torch.float32, device=dev)
     if states_out is True:
-        states_out = torch.empty((B, L, w.W_hh.shape[1]), dtype=torch.float32, device=dev)
+        states_out = torch.empty((B, L, Hs), dtype=torch.float32, device=dev)
     logits_out = None if logits_out is False else logits_out
     states_out = None if states_out is False else states_out
+    _check_greedy_outputs(tokens_out, logits_out, states_out, B, L, Hs, V, dev)
+    _expect_status(status, dev)
     sh = make_shape(w, B, L)
     ws = w.c_struct()
-    rc = lib().domino_draft_greedy_noalloc(ctypes.byref(sh), ctypes.byref(ws), _ptr(base_logits), _ptr(hidden),
-                                           _ptr(S0), _ptr(tokens_out), _ptr(logits_out), _ptr(states_out),
-                                           _ptr(status), _stream(stream))
+    rc = _launch(dev, lib().domino_draft_greedy_noalloc, ctypes.byref(sh), ctypes.byref(ws), _ptr(base_logits),
+                 _ptr(hidden), _ptr(S0), _ptr(tokens_out), _ptr(logits_out), _ptr(states_out), _ptr(status),
+                 _stream(stream, dev))
     _check(rc, "domino_draft_greedy_noalloc")
     return tokens_out, logits_out, states_out
 
@@ -355,43 +461,54 @@ def teacher_forced(w: HeadWeights, base_logits, hidden, S0, tokens, logits_out=N
                    workspace=None, status=None, stream=None, logits_dtype=torch.float32):
     """Teacher-forced logits (``domino_teacher_forced``, or ``domino_teacher_forced_ex`` for bf16
     logits: ``logits_dtype=torch.bfloat16``); returns (logits, states or None)."""
-    B, L, V = base_logits.shape
-    dev = base_logits.device
+    B, L, dev = _check_head_inputs(w, base_logits, hidden, S0)
+    d, Hs, r, V = w.dims()
+    _expect(tokens, "tokens", (B, L), torch.int32, dev)
     if logits_out is None:
         logits_out = torch.empty((B, L, V), dtype=logits_dtype, device=dev)
-    if logits_out.dtype not in (torch.float32, torch.bfloat16):
-        raise ValueError("logits_out must be float32 or bfloat16")
+    _expect(logits_out, "logits_out", (B, L, V), (torch.float32, torch.bfloat16), dev)
     if states_out is True:
-        states_out = torch.empty((B, L, w.W_hh.shape[1]), dtype=torch.float32, device=dev)
+        states_out = torch.empty((B, L, Hs), dtype=torch.float32, device=dev)
     if states_out is False:
         states_out = None
+    if states_out is not None:
+        _expect(states_out, "states_out", (B, L, Hs), torch.float32, dev)
+    _expect_status(status, dev)
     sh = make_shape(w, B, L)
     if workspace is None:
         workspace = alloc_workspace(workspace_bytes(w, B, L), dev)
+    _expect_workspace(workspace, dev)
     ws = w.c_struct()
     if logits_out.dtype == torch.float32:
-        rc = lib().domino_teacher_forced(ctypes.byref(sh), ctypes.byref(ws), _ptr(base_logits), _ptr(hidden),
-                                         _ptr(S0), _ptr(tokens), _ptr(logits_out), _ptr(states_out),
-                                         _ptr(workspace), workspace.numel(), _ptr(status), _stream(stream))
+        rc = _launch(dev, lib().domino_teacher_forced, ctypes.byref(sh), ctypes.byref(ws), _ptr(base_logits),
+                     _ptr(hidden), _ptr(S0), _ptr(tokens), _ptr(logits_out), _ptr(states_out), _ptr(workspace),
+                     workspace.numel(), _ptr(status), _stream(stream, dev))
         _check(rc, "domino_teacher_forced")
     else:
-        rc = lib().domino_teacher_forced_ex(ctypes.byref(sh), ctypes.byref(ws), _ptr(base_logits), _ptr(hidden),
-                                            _ptr(S0), _ptr(tokens), _ptr(logits_out), DTYPE_BF16, _ptr(states_out),
-                                            _ptr(workspace), workspace.numel(), _ptr(status), _stream(stream))
+        rc = _launch(dev, lib().domino_teacher_forced_ex, ctypes.byref(sh), ctypes.byref(ws), _ptr(base_logits),
+                     _ptr(hidden), _ptr(S0), _ptr(tokens), _ptr(logits_out), DTYPE_BF16, _ptr(states_out),
+                     _ptr(workspace), workspace.numel(), _ptr(status), _stream(stream, dev))
         _check(rc, "domino_teacher_forced_ex")
     return logits_out, states_out
 
 
 def accept_len(draft_tokens, target_logits, accept_out=None, workspace=None, status=None, stream=None):
     """Greedy accept length per row (``domino_accept_len``)."""
-    B, L, V = target_logits.shape
+    if not isinstance(target_logits, torch.Tensor) or target_logits.dim() != 3:
+        raise ValueError("target_logits must be a [B, L, V] tensor")
+    B, L, V = (int(x) for x in target_logits.shape)
     dev = target_logits.device
+    _expect(target_logits, "target_logits", (B, L, V), torch.float32, dev)
+    _expect(draft_tokens, "draft_tokens", (B, L), torch.int32, dev)
     if accept_out is None:
         accept_out = torch.empty((B,), dtype=torch.int32, device=dev)
+    _expect(accept_out, "accept_out", (B,), torch.int32, dev)
+    _expect_status(status, dev)
     if workspace is None:
         workspace = alloc_workspace(accept_workspace_bytes(B, L), dev)
-    rc = lib().domino_accept_len(B, L, V, _ptr(draft_tokens), _ptr(target_logits), _ptr(accept_out),
-                                 _ptr(workspace), workspace.numel(), _ptr(status), _stream(stream))
+    _expect_workspace(workspace, dev)
+    rc = _launch(dev, lib().domino_accept_len, B, L, V, _ptr(draft_tokens), _ptr(target_logits), _ptr(accept_out),
+                 _ptr(workspace), workspace.numel(), _ptr(status), _stream(stream, dev))
     _check(rc, "domino_accept_len")
     return accept_out
 

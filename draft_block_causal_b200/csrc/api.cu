@@ -21,6 +21,9 @@ std::atomic<int> g_ntrace{0};
 
 inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
+// Largest B * L any entry point accepts (grid y of the row-per-block launches).
+constexpr int64_t kMaxRows = 65535;
+
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // K dimension in 16-byte vectors: a multiple of 32 vectors, or a power of two up to 32.
@@ -39,7 +42,10 @@ int check_shape(const domino_shape_t* s) {
   if (s->B < 1 || s->L < 1 || s->L > DOMINO_MAX_L || s->d < 8 || s->Hs < 8 || s->r < 8 || s->V < 8)
     return DOMINO_ERR_INVALID_ARGUMENT;
   if (s->d % 8 || s->Hs % 8 || s->r % 8 || s->V % 8) return DOMINO_ERR_INVALID_ARGUMENT;
-  if ((int64_t)s->B * s->L > (1 << 19)) return DOMINO_ERR_UNSUPPORTED;
+  // launches with one row (or row tile) per block along grid y need B*L <= 65535; element loops over
+  // B*Hs and B*L*d/8 count in 32-bit integers
+  const int64_t BL = (int64_t)s->B * s->L;
+  if (BL > kMaxRows || BL * std::max<int64_t>(s->Hs, s->d / 8) > INT32_MAX) return DOMINO_ERR_UNSUPPORTED;
   if (s->r > 1024) return DOMINO_ERR_UNSUPPORTED;
   if (!vec_layout_ok(s->d, s->dtype) || !vec_layout_ok(s->Hs, s->dtype) || !vec_layout_ok(s->r, s->dtype))
     return DOMINO_ERR_UNSUPPORTED;
@@ -476,7 +482,7 @@ int domino_accept_len(int32_t B, int32_t L, int32_t V, const int32_t* draft_toke
                       domino_stream_t stream) {
   (void)status_dev;
   if (B < 1 || L < 1 || L > DOMINO_MAX_L || V < 8 || V % 8) return DOMINO_ERR_INVALID_ARGUMENT;
-  if ((int64_t)B * L > (1 << 19)) return DOMINO_ERR_UNSUPPORTED;
+  if ((int64_t)B * L > kMaxRows) return DOMINO_ERR_UNSUPPORTED;
   if (!draft_tokens || !target_logits || !accept_out) return DOMINO_ERR_INVALID_ARGUMENT;
   if (!aligned16(target_logits)) return DOMINO_ERR_INVALID_ARGUMENT;
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) ||

@@ -29,7 +29,8 @@
  *     fp32 in every mode.
  *   - Shapes: 1 <= B, 1 <= L <= DOMINO_MAX_L; d, Hs and r must each be a multiple of 8 and, in
  *     16-byte vectors, either a multiple of 32 vectors or a power of two up to 32 vectors; V must
- *     be a multiple of 8.
+ *     be a multiple of 8 (else DOMINO_ERR_INVALID_ARGUMENT).  B * L <= 65535, r <= 1024 and
+ *     B * L * max(Hs, d / 8) < 2^31 (else DOMINO_ERR_UNSUPPORTED).
  */
 #ifndef DOMINO_H_
 #define DOMINO_H_

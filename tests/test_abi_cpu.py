@@ -65,6 +65,12 @@ def test_workspace_bytes_host_logic(L):
     assert L.domino_workspace_bytes(ctypes.byref(_shape(d=2560))) > 0  # 320 vectors = 10 x 32
     assert L.domino_accept_workspace_bytes(32, 16) > 0
     assert L.domino_accept_workspace_bytes(0, 16) == 0
+    # B * L up to 65535 rows (launches with one row per block along grid y), and 32-bit element
+    # loops over B * L * Hs
+    assert L.domino_workspace_bytes(ctypes.byref(_shape(B=4095))) > 0
+    assert L.domino_workspace_bytes(ctypes.byref(_shape(B=4096))) == 0
+    assert L.domino_workspace_bytes(ctypes.byref(_shape(B=65535, L=1))) > 0
+    assert L.domino_workspace_bytes(ctypes.byref(_shape(B=8, Hs=1 << 24))) == 0
 
 
 def test_invalid_arguments_are_rejected_before_any_launch(L):
@@ -108,6 +114,8 @@ def test_invalid_arguments_are_rejected_before_any_launch(L):
                                None) == domino.ERR_INVALID_ARGUMENT
     assert L.domino_accept_len(i32(1), i32(16), i32(151936), fake, fake, fake, fake, 16, None,
                                None) == domino.ERR_WORKSPACE
+    assert L.domino_accept_len(i32(4096), i32(16), i32(151936), fake, fake, fake, fake, 1 << 30, None,
+                               None) == domino.ERR_UNSUPPORTED
 
 
 def test_arena_host_logic(L):

@@ -110,6 +110,7 @@ Workspace layout_workspace(const Shape& s, void* base) {
   w.keys = reinterpret_cast<uint64_t*>(take(BL * sizeof(uint64_t)));
   w.a_acc = reinterpret_cast<float*>(take(BL * s.r * kAccReplicas * sizeof(float)));
   w.acc_keys = reinterpret_cast<uint64_t*>(take(BL * sizeof(uint64_t)));
+  w.acc_count = reinterpret_cast<uint32_t*>(take((BL + s.B + 1) * sizeof(uint32_t)));
   w.P = reinterpret_cast<float*>(take(BL * s.r * sizeof(float)));
   w.u = reinterpret_cast<float*>(take(BL * s.r * sizeof(float)));
   w.S = reinterpret_cast<float*>(take(2 * (size_t)s.B * s.Hs * sizeof(float)));
@@ -492,9 +493,11 @@ int domino_accept_len(int32_t B, int32_t L, int32_t V, const int32_t* draft_toke
   const Workspace ws = layout_workspace(s, workspace);
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   const size_t BL = (size_t)B * L;
-  cudaError_t e = cudaMemsetAsync(ws.acc_keys, 0, BL * sizeof(uint64_t), cs);
-  if (e == cudaSuccess) e = launch_row_argmax(target_logits, (int)BL, V, ws.acc_keys, cs);
-  if (e == cudaSuccess) e = launch_accept_count(draft_tokens, ws.acc_keys, B, L, accept_out, cs);
+  // keys, counters, first-mismatch words and the completion word: adjacent, cleared together
+  const size_t clear = reinterpret_cast<char*>(ws.acc_count + BL + B + 1) - reinterpret_cast<char*>(ws.acc_keys);
+  cudaError_t e = cudaMemsetAsync(ws.acc_keys, 0, clear, cs);
+  if (e == cudaSuccess)
+    e = launch_accept_early(target_logits, draft_tokens, B, L, V, ws.acc_keys, ws.acc_count, accept_out, cs);
   return cuda_rc(e);
 }
 

@@ -25,6 +25,8 @@ struct Workspace {
   uint32_t* claim;     // [kClaimWords] work-slot claims of SM-affine GEMM launches (zeroed per call)
   uint64_t* keys;      // [L][B]   greedy argmax keys per position
   uint64_t* acc_keys;  // [B*L]    target-logit argmax keys (accept length)
+  uint32_t* acc_count; // [B*L]    chunks finished per (row, position); then [B] first mismatch (as L - j);
+                       //          then one grid-completion word -- contiguous with acc_keys (one memset)
   float* P;            // [B*L][r] W1 . H for every position
   float* u;            // [B*L][r] SiLU activations
   float* S;            // [2][B][Hs] greedy state ping-pong
@@ -74,11 +76,12 @@ cudaError_t launch_cell(const Shape& s, const float* Gx, int ldx, int xper, int 
                         int tok_add, const float* Sin, size_t sin_stride, float* Sout, size_t sout_stride,
                         float* Sout2, size_t sout2_stride, int32_t* status, cudaStream_t st,
                         __nv_bfloat16* S_hl = nullptr);
+// One launch: accept lengths with early exit (k_accept_early).  keys [B*L] and count
+// [B*L + B + 1] must be zero.
+cudaError_t launch_accept_early(const float* T, const int32_t* draft, int B, int L, int V, uint64_t* keys,
+                                uint32_t* count, int32_t* out, cudaStream_t st);
 cudaError_t launch_tokens_from_keys(const uint64_t* keys, int B, int L, int32_t* tokens, cudaStream_t st);
 cudaError_t launch_copy_rows(const float* src, size_t src_stride, float* dst, size_t dst_stride, int rows, int n,
                              cudaStream_t st);
-cudaError_t launch_row_argmax(const float* T, int rows, int V, uint64_t* keys, cudaStream_t st);
-cudaError_t launch_accept_count(const int32_t* draft, const uint64_t* keys, int B, int L, int32_t* out,
-                                cudaStream_t st);
 
 }  // namespace domino

@@ -391,46 +391,71 @@ __global__ void k_copy_rows(const float* __restrict__ src, size_t src_stride, fl
   }
 }
 
-// keys[n] = max over the row of argmax_key(T[n][v], v); blockIdx.y = row, blockIdx.x = chunk.
+// Columns of one target row that one block of the accept-length kernel reads.
 constexpr int kArgChunk = 8192;
-__global__ void __launch_bounds__(256) k_row_argmax(const float* __restrict__ T, int V, uint64_t* __restrict__ keys) {
+
+// Greedy accept length with early exit, in one launch.  Block (c, y) reads chunk c (kArgChunk
+// columns) of the target row of position j = y / B, batch row b = y % B: position-major, so that a
+// row's earlier positions are issued first.  It folds the chunk's argmax key into keys[b * L + j].
+// The last chunk block of a (row, position) compares the finished argmax with the draft token and,
+// on a mismatch, records it: first[b] = max(first[b], L - j), so 0 means "none" and the largest
+// value is the earliest mismatch.  A block whose position lies past a recorded mismatch of its row
+// skips its reads; such a position cannot change the row's result, because a mismatch can only
+// be recorded for it after an earlier one has been, and the earlier one wins the max.  The last
+// block of the grid writes out[b] = L - first[b].
+// count = [B*L chunk counters][B first-mismatch words][1 grid counter], all zero at launch.
+__global__ void __launch_bounds__(256) k_accept_early(const float* __restrict__ T, const int32_t* __restrict__ draft,
+                                                      int B, int L, int V, uint64_t* __restrict__ keys,
+                                                      uint32_t* __restrict__ count, int32_t* __restrict__ out) {
   pdl_wait();
   pdl_trigger();
   __shared__ uint64_t red[8];
-  const int n = blockIdx.y;
-  const int v0 = blockIdx.x * kArgChunk;
-  const int v1 = min(V, v0 + kArgChunk);
-  const float* row = T + (size_t)n * V;
-  uint64_t best = 0ull;
-  for (int v = v0 + 4 * threadIdx.x; v < v1; v += 4 * blockDim.x) {
-    float4 q = __ldcs(reinterpret_cast<const float4*>(row + v));
-    best = umax64(best, argmax_key(q.x, v));
-    best = umax64(best, argmax_key(q.y, v + 1));
-    best = umax64(best, argmax_key(q.z, v + 2));
-    best = umax64(best, argmax_key(q.w, v + 3));
-  }
+  __shared__ bool last_chunk, last_block;
+  const int y = blockIdx.y, j = y / B, b = y % B;
+  const size_t n = (size_t)b * L + j;
+  uint32_t* const first = count + (size_t)B * L;
+  uint32_t* const done = first + B;
+  const bool skip = *reinterpret_cast<volatile uint32_t*>(first + b) > (uint32_t)(L - j);
+  if (!skip) {  // block-uniform
+    const int v0 = blockIdx.x * kArgChunk, v1 = min(V, v0 + kArgChunk);
+    const float* row = T + n * V;
+    uint64_t best = 0ull;
+    for (int v = v0 + 4 * threadIdx.x; v < v1; v += 4 * blockDim.x) {
+      const float4 q = __ldcs(reinterpret_cast<const float4*>(row + v));
+      best = umax64(best, argmax_key(q.x, v));
+      best = umax64(best, argmax_key(q.y, v + 1));
+      best = umax64(best, argmax_key(q.z, v + 2));
+      best = umax64(best, argmax_key(q.w, v + 3));
+    }
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) best = umax64(best, __shfl_xor_sync(0xffffffffu, best, o));
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = best;
+    for (int o = 16; o > 0; o >>= 1) best = umax64(best, __shfl_xor_sync(0xffffffffu, best, o));
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = best;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      for (int w = 1; w < (int)(blockDim.x >> 5); ++w) best = umax64(best, red[w]);
+      atomicMax(reinterpret_cast<unsigned long long*>(keys + n), (unsigned long long)best);
+    }
+  }
+  if (threadIdx.x == 0) {
+    __threadfence();  // this block's key before its count
+    last_chunk = atomicAdd(count + n, 1u) == gridDim.x - 1;
+  }
   __syncthreads();
   if (threadIdx.x == 0) {
-    for (int w = 1; w < (int)(blockDim.x >> 5); ++w) best = umax64(best, red[w]);
-    atomicMax(reinterpret_cast<unsigned long long*>(keys + n), (unsigned long long)best);
+    if (last_chunk) {
+      __threadfence();
+      const uint64_t k = atomicAdd(reinterpret_cast<unsigned long long*>(keys + n), 0ull);
+      if (draft[n] != key_index(k)) atomicMax(first + b, (uint32_t)(L - j));
+    }
+    __threadfence();  // this block's record before its completion
+    last_block = atomicAdd(done, 1u) == gridDim.x * gridDim.y - 1;
   }
-}
-
-__global__ void k_accept_count(const int32_t* __restrict__ draft, const uint64_t* __restrict__ keys, int B, int L,
-                               int32_t* __restrict__ out) {
-  pdl_wait();
-  pdl_trigger();
-  int b = blockIdx.x * blockDim.x + threadIdx.x;
-  if (b >= B) return;
-  int k = 0;
-  for (int j = 0; j < L; ++j) {
-    if (draft[(size_t)b * L + j] != key_index(keys[(size_t)b * L + j])) break;
-    k = j + 1;
+  __syncthreads();
+  if (last_block) {
+    __threadfence();
+    for (int r = threadIdx.x; r < B; r += blockDim.x)
+      out[r] = L - (int)*reinterpret_cast<volatile uint32_t*>(first + r);
   }
-  out[b] = k;
 }
 
 inline unsigned cdiv(size_t a, size_t b) { return (unsigned)((a + b - 1) / b); }
@@ -563,15 +588,10 @@ cudaError_t launch_copy_rows(const float* src, size_t src_stride, float* dst, si
   return note_launch(e);
 }
 
-cudaError_t launch_row_argmax(const float* T, int rows, int V, uint64_t* keys, cudaStream_t st) {
-  dim3 grid(cdiv(V, kArgChunk), rows);
-  cudaError_t e = launch_pdl(k_row_argmax, grid, dim3(256), 0, st, T, V, keys);
-  return note_launch(e);
-}
-
-cudaError_t launch_accept_count(const int32_t* draft, const uint64_t* keys, int B, int L, int32_t* out,
-                                cudaStream_t st) {
-  cudaError_t e = launch_pdl(k_accept_count, dim3(cdiv(B, 128)), dim3(128), 0, st, draft, keys, B, L, out);
+cudaError_t launch_accept_early(const float* T, const int32_t* draft, int B, int L, int V, uint64_t* keys,
+                                uint32_t* count, int32_t* out, cudaStream_t st) {
+  dim3 grid(cdiv(V, kArgChunk), (unsigned)(B * L));  // B * L <= 65535 (shape checks)
+  cudaError_t e = launch_pdl(k_accept_early, grid, dim3(256), 0, st, T, draft, B, L, V, keys, count, out);
   return note_launch(e);
 }
 

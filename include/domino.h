@@ -200,9 +200,10 @@ DOMINO_API int domino_teacher_forced_ex(const domino_shape_t* shape, const domin
  *   accept_out[b] = number of leading positions j (0 <= j < L) with
  *                   draft_tokens[b, j] == argmax_v target_logits[b, j, v]  (lowest index on ties)
  * No bonus token is counted.  draft_tokens [B, L] int32, target_logits [B, L, V] fp32,
- * accept_out [B] int32.  Needs domino_accept_workspace_bytes(B, L) bytes of workspace (a
- * workspace sized by domino_workspace_bytes for the same B and L also suffices).
- * Returns DOMINO_OK or a negative DOMINO_ERR_* code. */
+ * accept_out [B] int32.  One kernel launch; the target logits of a row's positions after its first
+ * mismatch may be left unread (the result is the same).  Needs domino_accept_workspace_bytes(B, L)
+ * bytes of workspace (a workspace sized by domino_workspace_bytes for the same B and L also
+ * suffices).  Returns DOMINO_OK or a negative DOMINO_ERR_* code. */
 DOMINO_API size_t domino_accept_workspace_bytes(int32_t B, int32_t L);
 DOMINO_API int domino_accept_len(int32_t B, int32_t L, int32_t V, const int32_t* draft_tokens,
                       const float* target_logits, int32_t* accept_out, void* workspace,

@@ -485,6 +485,7 @@ def run_ours(args):
     total_ms = max_over_ranks(sum(step_ms), dist, device)
     torch.cuda.synchronize()
     assert int(pt.status.item()) == 0, domino.status_string(int(pt.status.item()))
+    pt_acc_mean = pt.acc.float().mean().item()
     sh = pt.sh
     B = sh["B"]
     value = job_throughput(B, world, args.steps, total_ms)
@@ -564,6 +565,8 @@ def run_ours(args):
                     "us_per_block": round(1e3 * statistics.mean(s_ms) / pb, 3),
                     "ms_per_step": round(statistics.mean(s_ms), 4),
                     "greedy_ms": round(ga, 4),
+                    # the accept length reads a row's target logits only up to its first mismatch
+                    "accept_mean": round(float(p.acc.float().mean().item()), 3),
                     "hbm_frac": round(greedy_bytes(psh) / (ga * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
                     "tensor_frac": round(fl / (ga * 1e-3) / 1e12 / peaks["bf16_tflops"], 4),
                     "greedy_tflops": round(fl / (ga * 1e-3) / 1e12, 2),
@@ -622,6 +625,7 @@ def run_ours(args):
                        "parallelism": f"replicas x{world} (rows independent, no collective)",
                        "l2": "flushed (256 MiB write) before every timed step"},
             "us_per_block": round(1e3 * total_ms / args.steps / B, 3),
+            "accept_mean": round(float(pt_acc_mean), 3),
             "roofline": roof,
             "roofline_l2": roof_l2,
             "cpu_baseline": cpu,

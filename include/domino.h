@@ -17,6 +17,10 @@
  *     memory is the caller's workspace.
  *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy default stream) and
  *     never synchronises the host.  Calls that share a workspace must be ordered on the GPU.
+ *   - Calls run on the calling thread's current device, which must hold every pointer passed.
+ *     Several host threads may call at once; calls whose GPU work overlaps need separate
+ *     workspaces (and see domino_draft_greedy_noalloc).  The debug hooks' settings are
+ *     process-wide.
  *   - Host-side checks happen before any launch: on a negative return code nothing was enqueued.
  *   - Device-side problems (a bounded wait that gave up, a token outside [0, V)) are reported by
  *     writing a positive DOMINO_STATUS_* code to *status_dev with an atomic compare-and-swap from

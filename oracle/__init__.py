@@ -56,6 +56,11 @@ def configure(lib: ctypes.CDLL) -> ctypes.CDLL:
     lib.oracle_accept_len.restype = ctypes.c_int
     lib.oracle_gru_step.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int] + [vp] * 7
     lib.oracle_gru_step.restype = None
+    lib.oracle_accept_sample.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, vp, vp, vp, ctypes.c_float, vp,
+                                         vp, vp, vp]
+    lib.oracle_accept_sample.restype = ctypes.c_int
+    lib.oracle_residual_cdf.argtypes = [ctypes.c_int, vp, vp, ctypes.c_int, ctypes.c_float, vp]
+    lib.oracle_residual_cdf.restype = ctypes.c_double
     lib.oracle_max_threads.argtypes = []
     lib.oracle_max_threads.restype = ctypes.c_int
     return lib
@@ -140,6 +145,39 @@ def accept_len(draft_tokens, target_logits) -> np.ndarray:
     if rc != 0:
         raise ValueError(f"oracle_accept_len failed with code {rc}")
     return out
+
+
+def accept_sample(draft_tokens, target_logits, temperature: float, uniforms, draft_logits=None) -> dict:
+    """Sampled verification of a block (see ``oracle_accept_sample`` in domino_oracle.c):
+    accept lengths [B], replacement tokens [B] (-1 when every position was accepted) and the
+    acceptance ratios p/q [B, L] of the decisions taken (-1 after)."""
+    B, L, V = target_logits.shape
+    _check(draft_tokens, np.int32, (B, L), "draft_tokens")
+    _check(target_logits, np.float32, (B, L, V), "target_logits")
+    _check(uniforms, np.float32, (B, L + 1), "uniforms")
+    if draft_logits is not None:
+        _check(draft_logits, np.float32, (B, L, V), "draft_logits")
+    acc = np.empty((B,), np.int32)
+    nxt = np.empty((B,), np.int32)
+    ratio = np.empty((B, L), np.float64)
+    rc = _load().oracle_accept_sample(B, L, V, _ptr(draft_tokens), _ptr(draft_logits), _ptr(target_logits),
+                                      float(temperature), _ptr(uniforms), _ptr(acc), _ptr(nxt), _ptr(ratio))
+    if rc != 0:
+        raise ValueError(f"oracle_accept_sample failed with code {rc}")
+    return {"accept": acc, "next": nxt, "ratio": ratio}
+
+
+def residual_cdf(target_row, draft_row, draft_token: int, temperature: float):
+    """Running sums of the resampling residual at one position (``oracle_residual_cdf``):
+    returns (cdf [V] float64, Z)."""
+    V = target_row.shape[0]
+    _check(target_row, np.float32, (V,), "target_row")
+    if draft_row is not None:
+        _check(draft_row, np.float32, (V,), "draft_row")
+    cdf = np.empty((V,), np.float64)
+    z = _load().oracle_residual_cdf(V, _ptr(target_row), _ptr(draft_row), int(draft_token), float(temperature),
+                                    _ptr(cdf))
+    return cdf, float(z)
 
 
 def gru_step(d: int, Hs: int, dtype: int, w: dict, x, h) -> np.ndarray:

@@ -24,6 +24,9 @@
  *     argmax of L_final; ties go to the lowest vocabulary index.
  *   - Accept length = number of leading positions j whose draft token equals the argmax
  *     (lowest index on ties) of the target logits at j; no bonus token.
+ *   - Sampled (temperature > 0) verification, which the pages call lossless without restating
+ *     it, follows the published speculative-sampling rule (see oracle_accept_sample); the random
+ *     draws it needs are inputs.
  *
  * Precision: every stored input (fp32, or bf16 bit patterns) is widened exactly to double;
  * all arithmetic is double; exp and tanh come from libm.  No blocking, fusion or reordering
@@ -209,4 +212,117 @@ int oracle_accept_len(int B, int L, int V, const int32_t* draft_tokens, const fl
     accept_out[b] = k;
   }
   return 0;
+}
+
+/*
+ * Stochastic (temperature > 0) verification of a draft block: the acceptance rule of speculative
+ * sampling (Leviathan, Kalman and Matias, "Fast Inference from Transformers via Speculative
+ * Decoding", ICML 2023; Chen et al., "Accelerating Large Language Model Decoding with Speculative
+ * Sampling", 2023).  The pages call Domino's verification lossless (review page, section 一: the
+ * target model checks the whole block in one parallel pass; researchpapers.dev summary) and spell
+ * out only the greedy setting; this is the published rule that makes sampled verification
+ * lossless, which they do not restate.
+ *
+ * Row b, positions j = 0, 1, ... in order:
+ *   p_j = softmax(target_logits[b, j, :] / T)
+ *   q_j = softmax(draft_logits[b, j, :] / T), or, when draft_logits is NULL (a greedy draft), the
+ *         one-hot distribution on the draft token
+ *   x = draft_tokens[b, j] is accepted when uniforms[b, j] < p_j(x) / q_j(x); the first rejected
+ *   position k ends the row.  Its replacement token is drawn from the residual
+ *   res(v) = max(0, p_k(v) - q_k(v)) by inverse transform with u = uniforms[b, L]: the smallest v
+ *   (ascending) whose running sum of res exceeds u * Z, Z = sum_v res(v) (the last v with
+ *   res(v) > 0 if the running sum never does).
+ * accept_out[b] = k (L when every position is accepted); next_out[b] = the replacement token, or
+ * -1 when all L were accepted (no bonus token: there are no target logits past the block).
+ * ratio_out (optional, [B, L]) receives p_j(x) / q_j(x) for j <= k and -1 after.
+ * uniforms is [B, L + 1] in [0, 1).  Returns 0, or -1 on a bad argument.
+ */
+static void softmax_row(const float* t, int V, double T, double* out) {
+  double m = (double)t[0];
+  for (int v = 1; v < V; ++v)
+    if ((double)t[v] > m) m = (double)t[v];
+  double s = 0.0;
+  for (int v = 0; v < V; ++v) {
+    out[v] = exp(((double)t[v] - m) / T);
+    s += out[v];
+  }
+  for (int v = 0; v < V; ++v) out[v] /= s;
+}
+
+/* Residual of position (p, q) for draft token x: res[v] = max(0, p[v] - q[v]) with q one-hot on x
+ * when q is NULL.  Returns Z = sum_v res[v] (ascending). */
+static double residual(const double* p, const double* q, int x, int V, double* res) {
+  double z = 0.0;
+  for (int v = 0; v < V; ++v) {
+    const double qv = q ? q[v] : (v == x ? 1.0 : 0.0);
+    const double r = p[v] - qv;
+    res[v] = r > 0.0 ? r : 0.0;
+    z += res[v];
+  }
+  return z;
+}
+
+int oracle_accept_sample(int B, int L, int V, const int32_t* draft_tokens, const float* draft_logits,
+                         const float* target_logits, float temperature, const float* uniforms, int32_t* accept_out,
+                         int32_t* next_out, double* ratio_out) {
+  if (B < 1 || L < 1 || V < 1 || !(temperature > 0.0f)) return -1;
+  const double T = (double)temperature;
+  double* p = (double*)malloc(sizeof(double) * (size_t)V);
+  double* q = draft_logits ? (double*)malloc(sizeof(double) * (size_t)V) : NULL;
+  double* res = (double*)malloc(sizeof(double) * (size_t)V);
+  if (!p || !res || (draft_logits && !q)) {
+    free(p); free(q); free(res);
+    return -1;
+  }
+  for (int b = 0; b < B; ++b) {
+    int k = L, next = -1;
+    for (int j = 0; j < L; ++j) {
+      const size_t row = (size_t)b * L + j;
+      const int x = draft_tokens[row];
+      if (x < 0 || x >= V) { free(p); free(q); free(res); return -1; }
+      softmax_row(target_logits + row * (size_t)V, V, T, p);
+      if (q) softmax_row(draft_logits + row * (size_t)V, V, T, q);
+      const double ratio = p[x] / (q ? q[x] : 1.0);
+      if (ratio_out) ratio_out[row] = ratio;
+      if ((double)uniforms[(size_t)b * (L + 1) + j] < ratio) continue;
+      k = j;
+      const double z = residual(p, q, x, V, res);
+      const double target = (double)uniforms[(size_t)b * (L + 1) + L] * z;
+      double run = 0.0;
+      int last = -1;
+      for (int v = 0; v < V; ++v) {
+        if (res[v] > 0.0) last = v;
+        run += res[v];
+        if (run > target && res[v] > 0.0) { next = v; break; }
+      }
+      if (next < 0) next = last;
+      break;
+    }
+    if (ratio_out)
+      for (int j = k + 1; j < L; ++j) ratio_out[(size_t)b * L + j] = -1.0;
+    accept_out[b] = k;
+    next_out[b] = next;
+  }
+  free(p); free(q); free(res);
+  return 0;
+}
+
+/* The running sums of the residual used by oracle_accept_sample at one position:
+ * cdf[v] = sum_{w <= v} res(w) (ascending), for the target row t, the draft row dq (NULL: one-hot
+ * on x) and temperature T.  Returns Z = cdf[V - 1]. */
+double oracle_residual_cdf(int V, const float* t, const float* dq, int x, float temperature, double* cdf) {
+  const double T = (double)temperature;
+  double* p = (double*)malloc(sizeof(double) * (size_t)V);
+  double* q = dq ? (double*)malloc(sizeof(double) * (size_t)V) : NULL;
+  if (!p || (dq && !q)) { free(p); free(q); return -1.0; }
+  softmax_row(t, V, T, p);
+  if (q) softmax_row(dq, V, T, q);
+  double z = residual(p, q, x, V, cdf);
+  double run = 0.0;
+  for (int v = 0; v < V; ++v) {
+    run += cdf[v];
+    cdf[v] = run;
+  }
+  free(p); free(q);
+  return z;
 }

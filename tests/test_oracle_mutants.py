@@ -1,5 +1,6 @@
 """The oracle's pins catch plausible mistakes: each mutant below is the oracle's C source with one
-planted error (a sign, a gate, a bias, an index, an operand order, the tie rule, the accept count),
+planted error (a sign, a gate, a bias, an index, an operand order, the tie rule, the accept count,
+the sampled-verification rule's clamp, ratio, draw, temperature and residual),
 built into a separate library on the CPU; at least one pin of tests/test_oracle_pins.py must fail
 on it.  The oracle itself is never modified."""
 import ctypes
@@ -10,6 +11,7 @@ import pytest
 
 import oracle
 from tests import test_oracle_pins as pins
+from tests import test_oracle_sampling_pins as spins
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "domino_oracle.c")
 
@@ -30,6 +32,16 @@ MUTANTS = [
     ("accept length counts a bonus token", "      k = j + 1;", "      k = j + 2;"),
     ("hidden state of the next position", "elem(hidden, pos * d + c, dt)",
      "elem(hidden, (pos + (i + 1 < L)) * d + c, dt)"),
+    # sampled verification
+    ("residual not clamped at zero", "res[v] = r > 0.0 ? r : 0.0;", "res[v] = r;"),
+    ("acceptance ratio inverted", "const double ratio = p[x] / (q ? q[x] : 1.0);",
+     "const double ratio = (q ? q[x] : 1.0) / p[x];"),
+    ("resampled with the position's acceptance draw",
+     "const double target = (double)uniforms[(size_t)b * (L + 1) + L] * z;",
+     "const double target = (double)uniforms[(size_t)b * (L + 1) + j] * z;"),
+    ("temperature ignored", "out[v] = exp(((double)t[v] - m) / T);", "out[v] = exp(((double)t[v] - m));"),
+    ("replacement drawn from the target instead of the residual",
+     "const double qv = q ? q[v] : (v == x ? 1.0 : 0.0);", "const double qv = 0.0 * (q ? q[v] : (double)x);"),
 ]
 
 PIN_CALLS = [
@@ -44,6 +56,11 @@ PIN_CALLS = [
     lambda: pins.test_greedy_is_the_unique_fixed_point_of_teacher_forcing(21),
     pins.test_accept_len_matches_numpy_first_argmax,
     pins.test_accept_len_hand_cases,
+    spins.test_identical_distributions_accept_every_position,
+    spins.test_token_outside_the_target_support_is_rejected_and_replaced_from_it,
+    lambda: spins.test_lossless_for_a_sampled_draft_on_five_tokens(0.5),
+    lambda: spins.test_lossless_for_a_greedy_draft_on_five_tokens(2),
+    spins.test_low_temperature_is_the_greedy_accept_rule,
 ]
 
 

@@ -309,6 +309,18 @@ def w2_kernel_us(pt: Point, flush, stream) -> float:
     return float((t[:, 1].max() - t[:, 15].min()) / 1e3)
 
 
+def full_accept_targets(pt: Point, stream):
+    """Target logits on which every draft token of the point's greedy call is the argmax: the
+    draft's own final logits (one greedy call with logits written, untimed)."""
+    torch = pt.torch
+    sh = pt.sh
+    logits = torch.empty((sh["B"], sh["L"], sh["V"]), dtype=torch.float32, device=pt.lb.device)
+    pt.domino.draft_greedy(pt.w, pt.lb, pt.h, pt.S0, tokens_out=pt.tok, logits_out=logits, workspace=pt.ws,
+                           status=pt.status, stream=stream)
+    torch.cuda.synchronize()
+    return logits
+
+
 def time_tf(pt: Point, steps: int, warmup: int, flush, stream, bf16_logits: bool = False) -> list:
     """Teacher-forced calls (uniform given tokens, logits out), each after an L2 flush; per-call
     device times in ms."""
@@ -510,9 +522,18 @@ def run_ours(args):
         t_bound_ms = (first / (peaks["hbm_gbs"] * 1e9) + (gbytes - first) / (l2_gbs * 1e9)) * 1e3
         roof_l2 = {"first_touch_bytes": first,
                    "first_touch_source": "ncu dram bytes of this kernel" if roof["traffic"] else "unique bytes",
-                   "reread_bytes": gbytes - first, "l2_reread_gbs": round(l2_gbs, 1), "hbm_gbs": peaks["hbm_gbs"],
+                   "reread_bytes": gbytes - first, "l2_reread_gbs": round(l2_gbs, 1),
+                   "l2_reread_source": "measured in this run by domino_debug_read_passes (one CTA per SM re-reading "
+                                       "a W2-sized buffer with 16-byte loads); builder-measured, not a "
+                                       "MEASURED_PEAKS figure",
+                   "hbm_gbs": peaks["hbm_gbs"],
                    "bound_ms": round(t_bound_ms, 4), "launch_ms": round(g_avg, 4),
                    "frac": round(t_bound_ms / g_avg, 4)}
+        # The weights' re-reads hit L2 (the committed capture shows an 83% L2 hit rate), so the bound
+        # that governs this kernel is the reuse-aware one; roofline.frac stays algorithmic bytes over
+        # HBM bandwidth, as the measurement contract defines it.
+        roof["frac_reuse_aware"] = roof_l2["frac"]
+        roof["governing"] = "reuse-aware (roofline_l2): weight re-reads are L2 hits"
         e2e_ms, h2d, d2h = time_e2e(pt, max(3, args.steps // 2), 3, flush, stream)
         e2e_val = B / (statistics.mean(e2e_ms) * 1e-3)
         e2e_serial_ms, _, _ = time_e2e(pt, max(3, args.steps // 2), 3, flush, stream, overlap=False)
@@ -575,6 +596,21 @@ def run_ours(args):
                                        "note": "last position's W2 GEMM with fused argmax, one launch, from its "
                                                "own device clock stamps"},
                 }
+                # The synthetic targets (base + N(0, 0.5)) reject most drafts within two positions, so
+                # the early-exit accept length skips most target reads.  For a step whose accept
+                # length is the whole block -- every target row read, as with drafts that mostly
+                # agree (the pages report about 7 accepted tokens) -- time it again with the targets
+                # set to the draft's own final logits, on which every draft token is the argmax.
+                p.T = full_accept_targets(p, stream)
+                fs, _, _ = time_steps(p, max(3, args.steps // 2), args.warmup, flush, stream)
+                points[str(pb)]["full_accept"] = {
+                    "blocks_per_s": round(pb * len(fs) / (sum(fs) * 1e-3), 1),
+                    "ms_per_step": round(statistics.mean(fs), 4),
+                    "accept_mean": round(float(p.acc.float().mean().item()), 3),
+                    "note": "targets = the draft's own final logits: no early exit, every target row read"}
+                p.T = None
+                torch.cuda.empty_cache()
+                p.T = torch.from_numpy(p.data["target_logits"]).to(device)
                 warm = time_steps_persisting(p, max(3, args.steps // 2), args.warmup, flush, stream)
                 if warm is not None:
                     points[str(pb)]["l2_persisting_blocks_per_s"] = round(pb * len(warm[0]) / (sum(warm[0]) * 1e-3), 1)
@@ -614,6 +650,28 @@ def run_ours(args):
                                                       / peaks["hbm_gbs"], 4)}
             del p
             torch.cuda.empty_cache()
+        # the Qwen3-4B-shaped head over the batch sweep: greedy call and step per batch size
+        points_4b = {}
+        if extras and not args.no_points:
+            for pb in synth.SWEEP_BATCHES:
+                p = Point(synth.workload("qwen3-4b-head-sweep", B=pb), device)
+                s_ms, g_ms, _ = time_steps(p, max(3, args.steps // 4), args.warmup, flush, stream)
+                ga = statistics.mean(g_ms)
+                psh = p.sh
+                ent = {"blocks_per_s": round(pb * len(s_ms) / (sum(s_ms) * 1e-3), 1),
+                       "us_per_block": round(1e3 * statistics.mean(s_ms) / pb, 3),
+                       "greedy_ms": round(ga, 4),
+                       "accept_mean": round(float(p.acc.float().mean().item()), 3),
+                       "hbm_frac": round(greedy_bytes(psh) / (ga * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
+                       "tensor_frac": round(greedy_flops(psh) / (ga * 1e-3) / 1e12 / peaks["bf16_tflops"], 4)}
+                if pb > 4:  # the batched path: one W2 argmax launch from its own clock stamps
+                    w2_us = w2_kernel_us(p, flush, stream)
+                    w2_flops = 2.0 * min(pb, 128) * psh["V"] * psh["r"]
+                    ent["w2_argmax_us"] = round(w2_us, 2)
+                    ent["w2_tensor_frac"] = round(w2_flops / (w2_us * 1e-6) / 1e12 / peaks["bf16_tflops"], 4)
+                points_4b[str(pb)] = ent
+                del p
+                torch.cuda.empty_cache()
         cpu = None if (args.no_cpu_baseline or not extras) else cpu_baseline(args.cpu_seconds)
         result = {
             "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -636,6 +694,7 @@ def run_ours(args):
             "gpu_launches": launches,
             "clocks": clocks,
             "points": points,
+            "points_4b": points_4b,
             "modes": modes,
             "variants": variants,
         }

@@ -108,7 +108,7 @@ Workspace layout_workspace(const Shape& s, void* base) {
   // sync, claim, keys and a_acc are adjacent so that one memset clears them together
   w.claim = reinterpret_cast<uint32_t*>(take(kClaimWords * sizeof(uint32_t)));
   w.keys = reinterpret_cast<uint64_t*>(take(BL * sizeof(uint64_t)));
-  w.a_acc = reinterpret_cast<float*>(take(BL * s.r * kAccReplicas * sizeof(float)));
+  w.a_acc = reinterpret_cast<unsigned long long*>(take(acc_bytes(s.B, s.r)));
   w.acc_keys = reinterpret_cast<uint64_t*>(take(BL * sizeof(uint64_t)));
   w.acc_count = reinterpret_cast<uint32_t*>(take((BL + s.B + 1) * sizeof(uint32_t)));
   w.P = reinterpret_cast<float*>(take(BL * s.r * sizeof(float)));
@@ -168,8 +168,10 @@ const char* domino_greedy_plan(const domino_shape_t* shape) {
     int bn_h = 0, ks_h = 0, bn_i = 0, ks_i = 0;
     gemm_tc_skinny_plan(3 * s.Hs + s.r, s.B, 2 * s.Hs, &bn_h, &ks_h);
     gemm_tc_skinny_plan(3 * s.Hs, s.B, s.d, &bn_i, &ks_i);
-    text = "per-phase kernels: tcgen05 H-projection GEMM; per position a tcgen05 W2 GEMM with the argmax in its "
-           "epilogue, the GRU input half (" +
+    text = std::string("per-phase kernels: tcgen05 H-projection GEMM; per position ") +
+           (s.r <= 256 ? "k_w2_argmax (tcgen05 W2 product, activations in TMEM, L_base and the argmax fused)"
+                       : "a tcgen05 W2 GEMM with the argmax in its epilogue") +
+           ", the GRU input half (" +
            std::string("embedding gather + W_ih GEMM, tiles 128x") + std::to_string(bn_i) + " K-split " +
            std::to_string(ks_i) + ", or a projection-table gather), k_cell, and one stacked W_hh|W1 GEMM (tiles 128x" +
            std::to_string(bn_h) + " K-split " + std::to_string(ks_h) + ") for the next gh and activations; k_tokens";
@@ -314,10 +316,17 @@ int domino_draft_greedy(const domino_shape_t* shape, const domino_weights_t* w, 
         const size_t row0 = (size_t)b0 * s.L + i;                   // (row b0, position i)
         // epochs distinct per launch of this call (the claims were zeroed above)
         const uint32_t epoch = (uint32_t)(i * ((s.B + 127) / 128) + b0 / 128 + 1);
-        e = gemm_tc_argmax(ws.u16 + (size_t)b0 * s.r, (const bf*)w->W2, std::min(128, s.B - b0), s.V, s.r,
-                           (const bf*)base_logits + row0 * s.V, (long long)s.L * s.V, ws.keys + (size_t)i * s.B + b0,
-                           logits_out ? logits_out + row0 * s.V : nullptr, (long long)s.L * s.V, st, spin_limit(),
-                           cs, ws.claim, epoch);
+        const bf* Ub = ws.u16 + (size_t)b0 * s.r;
+        const bf* Lbp = (const bf*)base_logits + row0 * s.V;
+        const int Mb = std::min(128, s.B - b0);
+        float* lo = logits_out ? logits_out + row0 * s.V : nullptr;
+        if (w2_argmax_supported(Mb, s.V, s.r, Ub, w->W2, Lbp, (long long)s.L * s.V))
+          e = w2_argmax(Ub, (const bf*)w->W2, Mb, s.V, s.r, Lbp, (long long)s.L * s.V, ws.keys + (size_t)i * s.B + b0,
+                        lo, (long long)s.L * s.V, i == s.L - 1 && b0 + 128 >= s.B, st, spin_limit(), cs);
+        else
+          e = gemm_tc_argmax(Ub, (const bf*)w->W2, Mb, s.V, s.r, Lbp, (long long)s.L * s.V,
+                             ws.keys + (size_t)i * s.B + b0, lo, (long long)s.L * s.V, st, spin_limit(), cs, ws.claim,
+                             epoch);
       }
     } else if (e == cudaSuccess) {
       e = launch_w2(s, w->W2, ws.u, s.B, base_logits, s.L, i, ws.keys + (size_t)i * s.B, logits_out, cs);

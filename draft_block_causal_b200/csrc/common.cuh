@@ -64,6 +64,20 @@ __device__ __forceinline__ float key_value(uint64_t k) {
 }
 __device__ __forceinline__ uint64_t umax64(uint64_t a, uint64_t b) { return a > b ? a : b; }
 
+// Fixed-point partial sums.  A sum whose partials arrive from many threads or CTAs in an order
+// that varies from run to run is kept as a signed 64-bit integer count of 2^-32 units: each fp32
+// partial is rounded once to that grid (|error| <= 2^-33) and integer addition is associative, so
+// the total -- and every result computed from it -- is the same bits on every run.  Sums must stay
+// below 2^31 in magnitude.  fix_add works on global and shared memory (generic address).
+constexpr float kFixOne = 4294967296.0f;  // 2^32 units per 1.0
+__device__ __forceinline__ unsigned long long fix_of(float x) {
+  return static_cast<unsigned long long>(__float2ll_rn(x * kFixOne));
+}
+__device__ __forceinline__ void fix_add(unsigned long long* p, float x) { atomicAdd(p, fix_of(x)); }
+__device__ __forceinline__ float fix_value(unsigned long long s) {
+  return __ll2float_rn(static_cast<long long>(s)) * (1.0f / kFixOne);
+}
+
 // First problem wins; the library never clears the word.
 __device__ __forceinline__ void set_status(int32_t* st, int code) { atomicCAS(st, 0, code); }
 

@@ -58,6 +58,15 @@ template <class Epi, class = void> struct GroupsOf {
 template <class Epi> struct GroupsOf<Epi, std::void_t<decltype(Epi::kGroups)>> {
   static constexpr int value = Epi::kGroups;
 };
+// An epilogue whose apply() is warp-cooperative (every lane of a warp calls it with the same column
+// group) states kWarpCoop; the split-K reduction, which hands units to threads individually, never
+// takes it.
+template <class Epi, class = void> struct WarpCoop {
+  static constexpr bool value = false;
+};
+template <class Epi> struct WarpCoop<Epi, std::void_t<decltype(Epi::kWarpCoop)>> {
+  static constexpr bool value = Epi::kWarpCoop;
+};
 template <class Epi> struct EpiWarps {
   static constexpr int kGroups = GroupsOf<Epi>::value;
   static constexpr int kThreads = 64 + 128 * kGroups;
@@ -137,13 +146,18 @@ struct EpiLogitsT {  // logits[n][m] = D + Lb[n][m]   (m = vocabulary row, n = (
 
 // Teacher-forced logits, row-major: m = row (b, i) < M, n = vocabulary column < N:
 //   logits[m * ld + n] = D + Lb[m * ld + n]
-// Each thread owns 16 consecutive columns of one row: two 16-byte loads and four (fp32) or two
-// (bf16) 16-byte stores (rows are 16-byte aligned since V % 8 == 0; n0 is a multiple of 16).
+// Each thread owns 16 consecutive columns of one row (n0 is a multiple of 16; rows are 16-byte
+// aligned since V % 8 == 0).  Full groups are written through a per-warp staging buffer: the warp's
+// 32 rows x 16 columns go to shared memory (16-byte chunks XOR-swizzled so that neither side has
+// bank conflicts) and come back so that each store instruction writes whole 64-byte (fp32) or
+// 32-byte (bf16) row segments -- 8 or 16 rows per instruction instead of 32 scattered 16-byte
+// pieces.  Every lane of the warp calls apply with the same n0.
 template <typename OutT>
 struct EpiLogitsRowT {
   static constexpr bool kSide = false;
   static constexpr bool kARes = false;
   static constexpr int kGroups = 2;  // the epilogue is the longest phase of a tile: two warps per lane quadrant
+  static constexpr bool kWarpCoop = true;
   using State = NoState;
   const bf16* Lb;
   OutT* logits;
@@ -153,38 +167,68 @@ struct EpiLogitsRowT {
   __device__ __forceinline__ void finish(State&, int) const {}
   __device__ __forceinline__ void apply(State&, int m, int n0, const float (&v)[16], int N, const uint8_t*, int,
                                         int) const {
-    if (m >= M) return;
-    const bf16* lr = Lb + (size_t)m * ld + n0;
-    OutT* o = logits + (size_t)m * ld + n0;
-    if (n0 + 16 <= N) {
-      float a[8], b[8], z[16];
-      widen(__ldg(reinterpret_cast<const uint4*>(lr)), a);
-      widen(__ldg(reinterpret_cast<const uint4*>(lr) + 1), b);
+    const int lane = threadIdx.x & 31;
+    if (n0 + 16 <= N) {  // warp-uniform
+      // per epilogue warp: 32 rows x 16 values (fp32: 64 B a row, four 16-byte chunks)
+      __shared__ __align__(16) uint32_t stage[8][32 * 16];
+      uint32_t* sw = stage[((threadIdx.x >> 5) - 2) & 7];
+      float z[16];
+      if (m < M) {
+        const bf16* lr = Lb + (size_t)m * ld + n0;
+        float a[8], b[8];
+        widen(__ldg(reinterpret_cast<const uint4*>(lr)), a);
+        widen(__ldg(reinterpret_cast<const uint4*>(lr) + 1), b);
 #pragma unroll
-      for (int j = 0; j < 8; ++j) { z[j] = v[j] + a[j]; z[8 + j] = v[8 + j] + b[j]; }
-      if constexpr (std::is_same<OutT, float>::value) {
-        float4* o4 = reinterpret_cast<float4*>(o);
-#pragma unroll
-        for (int q = 0; q < 4; ++q) o4[q] = make_float4(z[4 * q], z[4 * q + 1], z[4 * q + 2], z[4 * q + 3]);
+        for (int j = 0; j < 8; ++j) { z[j] = v[j] + a[j]; z[8 + j] = v[8 + j] + b[j]; }
       } else {
+#pragma unroll
+        for (int j = 0; j < 16; ++j) z[j] = 0.f;
+      }
+      const int mbase = m - lane;  // the row of lane 0 (the warp's rows are consecutive)
+      if constexpr (std::is_same<OutT, float>::value) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          *reinterpret_cast<uint4*>(sw + lane * 16 + ((j ^ ((lane >> 1) & 3)) << 2)) =
+              make_uint4(__float_as_uint(z[4 * j]), __float_as_uint(z[4 * j + 1]), __float_as_uint(z[4 * j + 2]),
+                         __float_as_uint(z[4 * j + 3]));
+        __syncwarp();
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {  // 8 rows a round, 4 lanes (16 bytes each) a row
+          const int r = 8 * i + (lane >> 2), c = lane & 3;
+          const uint4 x = *reinterpret_cast<const uint4*>(sw + r * 16 + ((c ^ ((r >> 1) & 3)) << 2));
+          if (mbase + r < M) *reinterpret_cast<uint4*>(logits + (size_t)(mbase + r) * ld + n0 + 4 * c) = x;
+        }
+      } else {  // bf16: 32 B a row, two 16-byte chunks
         uint32_t w[8];
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
           const __nv_bfloat162 pr = __floats2bfloat162_rn(z[2 * q], z[2 * q + 1]);
           w[q] = *reinterpret_cast<const uint32_t*>(&pr);
         }
-        uint4* o4 = reinterpret_cast<uint4*>(o);
-        o4[0] = make_uint4(w[0], w[1], w[2], w[3]);
-        o4[1] = make_uint4(w[4], w[5], w[6], w[7]);
+#pragma unroll
+        for (int j = 0; j < 2; ++j)
+          *reinterpret_cast<uint4*>(sw + lane * 8 + ((j ^ ((lane >> 2) & 1)) << 2)) =
+              make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+        __syncwarp();
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {  // 16 rows a round, 2 lanes a row
+          const int r = 16 * i + (lane >> 1), c = lane & 1;
+          const uint4 x = *reinterpret_cast<const uint4*>(sw + r * 8 + ((c ^ ((r >> 2) & 1)) << 2));
+          if (mbase + r < M) *reinterpret_cast<uint4*>(logits + (size_t)(mbase + r) * ld + n0 + 8 * c) = x;
+        }
       }
-    } else {
-      float l[16];
-#pragma unroll
-      for (int j = 0; j < 16; ++j) l[j] = (n0 + j < N) ? __bfloat162float(lr[j]) : 0.f;
-#pragma unroll
-      for (int j = 0; j < 16; ++j)
-        if (n0 + j < N) put(o + j, v[j] + l[j]);
+      __syncwarp();  // the buffer is reused by the warp's next group
+      return;
     }
+    if (m >= M) return;
+    const bf16* lr = Lb + (size_t)m * ld + n0;
+    OutT* o = logits + (size_t)m * ld + n0;
+    float l[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) l[j] = (n0 + j < N) ? __bfloat162float(lr[j]) : 0.f;
+#pragma unroll
+    for (int j = 0; j < 16; ++j)
+      if (n0 + j < N) put(o + j, v[j] + l[j]);
   }
 };
 
@@ -432,7 +476,7 @@ __global__ void __launch_bounds__(EpiWarps<Epi>::kThreads, 1)
               const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmS, int M, int N, int K,
               Epi epi, int32_t* status, unsigned long long limit, int a_kwrap, int a_split, int ksplit,
               int a_stream, int indep, uint32_t* __restrict__ claim, uint32_t epoch,
-              unsigned long long* __restrict__ trace) {
+              unsigned long long* __restrict__ trace, int mfirst) {
   static_assert(!SPLIT || (!Epi::kSide && !Epi::kARes), "split-K needs a plain epilogue");
   using C = Cfg<BN, Epi::kSide, Epi::kARes, SPLIT>;
   constexpr int S = C::kStages;
@@ -495,6 +539,10 @@ __global__ void __launch_bounds__(EpiWarps<Epi>::kThreads, 1)
 
   const int m_tiles = (M + kBM - 1) / kBM, n_tiles = (N + BN - 1) / BN, kblocks = K / kBK;
   const int tiles = m_tiles * n_tiles;
+  // output tile -> (first row, first column): N-tiles within an M band (default), or the M bands of
+  // one N tile in turn (mfirst: CTAs that run at the same time then share each B tile through L2)
+  auto tile_m0 = [&](int tile) { return (mfirst ? tile % m_tiles : tile / n_tiles) * kBM; };
+  auto tile_n0 = [&](int tile) { return (mfirst ? tile / m_tiles : tile % n_tiles) * BN; };
   // item t: output tile t / ksplit, K piece t % ksplit.  With ksplit > 1 the grid has one CTA per
   // item and the CTAs of a tile form one cluster (piece = rank in the cluster).
   const int items = tiles * ksplit;
@@ -510,7 +558,7 @@ __global__ void __launch_bounds__(EpiWarps<Epi>::kThreads, 1)
         int boxes = 0;
         for (int t = slot; t < items && boxes < 64; t += gridDim.x) {
           const int tile = t / ksplit, piece = t - tile * ksplit;
-          const int m0 = (tile / n_tiles) * kBM, n0 = (tile % n_tiles) * BN;
+          const int m0 = tile_m0(tile), n0 = tile_n0(tile);
           const int kb0 = piece * kblocks / ksplit, kb1 = (piece + 1) * kblocks / ksplit;
           const bool second = a_split && m0 >= a_split;
           for (int kb = kb0; kb < kb1; ++kb, ++boxes) {
@@ -534,7 +582,7 @@ __global__ void __launch_bounds__(EpiWarps<Epi>::kThreads, 1)
       }
       for (int t = slot; t < items && ok; t += gridDim.x) {
         const int tile = t / ksplit, piece = t - tile * ksplit;
-        const int m0 = (tile / n_tiles) * kBM, n0 = (tile % n_tiles) * BN;
+        const int m0 = tile_m0(tile), n0 = tile_n0(tile);
         const int kb0 = piece * kblocks / ksplit, kb1 = (piece + 1) * kblocks / ksplit;
         // rows at and past a_split come from the second A operand
         const bool second = a_split && m0 >= a_split;
@@ -546,7 +594,7 @@ __global__ void __launch_bounds__(EpiWarps<Epi>::kThreads, 1)
           const int ta2i = t + 2 * (int)gridDim.x;
           if (ta2i < items) {
             const int tile2 = ta2i / ksplit;
-            const int m2 = (tile2 / n_tiles) * kBM, n2 = (tile2 % n_tiles) * BN;
+            const int m2 = tile_m0(tile2), n2 = tile_n0(tile2);
             if constexpr (Epi::kARes)
               for (int kb = 0; kb < kblocks; ++kb) tma_prefetch_l2(&tmB, kb * kBK, n2);
             if constexpr (Epi::kSide)  // normal priority: the lines must survive until the side load
@@ -639,7 +687,7 @@ __global__ void __launch_bounds__(EpiWarps<Epi>::kThreads, 1)
     auto side_load = [&](uint32_t j, int t) -> bool {
       if constexpr (Epi::kSide) {
         if (!mbar_wait_bounded(&sidee[j & 1u], ((j >> 1) & 1u) ^ 1u, limit, abort_s)) return false;
-        const int m0 = (t / n_tiles) * kBM, n0 = (t % n_tiles) * BN;
+        const int m0 = tile_m0(t), n0 = tile_n0(t);
         mbar_arrive_expect_tx(&sidef[j & 1u], (uint32_t)C::kSideBytes);
         // the side operand (base logits) is read once: evict it first so that B stays in L2
         const uint64_t pol = l2_policy_evict_first();
@@ -663,7 +711,7 @@ __global__ void __launch_bounds__(EpiWarps<Epi>::kThreads, 1)
       if (Epi::kSide && !mbar_wait_warp(&sidef[a], aph, limit, abort_s)) { *abort_s = 1; break; }
       tmem_fence_after_sync();
       const int tile = t / ksplit;
-      const int m0 = (tile / n_tiles) * kBM, n0 = (tile % n_tiles) * BN;
+      const int m0 = tile_m0(tile), n0 = tile_n0(tile);
       const int row = q * 32 + lane;
       const int m = m0 + row;
       const uint32_t taddr = tbase + ((uint32_t)(q * 32) << 16) + a * BN;
@@ -758,7 +806,7 @@ __global__ void __launch_bounds__(EpiWarps<Epi>::kThreads, 1)
     if (warp >= 2) {
       constexpr int U = C::kUnits;
       const int tile = blockIdx.x / ksplit, piece = blockIdx.x - tile * ksplit;
-      const int m0 = (tile / n_tiles) * kBM, n0 = (tile % n_tiles) * BN;
+      const int m0 = tile_m0(tile), n0 = tile_n0(tile);
       const int nmax = (U + ksplit - 1) / ksplit;
       const int u0 = unit_first(piece, ksplit, U), u1 = unit_first(piece + 1, ksplit, U);
       const uint8_t* recv = recv_buf;
@@ -825,12 +873,6 @@ bool tmap_bf16(CUtensorMap* tm, const void* base, uint64_t rows, uint64_t cols, 
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-int sm_count() {
-  int dev = 0, n = 0;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-  return n;
-}
 
 // Fills g_sm_rank once per device (two small launches on `st`, no host synchronisation).
 cudaError_t ensure_sm_rank(cudaStream_t st) {
@@ -868,7 +910,7 @@ cudaError_t launch_gemm(const void* A, const void* Bm, int M, int N, int K, cons
                         uint64_t limit, cudaStream_t st, uint64_t lda = 0, uint64_t ldb = 0, int a_kwrap = 0,
                         const void* side = nullptr, uint64_t lds = 0, const void* A2 = nullptr, int a_split = 0,
                         uint64_t lda2 = 0, int ksplit = 1, int a_stream = 0, int indep = 0,
-                        uint32_t* claim = nullptr, uint32_t epoch = 0) {
+                        uint32_t* claim = nullptr, uint32_t epoch = 0, int mfirst = 0) {
   CUtensorMap ta, ta2, tb, ts;
   const uint64_t ka = a_kwrap ? (uint64_t)a_kwrap : (uint64_t)K;
   const uint64_t rows_a = a_split ? (uint64_t)a_split : (uint64_t)M;
@@ -891,7 +933,7 @@ cudaError_t launch_gemm(const void* A, const void* Bm, int M, int N, int K, cons
   int ntrace = 0;
   debug_trace(&trace, &ntrace);
   if (trace && (long long)ntrace < grid_ctas * kTraceSlots) trace = nullptr;
-  if constexpr (!Epi::kSide && !Epi::kARes) {
+  if constexpr (!Epi::kSide && !Epi::kARes && !WarpCoop<Epi>::value) {
     if (ksplit > 1) {  // one cluster of ksplit CTAs per output tile
       if (ksplit > 8 || K / kBK < ksplit || tiles * ksplit > (1LL << 30)) return cudaErrorInvalidValue;
       auto kern = k_gemm_tc<BN, Epi, true>;
@@ -914,7 +956,7 @@ cudaError_t launch_gemm(const void* A, const void* Bm, int M, int N, int K, cons
     cfg.numAttrs = 2;
     return note_launch(cudaLaunchKernelEx(&cfg, kern, ta, ta2, tb, ts, M, N, K, epi, status,
                                           (unsigned long long)limit, a_kwrap, a_split, ksplit, a_stream, indep,
-                                          (uint32_t*)nullptr, 0u, trace));
+                                          (uint32_t*)nullptr, 0u, trace, 0));
     }
   }
   if (ksplit > 1) return cudaErrorInvalidValue;
@@ -925,7 +967,7 @@ cudaError_t launch_gemm(const void* A, const void* Bm, int M, int N, int K, cons
   const int grid = (int)grid_ctas;
   return note_launch(launch_pdl(kern, dim3(grid), dim3(EpiWarps<Epi>::kThreads), smem, st, ta, ta2, tb, ts, M, N, K, epi, status,
                                 (unsigned long long)limit, a_kwrap, a_split, 1, a_stream, indep,
-                                grid == sm_count() ? claim : nullptr, epoch, trace));
+                                grid == sm_count() ? claim : nullptr, epoch, trace, mfirst));
 }
 
 // A is a weight operand (no earlier kernel writes it): its first tiles are prefetched to L2.
@@ -1046,6 +1088,17 @@ cudaError_t launch_gemm_skinny(const void* A, const void* Bm, int M, int N, int 
 
 }  // namespace
 
+bool tmap_bf16_tiles(CUtensorMap* tm, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows, uint64_t ld) {
+  return tmap_bf16(tm, base, rows, cols, box_rows, ld);
+}
+
+int sm_count() {
+  int dev = 0, n = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n;
+}
+
 cudaError_t gemm_tc_debug(const bf16* A, const bf16* Bm, int M, int N, int K, int a_kwrap, float* out, long long ldo,
                           int trans, int bn, int ks, int32_t* status, uint64_t limit, cudaStream_t st) {
   EpiStore e{out, M, ldo, trans};
@@ -1120,8 +1173,10 @@ template <typename OutT>
 cudaError_t logits_t(const bf16* W2, const bf16* U, int V, int N, int r, const bf16* Lb, OutT* logits, int32_t* status,
                      uint64_t limit, cudaStream_t st) {
   if (N >= 64) {  // enough rows for the row-major orientation: vector loads and stores in the epilogue
+    // the row bands of one vocabulary tile run side by side, so each W2 tile is read from HBM once
     EpiLogitsRowT<OutT> e{Lb, logits, N, (long long)V};
-    return launch_gemm<256>(U, W2, N, V, r, e, status, limit, st, 0, 0, 0, nullptr, 0, nullptr, 0, 0, 1, 0, 2);
+    return launch_gemm<256>(U, W2, N, V, r, e, status, limit, st, 0, 0, 0, nullptr, 0, nullptr, 0, 0, 1, 0, 2,
+                            nullptr, 0, 1);
   }
   EpiLogitsT<OutT> e{Lb, logits, V};
   return launch_gemm_bn(W2, U, V, N, r, e, status, limit, st);

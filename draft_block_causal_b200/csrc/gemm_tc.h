@@ -1,6 +1,7 @@
 // gemm_tc.h -- host entry points of the tcgen05 GEMM (gemm_tc.cu).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -10,6 +11,13 @@
 
 namespace domino {
 
+// A bf16 matrix [rows x cols] (row stride ld elements; 0 = cols) as a TMA tensor map of
+// box_rows x 64 tiles with 128-byte swizzling -- the shared-memory layout the tcgen05 descriptors
+// of this library expect.  False when the driver's encoder is missing or refuses the map.
+bool tmap_bf16_tiles(CUtensorMap* tm, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows,
+                     uint64_t ld = 0);
+// SM count of the current device.
+int sm_count();
 
 // True when the tensor-core GEMM handles these sizes and pointers (K a multiple of 64, 16-byte
 // aligned operands, the driver's tensor-map encoder available).
@@ -32,6 +40,16 @@ cudaError_t gemm_tc_argmax(const __nv_bfloat16* U, const __nv_bfloat16* W2, int 
                            const __nv_bfloat16* Lb, long long ldl, uint64_t* keys, float* out, long long ldo,
                            int32_t* status, uint64_t limit, cudaStream_t st, uint32_t* claim = nullptr,
                            uint32_t epoch = 0);
+
+// The same greedy step as gemm_tc_argmax on the dedicated kernel of w2_argmax.cu (activations
+// resident in TMEM, W2 kept in L2 across positions, balanced vocabulary ranges): M <= 128 rows,
+// r a multiple of 64 up to 256, U, W2 and Lb 16-byte aligned, Lb's row stride ldl (elements) a
+// multiple of 8.  w2_argmax_supported tells whether a call qualifies.  last: this is the call's last
+// read of W2 (its lines are then marked evict-first rather than evict-last).
+bool w2_argmax_supported(int M, int V, int r, const void* U, const void* W2, const void* Lb, long long ldl);
+cudaError_t w2_argmax(const __nv_bfloat16* U, const __nv_bfloat16* W2, int M, int V, int r, const __nv_bfloat16* Lb,
+                      long long ldl, uint64_t* keys, float* out, long long ldo, bool last, int32_t* status,
+                      uint64_t limit, cudaStream_t st);
 
 // u16[n][k] = bf16(SiLU(P[n * ldp + k] + sum_j W1s[k][j] S[n][j])) for k < r, n < N, where the
 // fp32 state arrives as its two-term bf16 split S_hl [N x 2Hs] and W1s [r x Hs] has row stride ldw

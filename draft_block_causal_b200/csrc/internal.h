@@ -36,7 +36,8 @@ struct Workspace {
   float* Gx;           // [B*L][3Hs] W_ih . x for every gathered row
   float* Gh;           // [B][3Hs] W_hh . S
   __nv_bfloat16* S_hl; // [B*L][2Hs] two-term bf16 split of states
-  float* a_acc;        // [L][kAccReplicas][B][r] pre-activation accumulators of the fused kernels
+  unsigned long long* a_acc;  // [2][kAccReplicas][B][r] W1 state-block sums of the fused kernels
+                              // (fixed point, see fix_add; ping-pong over positions)
   size_t bytes;
 };
 constexpr int kSyncWords = 64;
@@ -44,6 +45,8 @@ constexpr int kClaimWords = 1024;
 // The fused greedy kernels spread the W1 state-block partial sums over this many copies of the
 // accumulator (fewer atomics per address); the reader adds the copies.
 constexpr int kAccReplicas = 4;
+// Bytes of the fused kernels' accumulator ping-pong for B rows of rank r.
+constexpr size_t acc_bytes(int B, int r) { return (size_t)2 * kAccReplicas * B * r * sizeof(unsigned long long); }
 
 Workspace layout_workspace(const Shape& s, void* base);
 

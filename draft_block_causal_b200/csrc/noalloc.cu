@@ -18,7 +18,8 @@ namespace domino {
 namespace {
 
 // Scratch of the fused greedy kernel: status word, barrier counter, argmax keys, the W1
-// accumulators and the state ping-pong.  DOMINO_NOALLOC_SCRATCH_BYTES bytes per device.
+// accumulators, the H-projections and the state ping-pong.  DOMINO_NOALLOC_SCRATCH_BYTES bytes
+// per device.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[DOMINO_NOALLOC_SCRATCH_BYTES];
 
 constexpr int kMaxDevices = 64;
@@ -42,7 +43,8 @@ Workspace compact_layout(const Shape& s, void* base) {
   w.status = reinterpret_cast<int32_t*>(take(sizeof(int32_t)));
   w.sync = reinterpret_cast<uint32_t*>(take(kSyncWords * sizeof(uint32_t)));
   w.keys = reinterpret_cast<uint64_t*>(take(BL * sizeof(uint64_t)));
-  w.a_acc = reinterpret_cast<float*>(take(BL * s.r * kAccReplicas * sizeof(float)));
+  w.a_acc = reinterpret_cast<unsigned long long*>(take(acc_bytes(s.B, s.r)));
+  w.P = reinterpret_cast<float*>(take(BL * s.r * sizeof(float)));
   w.S = reinterpret_cast<float*>(take(2 * (size_t)s.B * s.Hs * sizeof(float)));
   w.bytes = off;
   return w;
@@ -77,11 +79,10 @@ extern "C" int domino_draft_greedy_noalloc(const domino_shape_t* shape, const do
                                            int32_t* tokens_out, float* logits_out, float* states_out,
                                            int32_t* status_dev, domino_stream_t stream) {
   auto a16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
-  if (!shape || !w) return DOMINO_ERR_INVALID_ARGUMENT;
-  if (domino_workspace_bytes(shape) == 0) return DOMINO_ERR_INVALID_ARGUMENT;  // shape checks
-  const void* wp[] = {w->embed, w->W_ih, w->W_hh, w->b_ih, w->b_hh, w->W1, w->W2};
-  for (const void* q : wp)
-    if (!q || !a16(q)) return DOMINO_ERR_INVALID_ARGUMENT;
+  int rc = check_shape(shape);
+  if (rc != DOMINO_OK) return rc;
+  // the same weight checks as domino_draft_greedy, the optional projection table included
+  if ((rc = check_weights(w)) != DOMINO_OK) return rc;
   if (!base_logits || !hidden || !S0 || !tokens_out) return DOMINO_ERR_INVALID_ARGUMENT;
   if (!a16(base_logits) || !a16(hidden) || !a16(S0) || !a16(tokens_out) || (logits_out && !a16(logits_out)) ||
       (states_out && !a16(states_out)))

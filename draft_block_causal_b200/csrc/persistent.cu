@@ -8,17 +8,20 @@
 // with one CTA per SM for the whole block.  The 16 positions are sequential through the argmax,
 // so the kernel walks them in a loop separated by bounded grid-wide barriers:
 //
-//   prologue  a_acc[i] += W1[:, :d] . H[b,i] for every i (rank rows split over CTAs)
+//   prologue  P[i] = W1[:, :d] . H[b,i] for every i (rank rows split over CTAs)
 //             a_acc[0] += W1[:, d:] . S0   (each CTA adds the part of its own GRU units)
 //   -- barrier --
-//   step i    u = SiLU(a_acc[i]) in every CTA (r floats per row)
+//   step i    u = SiLU(P[i] + a_acc[i & 1]) in every CTA (r floats per row)
 //             gh = W_hh . S_{i-1} for the CTA's GRU units (independent of the argmax)
 //             z = L_base + W2 . u over the CTA's contiguous vocabulary slice; per-CTA argmax
 //             folded into one u64 key per row with atomicMax (value, then lowest index)
 //   -- barrier --
 //             t_i from the key; gi = W_ih . embed[t_i] for the CTA's units; GRU cell -> S_i
-//             a_acc[i+1] += W1[:, d:] (own columns) . S_i   (float4 atomics)
+//             a_acc[(i+1) & 1] += W1[:, d:] (own columns) . S_i
 //   -- barrier --
+// Sums that several CTAs or warps add into (a_acc, and the gate sums in shared memory) are kept
+// in 64-bit fixed point (fix_add): the order of the atomics does not change a bit, so repeated
+// calls on the same inputs give identical outputs.
 //
 // Weights stream from L2/HBM with 16-byte loads straight into registers.  The W2 rows of a warp
 // are reduced eight at a time with a transpose-reduction (9 shuffles per 8 rows).  Every wait
@@ -26,6 +29,8 @@
 // status word and every CTA returns (no copy or TMEM is ever held across a wait).
 #include "common.cuh"
 #include "persistent.h"
+
+#include <atomic>
 
 #include <algorithm>
 
@@ -47,7 +52,8 @@ struct PArgs {
   float* logits;
   float* states;
   uint64_t* keys;   // [L][B]
-  float* a_acc;     // [L][B][r]
+  unsigned long long* a_acc;  // [2][kAccReplicas][B][r] W1 state-block sums, fixed point
+  float* P;         // [L][B][r] W1[:, :d] . H[b, i]
   float* Sbuf;      // [2][B][Hs]
   unsigned* bar;    // grid barrier counter (zeroed before launch)
   int32_t* status;
@@ -120,11 +126,12 @@ __device__ __forceinline__ void fma8(const uint4& q, const float (&x)[8], float&
 
 // CTA-wide dot products of `nrows` rows of a bf16 matrix (row length K, a multiple of kSeg) with
 // up to kMaxB input vectors held in shared memory (fp32 [BMAX][K] or bf16 [BMAX][K]), adding the
-// results into acc_s[b * acc_stride + row].  Work items are (row, K-segment) pairs, four per warp
-// iteration, reduced with one transpose-reduction.  row_ptr(row) gives the row's address.
+// results into acc_s[b * acc_stride + row] (fixed point).  Work items are (row, K-segment) pairs,
+// four per warp iteration, reduced with one transpose-reduction.  row_ptr(row) gives the row's
+// address.
 template <int BMAX, typename In, typename RowPtr>
-__device__ void cta_rows_dot(RowPtr row_ptr, int nrows, int K, const In* in_s, int B, float* acc_s, int acc_stride,
-                             int warp, int lane) {
+__device__ void cta_rows_dot(RowPtr row_ptr, int nrows, int K, const In* in_s, int B, unsigned long long* acc_s,
+                             int acc_stride, int warp, int lane) {
   const int nseg = K / kSeg;
   const int nitems = nrows * nseg;
   for (int base = warp * 4; base < nitems; base += kPWarps * 4) {
@@ -166,7 +173,7 @@ __device__ void cta_rows_dot(RowPtr row_ptr, int nrows, int K, const In* in_s, i
       if (b < B) {
         const float s = transpose_reduce<4>(acc[b], lane);
         const int it = base + (lane >> 3);
-        if ((lane & 7) == 0 && it < nitems) atomicAdd(acc_s + b * acc_stride + it / nseg, s);
+        if ((lane & 7) == 0 && it < nitems) fix_add(acc_s + b * acc_stride + it / nseg, s);
       }
     }
   }
@@ -187,9 +194,10 @@ __global__ void __launch_bounds__(kPThreads, 1) k_greedy_persistent(PArgs p) {
   float* S_s = u_s + BMAX * kR;                                      // [BMAX][Hs]  S_{i-1}
   bf16* x_s = reinterpret_cast<bf16*>(S_s + (size_t)BMAX * Hs);      // [BMAX][d]   embed[t_i]
   float* w1s_s = reinterpret_cast<float*>(x_s + (size_t)BMAX * d);   // [maxu][kR]  W1[:, d + j0 + jj]
-  float* gh_s = w1s_s + (size_t)maxu * kR;                           // [BMAX][3*maxu]
-  float* gi_s = gh_s + BMAX * 3 * maxu;                              // [BMAX][3*maxu]
-  float* sn_s = gi_s + BMAX * 3 * maxu;                              // [BMAX][maxu]  S_i (own units)
+  // gate sums, fixed point (8-byte aligned: every piece before them is a multiple of 16 bytes)
+  unsigned long long* gh_s = reinterpret_cast<unsigned long long*>(w1s_s + (size_t)maxu * kR);  // [BMAX][3*maxu]
+  unsigned long long* gi_s = gh_s + BMAX * 3 * maxu;                 // [BMAX][3*maxu]
+  float* sn_s = reinterpret_cast<float*>(gi_s + BMAX * 3 * maxu);    // [BMAX][maxu]  S_i (own units)
   uint64_t* best_s = reinterpret_cast<uint64_t*>(sn_s + ((BMAX * maxu + 3) & ~3));  // [kPWarps][BMAX]
   int* flag_s = reinterpret_cast<int*>(best_s + kPWarps * BMAX);
   unsigned epoch = 0;
@@ -199,8 +207,9 @@ __global__ void __launch_bounds__(kPThreads, 1) k_greedy_persistent(PArgs p) {
     const int jj = k / kR, kk = k % kR;
     w1s_s[k] = (jj < nu) ? __bfloat162float(p.W1[(size_t)kk * ldw1 + d + j0 + jj]) : 0.f;
   }
-  for (int k = tid; k < BMAX * 6 * maxu; k += kPThreads) gh_s[k] = 0.f;  // gh_s and gi_s
-  // a_acc[i][b][k] += W1[k, :d] . H[b, i]   for the rank rows k = c, c + G, ...
+  for (int k = tid; k < BMAX * 6 * maxu; k += kPThreads) gh_s[k] = 0ull;  // gh_s and gi_s
+  const int rep = c % kAccReplicas;
+  // P[i][b][k] = W1[k, :d] . H[b, i]   for the rank rows k = c, c + G, ... (one warp per value)
   {
     const int nk = (kR - c + G - 1) / G;  // rank rows owned by this CTA
     const int npos = B * L;
@@ -217,11 +226,12 @@ __global__ void __launch_bounds__(kPThreads, 1) k_greedy_persistent(PArgs p) {
       }
       acc = warp_sum(acc);
       const int b = n / L, i = n % L;
-      if (lane == 0) atomicAdd(p.a_acc + ((size_t)i * B + b) * kR + k, acc);
+      if (lane == 0) p.P[((size_t)i * B + b) * kR + k] = acc;
     }
   }
   __syncthreads();
-  // a_acc[0][b] += W1[:, d + own units] . S0[b, own units];  states_out[b, 0] = S0[b]
+  // a_acc[0][rep][b] += W1[:, d + own units] . S0[b, own units];  states_out[b, 0] = S0[b]
+  // (slot 1 is zero at launch; slot i & 1 is cleared again once every CTA has read it)
   for (int t = tid; t < BMAX * (kR / 4); t += kPThreads) {
     const int b = t / (kR / 4), k4 = (t % (kR / 4)) * 4;
     if (b < B && nu > 0) {
@@ -231,7 +241,8 @@ __global__ void __launch_bounds__(kPThreads, 1) k_greedy_persistent(PArgs p) {
         const float* w = w1s_s + jj * kR + k4;
         s.x = fmaf(w[0], h, s.x); s.y = fmaf(w[1], h, s.y); s.z = fmaf(w[2], h, s.z); s.w = fmaf(w[3], h, s.w);
       }
-      atomicAdd(reinterpret_cast<float4*>(p.a_acc + (size_t)b * kR + k4), s);
+      unsigned long long* acc = p.a_acc + ((size_t)rep * B + b) * kR + k4;
+      fix_add(acc, s.x); fix_add(acc + 1, s.y); fix_add(acc + 2, s.z); fix_add(acc + 3, s.w);
     }
   }
   if (p.states)
@@ -243,10 +254,18 @@ __global__ void __launch_bounds__(kPThreads, 1) k_greedy_persistent(PArgs p) {
 
   // ---------------- the block, one position at a time ----------------
   for (int i = 0; i < L; ++i) {
-    // u = SiLU(a_acc[i]) ; S_{i-1} into shared memory
+    // u = SiLU(P[i] + the replicas of a_acc[i & 1], added as integers) ; S_{i-1} into shared memory
     for (int t = tid; t < BMAX * kR; t += kPThreads) {
-      const int b = t / kR;
-      u_s[t] = (b < B) ? siluf_(__ldcg(p.a_acc + ((size_t)i * B + b) * kR + (t % kR))) : 0.f;
+      const int b = t / kR, k = t % kR;
+      float a = 0.f;
+      if (b < B) {
+        unsigned long long q = 0ull;
+#pragma unroll
+        for (int r = 0; r < kAccReplicas; ++r)
+          q += __ldcg(p.a_acc + (((size_t)(i & 1) * kAccReplicas + r) * B + b) * kR + k);
+        a = __ldcg(p.P + ((size_t)i * B + b) * kR + k) + fix_value(q);
+      }
+      u_s[t] = (b < B) ? siluf_(a) : 0.f;
     }
     if (i < L - 1) {
       const float* Sprev = (i == 0) ? p.S0 : p.Sbuf + (size_t)((i - 1) & 1) * B * Hs;
@@ -322,6 +341,12 @@ __global__ void __launch_bounds__(kPThreads, 1) k_greedy_persistent(PArgs p) {
     }
     if (!grid_sync(p, epoch, flag_s)) return;
     if (i == L - 1) break;
+    // every CTA has read slot i & 1 (before the barrier just passed): clear this CTA's share of it
+    // for position i + 2, whose sums are added only after the next barrier
+    {
+      const int n = kAccReplicas * B * kR, z0 = (int)((long long)n * c / G), z1 = (int)((long long)n * (c + 1) / G);
+      for (int t = z0 + tid; t < z1; t += kPThreads) p.a_acc[(size_t)(i & 1) * n + t] = 0ull;
+    }
 
     // t_i, x = embed[t_i], gi = W_ih . x for the own units (or gathered from the projection
     // table), GRU cell -> S_i
@@ -329,7 +354,7 @@ __global__ void __launch_bounds__(kPThreads, 1) k_greedy_persistent(PArgs p) {
       for (int t = tid; t < B * 3 * nu; t += kPThreads) {
         const int b = t / (3 * nu), R = t % (3 * nu), g = R / nu, jj = R % nu;
         const int tok = min(max(key_index(__ldcg(p.keys + (size_t)i * B + b)), 0), V - 1);
-        gi_s[b * 3 * maxu + R] = __ldg(p.Xp + (size_t)tok * 3 * Hs + (size_t)g * Hs + j0 + jj);
+        gi_s[b * 3 * maxu + R] = fix_of(__ldg(p.Xp + (size_t)tok * 3 * Hs + (size_t)g * Hs + j0 + jj));
       }
     }
     for (int t = tid; t < (p.Xp ? 0 : B * (d / 8)); t += kPThreads) {
@@ -350,10 +375,10 @@ __global__ void __launch_bounds__(kPThreads, 1) k_greedy_persistent(PArgs p) {
       float gi[3], gh[3];
 #pragma unroll
       for (int g = 0; g < 3; ++g) {
-        gi[g] = gi_s[b * 3 * maxu + g * nu + jj] + __bfloat162float(p.b_ih[(size_t)g * Hs + j]);
-        gh[g] = gh_s[b * 3 * maxu + g * nu + jj] + __bfloat162float(p.b_hh[(size_t)g * Hs + j]);
-        gi_s[b * 3 * maxu + g * nu + jj] = 0.f;
-        gh_s[b * 3 * maxu + g * nu + jj] = 0.f;
+        gi[g] = fix_value(gi_s[b * 3 * maxu + g * nu + jj]) + __bfloat162float(p.b_ih[(size_t)g * Hs + j]);
+        gh[g] = fix_value(gh_s[b * 3 * maxu + g * nu + jj]) + __bfloat162float(p.b_hh[(size_t)g * Hs + j]);
+        gi_s[b * 3 * maxu + g * nu + jj] = 0ull;
+        gh_s[b * 3 * maxu + g * nu + jj] = 0ull;
       }
       const float rg = sigmoidf_(gi[0] + gh[0]);
       const float zg = sigmoidf_(gi[1] + gh[1]);
@@ -364,7 +389,7 @@ __global__ void __launch_bounds__(kPThreads, 1) k_greedy_persistent(PArgs p) {
       if (p.states) p.states[((size_t)b * L + i + 1) * Hs + j] = hn;
     }
     __syncthreads();
-    // a_acc[i+1][b] += W1[:, d + own units] . S_i[b, own units]
+    // a_acc[(i+1) & 1][rep][b] += W1[:, d + own units] . S_i[b, own units]
     for (int t = tid; t < BMAX * (kR / 4); t += kPThreads) {
       const int b = t / (kR / 4), k4 = (t % (kR / 4)) * 4;
       if (b < B && nu > 0) {
@@ -374,7 +399,8 @@ __global__ void __launch_bounds__(kPThreads, 1) k_greedy_persistent(PArgs p) {
           const float* w = w1s_s + jj * kR + k4;
           s.x = fmaf(w[0], h, s.x); s.y = fmaf(w[1], h, s.y); s.z = fmaf(w[2], h, s.z); s.w = fmaf(w[3], h, s.w);
         }
-        atomicAdd(reinterpret_cast<float4*>(p.a_acc + ((size_t)(i + 1) * B + b) * kR + k4), s);
+        unsigned long long* acc = p.a_acc + (((size_t)((i + 1) & 1) * kAccReplicas + rep) * B + b) * kR + k4;
+        fix_add(acc, s.x); fix_add(acc + 1, s.y); fix_add(acc + 2, s.z); fix_add(acc + 3, s.w);
       }
     }
     if (!grid_sync(p, epoch, flag_s)) return;
@@ -390,20 +416,27 @@ __global__ void __launch_bounds__(kPThreads, 1) k_greedy_persistent(PArgs p) {
 size_t smem_bytes(int bmax, int d, int Hs, int maxu) {
   size_t f = (size_t)bmax * kR + (size_t)bmax * Hs;
   size_t bytes = f * 4 + (size_t)bmax * d * 2;
-  bytes += ((size_t)maxu * kR + 6 * (size_t)bmax * maxu + (((size_t)bmax * maxu + 3) & ~(size_t)3)) * 4;
+  bytes += ((size_t)maxu * kR + (((size_t)bmax * maxu + 3) & ~(size_t)3)) * 4 + 6 * (size_t)bmax * maxu * 8;
   bytes += (size_t)kPWarps * bmax * 8 + 16;
   return bytes;
 }
 
-int g_num_sms = 0;
+// SM count of the current device, cached per device index (a process may drive GPUs of
+// different sizes; the cooperative grid has one CTA per SM of the device it runs on).
+constexpr int kMaxDevs = 64;
+std::atomic<int> g_num_sms[kMaxDevs];
 
 int num_sms() {
-  if (g_num_sms == 0) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&g_num_sms, cudaDevAttrMultiProcessorCount, dev);
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (dev < 0 || dev >= kMaxDevs) {
+    int n = 0;
+    return cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess ? n : 0;
   }
-  return g_num_sms;
+  int n = g_num_sms[dev].load(std::memory_order_relaxed);
+  if (n == 0 && cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess)
+    g_num_sms[dev].store(n, std::memory_order_relaxed);
+  return n;
 }
 
 template <int BMAX, int ROWS>
@@ -451,13 +484,13 @@ cudaError_t launch_persistent_greedy(const Shape& s, const domino_weights_t& w, 
   a.b_ih = (const bf16*)w.b_ih; a.b_hh = (const bf16*)w.b_hh; a.W1 = (const bf16*)w.W1; a.W2 = (const bf16*)w.W2;
   a.Lb = (const bf16*)base_logits; a.H = (const bf16*)hidden; a.S0 = S0;
   a.tokens = tokens_out; a.logits = logits_out; a.states = states_out;
-  a.keys = ws.keys; a.a_acc = ws.a_acc; a.Sbuf = ws.S; a.bar = ws.sync; a.status = status;
+  a.keys = ws.keys; a.a_acc = ws.a_acc; a.P = ws.P; a.Sbuf = ws.S; a.bar = ws.sync; a.status = status;
   a.B = s.B; a.L = s.L; a.d = s.d; a.Hs = s.Hs; a.V = s.V;
   a.maxu = (s.Hs + G - 1) / G;
   a.spin_limit = spin;
   a.Xp = w.embed_proj;
   // barrier counter, argmax keys and accumulators are contiguous in the workspace: one memset
-  const size_t zero_bytes = (size_t)((char*)(ws.a_acc + (size_t)s.L * s.B * s.r) - (char*)ws.sync);
+  const size_t zero_bytes = (size_t)((char*)ws.a_acc + acc_bytes(s.B, s.r) - (char*)ws.sync);
   cudaError_t e = cudaMemsetAsync(ws.sync, 0, zero_bytes, st);
   if (e != cudaSuccess) return e;
   const int bmax = s.B <= 1 ? 1 : (s.B <= 2 ? 2 : 4);

@@ -13,8 +13,14 @@
 //     columns [R*d/256, (R+1)*d/256) and the W_hh rows after them (packed bf16 pairs).
 //  2. The W2 stream is register double-buffered (the next chunk's loads are issued before the
 //     current chunk is reduced) and its first chunk is issued between barrier arrival and wait.
+//     The slack of the shared memory reserved to keep one CTA per SM (about 100 KB at B = 1) holds
+//     m of every 8 of its W2 chunks for the whole call (w2_slot), so each position streams only
+//     the rest of its slice from L2.
 //  3. The W1 state-block partials are spread over kRep replicas of the accumulator, cutting the
-//     number of same-address atomics per replica from G to G/kRep.
+//     number of same-address atomics per replica from G to G/kRep.  Every partial sum that
+//     several CTAs or warps add into (these accumulators, and the GRU gate sums in shared
+//     memory) is kept in 64-bit fixed point (fix_add), so the order in which the atomics land
+//     does not change a single bit: two calls on the same inputs give identical outputs.
 // Teacher-forced mode (tf_tokens set): the given tokens drive the GRU, so the kernel runs only the
 // L - 1 state updates (TMEM-resident rows, one grid barrier each) and writes every state; the
 // activations and logits of all positions then come from two batched tensor-core products.
@@ -23,6 +29,7 @@
 #include "persistent.h"
 #include "tmem.cuh"
 
+#include <algorithm>
 #include <type_traits>
 
 namespace domino {
@@ -44,7 +51,8 @@ struct TArgs {
   float* logits;
   float* states;
   uint64_t* keys;   // [L][B]
-  float* a_acc;     // [L][kRep][B][r]
+  unsigned long long* a_acc;  // [2][kRep][B][r] W1 state-block sums, fixed point, position i in slot i & 1
+  float* P;         // [L][B][r] W1[:, :d] . H[b, i]
   float* Sbuf;      // [2][B][Hs]
   unsigned* bar;
   int32_t* status;
@@ -55,6 +63,8 @@ struct TArgs {
   const float* Xp;  // [V][3Hs] input projection of the embedding table, or null
   const int32_t* tf_tokens;  // [B][L] given tokens (teacher-forced mode), or null (greedy)
   const float* Gx;           // teacher-forced mode: [B][L-1][3Hs] W_ih . embed[y_i] precomputed, or null
+  int w2m;                   // W2 chunks kept in shared memory per aligned block of 8 (0..8)
+  unsigned w2r_off;          // byte offset of those chunks in dynamic shared memory (16-aligned)
 };
 
 __device__ __forceinline__ unsigned ld_acquire_u32(const unsigned* p) {
@@ -133,10 +143,11 @@ __device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 
 // [col0 + R*cpr, col0 + (R+1)*cpr) of every lane.  Input for batch row b, word c of lane l is
 //   bf16 pair x_t[(b*cpr + c)*128 + l]           (In = uint32_t, the embedding row), or
 //   floats    s_t[(b*2cpr + 2c + {0,1})*128 + l] (In = float, the previous state).
-// Sums go to acc_s[b*acc_stride + R] with shared-memory atomics (4 warps share each row).
+// Sums go to acc_s[b*acc_stride + R] with fixed-point shared-memory atomics (4 warps share each
+// row; the total does not depend on their order).
 template <int BMAX, typename In, int CH>
-__device__ void tmem_rows_dot_ch(uint32_t tbase, int col0, int cpr, int nrows, const In* in_t, int B, float* acc_s,
-                                 int acc_stride, int warp, int lane) {
+__device__ void tmem_rows_dot_ch(uint32_t tbase, int col0, int cpr, int nrows, const In* in_t, int B,
+                                 unsigned long long* acc_s, int acc_stride, int warp, int lane) {
   const int q = warp & 3, group = warp >> 2;
   const int l = q * 32 + lane;
   const uint32_t taddr_lane = tbase + ((uint32_t)(q * 32) << 16);
@@ -187,7 +198,7 @@ __device__ void tmem_rows_dot_ch(uint32_t tbase, int col0, int cpr, int nrows, c
       if (b < B) {
         const float s = transpose_reduce2<4>(acc[b], lane);
         const int R = r0 + 4 * (lane >> 3);
-        if ((lane & 7) == 0 && R < nrows) atomicAdd(acc_s + b * acc_stride + R, s);
+        if ((lane & 7) == 0 && R < nrows) fix_add(acc_s + b * acc_stride + R, s);
       }
     }
   }
@@ -198,11 +209,11 @@ __device__ void tmem_rows_dot_ch(uint32_t tbase, int col0, int cpr, int nrows, c
 // [col0 + R*cpr, col0 + (R+1)*cpr) of every lane.  Input for batch row b, word c of lane l is
 //   bf16 pair x_t[(b*cpr + c)*128 + l]           (In = uint32_t, the embedding row), or
 //   floats    s_t[(b*2cpr + 2c + {0,1})*128 + l] (In = float, the previous state).
-// Sums go to acc_s[b*acc_stride + R] with shared-memory atomics (4 warps share each row).
+// Sums go to acc_s[b*acc_stride + R] in fixed point (see tmem_rows_dot_ch).
 // cpr is even; the widest load that divides it is used.
 template <int BMAX, typename In>
-__device__ void tmem_rows_dot(uint32_t tbase, int col0, int cpr, int nrows, const In* in_t, int B, float* acc_s,
-                              int acc_stride, int warp, int lane) {
+__device__ void tmem_rows_dot(uint32_t tbase, int col0, int cpr, int nrows, const In* in_t, int B,
+                              unsigned long long* acc_s, int acc_stride, int warp, int lane) {
   if (cpr % 8 == 0)
     tmem_rows_dot_ch<BMAX, In, 8>(tbase, col0, cpr, nrows, in_t, B, acc_s, acc_stride, warp, lane);
   else if (cpr % 4 == 0)
@@ -211,13 +222,26 @@ __device__ void tmem_rows_dot(uint32_t tbase, int col0, int cpr, int nrows, cons
     tmem_rows_dot_ch<BMAX, In, 2>(tbase, col0, cpr, nrows, in_t, B, acc_s, acc_stride, warp, lane);
 }
 
+// Shared-memory slot of chunk ch of the CTA's W2 slice, or -1 when the chunk streams from L2: m of
+// every aligned block of 8 chunks are resident, chosen by (ch ^ (ch >> 4)) & 7 < m -- a permutation
+// of each block -- so that every warp (chunks ch = warp + 16k) and every iteration k mixes resident
+// and streamed chunks.
+__device__ __forceinline__ int w2_slot(int ch, int m) {
+  const int rk = (ch ^ (ch >> 4)) & 7;
+  return rk < m ? (ch >> 3) * m + rk : -1;
+}
+
 template <int BMAX, int ROWS>
 __device__ __forceinline__ void w2_load(const TArgs& p, int v0, int v1, int ch, int lane, size_t lrow, int L,
-                                        uint4 (&q)[ROWS], float (&lb)[BMAX]) {
+                                        uint4 (&q)[ROWS], float (&lb)[BMAX], const uint8_t* w2r) {
   const int vb = v0 + ch * ROWS;
+  const int slot = w2_slot(ch, p.w2m);
+  const uint8_t* rs = w2r + (size_t)slot * ROWS * (kR2 * 2) + lane * 16;
 #pragma unroll
   for (int k = 0; k < ROWS; ++k)
-    q[k] = (vb + k < v1) ? ldg16_w2(p.W2 + (size_t)(vb + k) * kR2 + lane * 8) : make_uint4(0u, 0u, 0u, 0u);
+    q[k] = (vb + k < v1) ? (slot >= 0 ? *reinterpret_cast<const uint4*>(rs + k * (kR2 * 2))
+                                      : ldg16_w2(p.W2 + (size_t)(vb + k) * kR2 + lane * 8))
+                         : make_uint4(0u, 0u, 0u, 0u);
   const int v = vb + (lane / (32 / ROWS));
 #pragma unroll
   for (int b = 0; b < BMAX; ++b)
@@ -277,13 +301,16 @@ __global__ void __launch_bounds__(kThreads2, 1) k_greedy_tmem(TArgs p) {
   float* s_t = u_s + BMAX * kR2;                                        // [BMAX][2*cprh][128] S_{i-1}
   uint32_t* x_t = reinterpret_cast<uint32_t*>(s_t + (size_t)BMAX * Hs); // [BMAX][cpri][128]  embed[t_i]
   float* w1s_s = reinterpret_cast<float*>(x_t + (size_t)BMAX * (d / 2));  // [maxu][256]
-  float* gh_s = w1s_s + (size_t)maxu * kR2;                             // [BMAX][3*maxu]
-  float* gi_s = gh_s + BMAX * 3 * maxu;                                 // [BMAX][3*maxu]
-  float* sn_s = gi_s + BMAX * 3 * maxu;                                 // [BMAX][maxu]
+  // gate sums W_hh . S and W_ih . x for the own units, fixed point (8-byte aligned: every piece
+  // before them is a multiple of 8 bytes)
+  unsigned long long* gh_s = reinterpret_cast<unsigned long long*>(w1s_s + (size_t)maxu * kR2);  // [BMAX][3*maxu]
+  unsigned long long* gi_s = gh_s + BMAX * 3 * maxu;                    // [BMAX][3*maxu]
+  float* sn_s = reinterpret_cast<float*>(gi_s + BMAX * 3 * maxu);       // [BMAX][maxu]
   uint64_t* best_s = reinterpret_cast<uint64_t*>(sn_s + ((BMAX * maxu + 3) & ~3));  // [warps][BMAX]
   int* tok_s = reinterpret_cast<int*>(best_s + kWarps2 * BMAX);        // [BMAX]
   int* flag_s = tok_s + BMAX;
   uint32_t* tbase_s = reinterpret_cast<uint32_t*>(flag_s + 1);
+  const uint8_t* w2r = smem + p.w2r_off;  // resident W2 chunks (greedy mode)
   unsigned epoch = 0;
 
   // ---- TMEM: one allocation for the whole call ----
@@ -337,12 +364,25 @@ __global__ void __launch_bounds__(kThreads2, 1) k_greedy_tmem(TArgs p) {
     tmem_wait_st();
   }
   const bool tf = p.tf_tokens != nullptr;
+  // this CTA's resident W2 chunks, once for the call (read after the barrier below)
+  if (!tf && p.w2m > 0) {
+    const int nchunks = (v1 - v0 + ROWS - 1) / ROWS;
+    uint8_t* w2w = smem + p.w2r_off;
+    for (int t = tid; t < nchunks * ROWS * 32; t += kThreads2) {
+      const int ch = t / (ROWS * 32), k = (t / 32) % ROWS, ln = t % 32;
+      const int slot = w2_slot(ch, p.w2m);
+      const int v = v0 + ch * ROWS + k;
+      if (slot >= 0 && v < v1)
+        *reinterpret_cast<uint4*>(w2w + ((size_t)slot * ROWS + k) * (kR2 * 2) + ln * 16) =
+            ldg16(p.W2 + (size_t)v * kR2 + ln * 8);
+    }
+  }
   for (int k = tid; k < maxu * kR2 && !tf; k += kThreads2) {
     const int jj = k / kR2, kk = k % kR2;
     w1s_s[k] = (jj < nu) ? __bfloat162float(p.W1[(size_t)kk * ldw1 + d + j0 + jj]) : 0.f;
   }
-  for (int k = tid; k < BMAX * 6 * maxu; k += kThreads2) gh_s[k] = 0.f;  // gh_s and gi_s
-  // a_acc[i][rep][b][k] += W1[k, :d] . H[b, i]  for the rank rows k = c, c + G, ...
+  for (int k = tid; k < BMAX * 6 * maxu; k += kThreads2) gh_s[k] = 0ull;  // gh_s and gi_s
+  // P[i][b][k] = W1[k, :d] . H[b, i]  for the rank rows k = c, c + G, ... (one warp per value)
   if (!tf) {
     const int nk = (kR2 - c + G - 1) / G;
     const int npos = B * L;
@@ -373,11 +413,12 @@ __global__ void __launch_bounds__(kThreads2, 1) k_greedy_tmem(TArgs p) {
       }
       const float acc = warp_sum(acc0 + acc1);
       const int b = n / L, i = n % L;
-      if (lane == 0) atomicAdd(p.a_acc + (((size_t)i * kRep + rep) * B + b) * kR2 + k, acc);
+      if (lane == 0) p.P[((size_t)i * B + b) * kR2 + k] = acc;
     }
   }
   __syncthreads();
   // a_acc[0][rep][b] += W1[:, d + own units] . S0[b, own units];  states_out[b, 0] = S0[b]
+  // (slot 1 is zero at launch; slot i & 1 is cleared again once every CTA has read it)
   for (int t = tid; t < BMAX * (kR2 / 4) && !tf; t += kThreads2) {
     const int b = t / (kR2 / 4), k4 = (t % (kR2 / 4)) * 4;
     if (b < B && nu > 0) {
@@ -387,7 +428,8 @@ __global__ void __launch_bounds__(kThreads2, 1) k_greedy_tmem(TArgs p) {
         const float* w = w1s_s + jj * kR2 + k4;
         s.x = fmaf(w[0], h, s.x); s.y = fmaf(w[1], h, s.y); s.z = fmaf(w[2], h, s.z); s.w = fmaf(w[3], h, s.w);
       }
-      atomicAdd(reinterpret_cast<float4*>(p.a_acc + ((size_t)rep * B + b) * kR2 + k4), s);
+      unsigned long long* acc = p.a_acc + ((size_t)rep * B + b) * kR2 + k4;
+      fix_add(acc, s.x); fix_add(acc + 1, s.y); fix_add(acc + 2, s.z); fix_add(acc + 3, s.w);
     }
   }
   if (p.states)
@@ -408,7 +450,7 @@ __global__ void __launch_bounds__(kThreads2, 1) k_greedy_tmem(TArgs p) {
 
   stamp(p.trace, p.ntrace, 1);
   grid_arrive(p, epoch);
-  if (!tf && warp < nch) w2_load<BMAX, ROWS>(p, v0, v1, warp, lane, 0, L, qa, lba);
+  if (!tf && warp < nch) w2_load<BMAX, ROWS>(p, v0, v1, warp, lane, 0, L, qa, lba, w2r);
   if (!grid_wait(p, epoch, flag_s)) { leave(); return; }
   stamp(p.trace, p.ntrace, 2);
 
@@ -433,13 +475,15 @@ __global__ void __launch_bounds__(kThreads2, 1) k_greedy_tmem(TArgs p) {
       if (nu > 0) tmem_rows_dot<BMAX, float>(tbase, colh, cprh, 3 * nu, s_t, B, gh_s, 3 * maxu, warp, lane);
       stamp(p.trace, p.ntrace, 4 + 10 * i + 3);
     } else {
-    // u = SiLU(sum of the accumulator replicas); S_{i-1} into the lane-sliced layout
+    // u = SiLU(P + the state block: the accumulator replicas, added as integers)
     for (int t = tid; t < BMAX * kR2; t += kThreads2) {
       const int b = t / kR2, k = t % kR2;
       float a = 0.f;
       if (b < B) {
+        unsigned long long q = 0ull;
 #pragma unroll
-        for (int r = 0; r < kRep; ++r) a += __ldcg(p.a_acc + (((size_t)i * kRep + r) * B + b) * kR2 + k);
+        for (int r = 0; r < kRep; ++r) q += __ldcg(p.a_acc + (((size_t)(i & 1) * kRep + r) * B + b) * kR2 + k);
+        a = __ldcg(p.P + ((size_t)i * B + b) * kR2 + k) + fix_value(q);
       }
       u_s[t] = (b < B) ? siluf_(a) : 0.f;
     }
@@ -466,10 +510,10 @@ __global__ void __launch_bounds__(kThreads2, 1) k_greedy_tmem(TArgs p) {
 #pragma unroll
       for (int b = 0; b < BMAX; ++b) best[b] = 0ull;
       for (int ch = warp; ch < nch; ch += 2 * kWarps2) {
-        if (ch + kWarps2 < nch) w2_load<BMAX, ROWS>(p, v0, v1, ch + kWarps2, lane, lrow, L, qb, lbb);
+        if (ch + kWarps2 < nch) w2_load<BMAX, ROWS>(p, v0, v1, ch + kWarps2, lane, lrow, L, qb, lbb, w2r);
         w2_chunk<BMAX, ROWS>(p, v0, v1, ch, lane, lrow, L, qa, lba, uv, best);
         if (ch + kWarps2 >= nch) break;
-        if (ch + 2 * kWarps2 < nch) w2_load<BMAX, ROWS>(p, v0, v1, ch + 2 * kWarps2, lane, lrow, L, qa, lba);
+        if (ch + 2 * kWarps2 < nch) w2_load<BMAX, ROWS>(p, v0, v1, ch + 2 * kWarps2, lane, lrow, L, qa, lba, w2r);
         w2_chunk<BMAX, ROWS>(p, v0, v1, ch + kWarps2, lane, lrow, L, qb, lbb, uv, best);
       }
 #pragma unroll
@@ -515,6 +559,12 @@ __global__ void __launch_bounds__(kThreads2, 1) k_greedy_tmem(TArgs p) {
     if (!grid_wait(p, epoch, flag_s)) { leave(); return; }
     stamp(p.trace, p.ntrace, tb + 3);
     if (i == L - 1) break;
+    // every CTA has read slot i & 1 (before the barrier just passed): clear this CTA's share of it
+    // for position i + 2, whose sums are added only after the next barrier
+    {
+      const int n = kRep * B * kR2, z0 = (int)((long long)n * c / G), z1 = (int)((long long)n * (c + 1) / G);
+      for (int t = z0 + tid; t < z1; t += kThreads2) p.a_acc[(size_t)(i & 1) * n + t] = 0ull;
+    }
     }  // greedy step
     const int tb = 4 + 10 * i;
 
@@ -524,11 +574,11 @@ __global__ void __launch_bounds__(kThreads2, 1) k_greedy_tmem(TArgs p) {
       for (int t = tid; t < B * 3 * nu; t += kThreads2) {
         const int b = t / (3 * nu), R = t % (3 * nu), g = R / nu, jj = R % nu;
         if (p.Gx) {  // teacher forcing: the gates of (row b, position i) were computed up front
-          gi_s[b * 3 * maxu + R] = __ldg(p.Gx + ((size_t)b * (L - 1) + i) * 3 * Hs + (size_t)g * Hs + j0 + jj);
+          gi_s[b * 3 * maxu + R] = fix_of(__ldg(p.Gx + ((size_t)b * (L - 1) + i) * 3 * Hs + (size_t)g * Hs + j0 + jj));
           continue;
         }
         const int tok = tf ? tok_s[b] : min(max(key_index(__ldcg(p.keys + (size_t)i * B + b)), 0), V - 1);
-        gi_s[b * 3 * maxu + R] = __ldg(p.Xp + (size_t)tok * 3 * Hs + (size_t)g * Hs + j0 + jj);
+        gi_s[b * 3 * maxu + R] = fix_of(__ldg(p.Xp + (size_t)tok * 3 * Hs + (size_t)g * Hs + j0 + jj));
       }
       __syncthreads();
       stamp(p.trace, p.ntrace, tb + 4);
@@ -551,10 +601,10 @@ __global__ void __launch_bounds__(kThreads2, 1) k_greedy_tmem(TArgs p) {
       float gi[3], gh[3];
 #pragma unroll
       for (int g = 0; g < 3; ++g) {
-        gi[g] = gi_s[b * 3 * maxu + g * nu + jj] + __bfloat162float(p.b_ih[(size_t)g * Hs + j]);
-        gh[g] = gh_s[b * 3 * maxu + g * nu + jj] + __bfloat162float(p.b_hh[(size_t)g * Hs + j]);
-        gi_s[b * 3 * maxu + g * nu + jj] = 0.f;
-        gh_s[b * 3 * maxu + g * nu + jj] = 0.f;
+        gi[g] = fix_value(gi_s[b * 3 * maxu + g * nu + jj]) + __bfloat162float(p.b_ih[(size_t)g * Hs + j]);
+        gh[g] = fix_value(gh_s[b * 3 * maxu + g * nu + jj]) + __bfloat162float(p.b_hh[(size_t)g * Hs + j]);
+        gi_s[b * 3 * maxu + g * nu + jj] = 0ull;
+        gh_s[b * 3 * maxu + g * nu + jj] = 0ull;
       }
       const float rg = sigmoidf_(gi[0] + gh[0]);
       const float zg = sigmoidf_(gi[1] + gh[1]);
@@ -575,12 +625,13 @@ __global__ void __launch_bounds__(kThreads2, 1) k_greedy_tmem(TArgs p) {
           const float* w = w1s_s + jj * kR2 + k4;
           s.x = fmaf(w[0], h, s.x); s.y = fmaf(w[1], h, s.y); s.z = fmaf(w[2], h, s.z); s.w = fmaf(w[3], h, s.w);
         }
-        atomicAdd(reinterpret_cast<float4*>(p.a_acc + (((size_t)(i + 1) * kRep + rep) * B + b) * kR2 + k4), s);
+        unsigned long long* acc = p.a_acc + (((size_t)((i + 1) & 1) * kRep + rep) * B + b) * kR2 + k4;
+        fix_add(acc, s.x); fix_add(acc + 1, s.y); fix_add(acc + 2, s.z); fix_add(acc + 3, s.w);
       }
     }
     stamp(p.trace, p.ntrace, tb + 6);
     grid_arrive(p, epoch);
-    if (!tf && warp < nch) w2_load<BMAX, ROWS>(p, v0, v1, warp, lane, lrow + V, L, qa, lba);
+    if (!tf && warp < nch) w2_load<BMAX, ROWS>(p, v0, v1, warp, lane, lrow + V, L, qa, lba, w2r);
     if (!grid_wait(p, epoch, flag_s)) { leave(); return; }
     stamp(p.trace, p.ntrace, tb + 7);
   }
@@ -593,10 +644,15 @@ __global__ void __launch_bounds__(kThreads2, 1) k_greedy_tmem(TArgs p) {
   leave();
 }
 
-size_t smem_bytes_tmem(int bmax, int d, int Hs, int maxu) {
+// Shared memory of the kernel's working arrays (before the resident W2 chunks).
+size_t smem_work_bytes(int bmax, int d, int Hs, int maxu) {
   size_t bytes = ((size_t)bmax * kR2 + (size_t)bmax * Hs) * 4 + (size_t)bmax * (d / 2) * 4;
-  bytes += ((size_t)maxu * kR2 + 6 * (size_t)bmax * maxu + (((size_t)bmax * maxu + 3) & ~(size_t)3)) * 4;
+  bytes += ((size_t)maxu * kR2 + (((size_t)bmax * maxu + 3) & ~(size_t)3)) * 4 + 6 * (size_t)bmax * maxu * 8;
   bytes += (size_t)kWarps2 * bmax * 8 + (size_t)bmax * 4 + 16;
+  return (bytes + 15) & ~(size_t)15;
+}
+size_t smem_bytes_tmem(int bmax, int d, int Hs, int maxu) {
+  const size_t bytes = smem_work_bytes(bmax, d, Hs, maxu);
   return bytes < kMinSmem ? kMinSmem : bytes;
 }
 
@@ -635,17 +691,29 @@ cudaError_t launch_tmem_common(const Shape& s, const domino_weights_t& w, const 
   a.b_ih = (const bf16*)w.b_ih; a.b_hh = (const bf16*)w.b_hh; a.W1 = (const bf16*)w.W1; a.W2 = (const bf16*)w.W2;
   a.Lb = (const bf16*)base_logits; a.H = (const bf16*)hidden; a.S0 = S0;
   a.tokens = tokens_out; a.logits = logits_out; a.states = states_out;
-  a.keys = ws.keys; a.a_acc = ws.a_acc; a.Sbuf = ws.S; a.bar = ws.sync; a.status = status;
+  a.keys = ws.keys; a.a_acc = ws.a_acc; a.P = ws.P; a.Sbuf = ws.S; a.bar = ws.sync; a.status = status;
   a.B = s.B; a.L = s.L; a.d = s.d; a.Hs = s.Hs; a.V = s.V;
   a.maxu = (s.Hs + G - 1) / G;
   a.spin_limit = spin;
   a.Xp = w.embed_proj;
   debug_trace(&a.trace, &a.ntrace);
-  const size_t zero_bytes = (size_t)((char*)(ws.a_acc + (size_t)s.L * kRep * s.B * s.r) - (char*)ws.sync);
+  // barrier counter, argmax keys and accumulators are contiguous in the workspace: one memset
+  const size_t zero_bytes = (size_t)((char*)ws.a_acc + acc_bytes(s.B, s.r) - (char*)ws.sync);
   cudaError_t e = cudaMemsetAsync(ws.sync, 0, zero_bytes, st);
   if (e != cudaSuccess) return e;
   const int bmax = s.B <= 1 ? 1 : (s.B <= 2 ? 2 : 4);
-  const size_t smem = smem_bytes_tmem(bmax, s.d, s.Hs, a.maxu);
+  size_t smem = smem_bytes_tmem(bmax, s.d, s.Hs, a.maxu);
+  if (!tf_tokens) {
+    // greedy: the shared memory reserved to keep one CTA per SM but not used by the working arrays
+    // holds W2 chunks for the whole call.  The reservation is not grown for them: shared memory and
+    // L1 share one array per SM, and the W2 stream needs the L1 capacity for its loads in flight.
+    const int rows = bmax == 4 ? 4 : 8;
+    const size_t work = smem_work_bytes(bmax, s.d, s.Hs, a.maxu), chunk = (size_t)rows * s.r * 2;
+    const int nblk = ((s.V + G - 1) / G + rows * 8 - 1) / (rows * 8);  // aligned blocks of 8 chunks
+    const size_t avail = smem > work ? smem - work : 0;
+    a.w2m = (int)std::min<size_t>(8, avail / (chunk * (size_t)nblk));
+    a.w2r_off = (unsigned)work;
+  }
   if (bmax == 1) e = launch_tmem_t<1, 8>(a, G, smem, st);
   else if (bmax == 2) e = launch_tmem_t<2, 8>(a, G, smem, st);
   else e = launch_tmem_t<4, 4>(a, G, smem, st);

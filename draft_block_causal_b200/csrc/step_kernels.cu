@@ -410,12 +410,16 @@ __global__ void __launch_bounds__(256) k_accept_early(const float* __restrict__ 
   pdl_wait();
   pdl_trigger();
   __shared__ uint64_t red[8];
-  __shared__ bool last_chunk, last_block;
+  __shared__ bool last_chunk, last_block, skip_s;
   const int y = blockIdx.y, j = y / B, b = y % B;
   const size_t n = (size_t)b * L + j;
   uint32_t* const first = count + (size_t)B * L;
   uint32_t* const done = first + B;
-  const bool skip = *reinterpret_cast<volatile uint32_t*>(first + b) > (uint32_t)(L - j);
+  // one read of the row's mismatch word for the whole block: another block may raise it at any
+  // moment, and every thread must take the same branch around the block barriers below
+  if (threadIdx.x == 0) skip_s = *reinterpret_cast<volatile uint32_t*>(first + b) > (uint32_t)(L - j);
+  __syncthreads();
+  const bool skip = skip_s;
   if (!skip) {  // block-uniform
     const int v0 = blockIdx.x * kArgChunk, v1 = min(V, v0 + kArgChunk);
     const float* row = T + n * V;

@@ -38,7 +38,8 @@ EXPORTS = ("domino_workspace_bytes", "domino_draft_greedy", "domino_teacher_forc
            "domino_greedy_plan", "domino_draft_greedy_noalloc", "domino_debug_set_trace",
            "domino_embed_proj_bytes", "domino_project_embeddings", "domino_arena_bytes",
            "domino_pack_weights", "domino_set_l2_persistence", "domino_debug_gemm",
-           "domino_debug_read_passes", "domino_teacher_forced_ex")
+           "domino_debug_read_passes", "domino_teacher_forced_ex", "domino_accept_sample_workspace_bytes",
+           "domino_accept_sample")
 
 
 class DominoError(RuntimeError):
@@ -111,6 +112,10 @@ def lib(path: str = LIB_PATH) -> ctypes.CDLL:
         L.domino_teacher_forced_ex.restype = ctypes.c_int
         L.domino_debug_read_passes.argtypes = [vp, sz, i32, vp]
         L.domino_debug_read_passes.restype = ctypes.c_int
+        L.domino_accept_sample_workspace_bytes.argtypes = [i32, i32, i32]
+        L.domino_accept_sample_workspace_bytes.restype = sz
+        L.domino_accept_sample.argtypes = [i32, i32, i32, vp, vp, vp, ctypes.c_float, vp, vp, vp, vp, sz, vp, vp]
+        L.domino_accept_sample.restype = ctypes.c_int
         _lib = L
     return _lib
 
@@ -511,6 +516,40 @@ def accept_len(draft_tokens, target_logits, accept_out=None, workspace=None, sta
                  _ptr(workspace), workspace.numel(), _ptr(status), _stream(stream, dev))
     _check(rc, "domino_accept_len")
     return accept_out
+
+
+def accept_sample(draft_tokens, target_logits, temperature: float, uniforms, draft_logits=None, accept_out=None,
+                  next_out=None, workspace=None, status=None, stream=None):
+    """Sampled verification (``domino_accept_sample``): returns (accept lengths [B], replacement
+    tokens [B], -1 where every position was accepted).  ``draft_logits`` None means a greedy draft
+    (one-hot draft distribution); ``uniforms`` [B, L + 1] fp32 are the caller's random draws."""
+    if not isinstance(target_logits, torch.Tensor) or target_logits.dim() != 3:
+        raise ValueError("target_logits must be a [B, L, V] tensor")
+    B, L, V = (int(x) for x in target_logits.shape)
+    dev = target_logits.device
+    _expect(target_logits, "target_logits", (B, L, V), torch.float32, dev)
+    if draft_logits is not None:
+        _expect(draft_logits, "draft_logits", (B, L, V), torch.float32, dev)
+    _expect(draft_tokens, "draft_tokens", (B, L), torch.int32, dev)
+    _expect(uniforms, "uniforms", (B, L + 1), torch.float32, dev)
+    if accept_out is None:
+        accept_out = torch.empty((B,), dtype=torch.int32, device=dev)
+    if next_out is None:
+        next_out = torch.empty((B,), dtype=torch.int32, device=dev)
+    _expect(accept_out, "accept_out", (B,), torch.int32, dev)
+    _expect(next_out, "next_out", (B,), torch.int32, dev)
+    _expect_status(status, dev)
+    if workspace is None:
+        n = int(lib().domino_accept_sample_workspace_bytes(B, L, V))
+        if n == 0:
+            raise DominoError(ERR_INVALID_ARGUMENT, "domino_accept_sample_workspace_bytes")
+        workspace = alloc_workspace(n, dev)
+    _expect_workspace(workspace, dev)
+    rc = _launch(dev, lib().domino_accept_sample, B, L, V, _ptr(draft_tokens), _ptr(draft_logits),
+                 _ptr(target_logits), float(temperature), _ptr(uniforms), _ptr(accept_out), _ptr(next_out),
+                 _ptr(workspace), workspace.numel(), _ptr(status), _stream(stream, dev))
+    _check(rc, "domino_accept_sample")
+    return accept_out, next_out
 
 
 def to_device_weights(host: dict, dtype_code: int, device="cuda") -> HeadWeights:

@@ -53,6 +53,9 @@ WORKLOADS = {
     # Qwen3-8B-shaped head, batch sweep (B and peak overridden per point)
     "qwen3-8b-head-sweep": dict(B=1, L=16, d=4096, Hs=1024, r=256, V=151936, dtype=BF16,
                                 weight_seed=0, input_seed=4, s0_std=0.1, peak=4.0),
+    # Qwen3-4B-shaped head, the same batch sweep
+    "qwen3-4b-head-sweep": dict(B=1, L=16, d=2560, Hs=1024, r=256, V=151936, dtype=BF16,
+                                weight_seed=0, input_seed=5, s0_std=0.1, peak=4.0),
 }
 SWEEP_BATCHES = (1, 4, 16, 64, 128, 256)
 SWEEP_PEAKS = (1.0, 2.0, 4.0)

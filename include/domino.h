@@ -213,6 +213,37 @@ DOMINO_API int domino_accept_len(int32_t B, int32_t L, int32_t V, const int32_t*
                       const float* target_logits, int32_t* accept_out, void* workspace,
                       size_t workspace_bytes, int32_t* status_dev, domino_stream_t stream);
 
+/* Sampled (temperature > 0) verification of a draft block.  The pages call Domino's verification
+ * lossless (review page, section 一: the target model checks the whole block in one parallel pass;
+ * researchpapers.dev summary) and spell out only the greedy setting (domino_accept_len).  For a
+ * target that samples at temperature T, this is the published speculative-sampling rule that keeps
+ * verification lossless (Leviathan, Kalman and Matias, ICML 2023; Chen et al. 2023):
+ *   p_j = softmax(target_logits[b, j] / T)
+ *   q_j = softmax(draft_logits[b, j] / T), or, when draft_logits is NULL, the one-hot distribution
+ *         on draft_tokens[b, j] (greedy drafting, as domino_draft_greedy does, is that case)
+ *   position j is accepted when uniforms[b, j] < p_j(x) / q_j(x), x = draft_tokens[b, j]; the row
+ *   stops at its first rejected position k, whose replacement token is drawn from the residual
+ *   max(0, p_k - q_k) by inverse transform with uniforms[b, L]: the smallest v whose running sum
+ *   (ascending v) exceeds uniforms[b, L] times the residual's total.
+ * Inputs: draft_tokens [B, L] int32 (each in [0, V); an out-of-range token sets
+ *         DOMINO_STATUS_BAD_TOKEN and is rejected), draft_logits [B, L, V] fp32 or NULL,
+ *         target_logits [B, L, V] fp32, uniforms [B, L + 1] fp32 in [0, 1) -- the random draws are
+ *         the caller's, so a call is reproducible -- and 0 < temperature < infinity.
+ * Outputs: accept_out [B] int32 = k (L when every position is accepted); next_out [B] int32 = the
+ *          replacement token at position k, or -1 when all L positions were accepted (no bonus
+ *          token: there are no target logits past the block).
+ * Two launches; logits of a row's positions after its first rejection may be left unread (the
+ * result is the same).  Needs domino_accept_sample_workspace_bytes(B, L, V) bytes of workspace
+ * (device memory, 256-byte aligned).  Returns DOMINO_OK, DOMINO_ERR_INVALID_ARGUMENT (null pointer,
+ * misaligned logits, bad shape or temperature), DOMINO_ERR_UNSUPPORTED (B * L > 65535),
+ * DOMINO_ERR_WORKSPACE or DOMINO_ERR_CUDA; nothing is launched on a negative code. */
+DOMINO_API size_t domino_accept_sample_workspace_bytes(int32_t B, int32_t L, int32_t V);
+DOMINO_API int domino_accept_sample(int32_t B, int32_t L, int32_t V, const int32_t* draft_tokens,
+                                    const float* draft_logits, const float* target_logits, float temperature,
+                                    const float* uniforms, int32_t* accept_out, int32_t* next_out,
+                                    void* workspace, size_t workspace_bytes, int32_t* status_dev,
+                                    domino_stream_t stream);
+
 /* Human-readable text for a DOMINO_ERR_* or DOMINO_STATUS_* code (static storage). */
 DOMINO_API const char* domino_status_string(int code);
 
@@ -241,9 +272,9 @@ DOMINO_API const char* domino_greedy_plan(const domino_shape_t* shape);
  * allocated or freed by this call.  Limits:
  *   - only shapes the fused small-batch kernel handles (bf16, r = 256, B <= 4, d and Hs
  *     multiples of 256) are accepted, else DOMINO_ERR_UNSUPPORTED;
- *   - the kernel's scratch (16*B*L*r + 8*B*L + 8*B*Hs + 512 bytes, each piece rounded up to 256)
- *     must fit the array, else DOMINO_ERR_SCRATCH_LIMIT -- e.g. B=4, L=16, Hs=1024 needs
- *     295,936 bytes and fits; B=4, L=64 does not;
+ *   - the kernel's scratch (4*B*L*r + 64*B*r + 8*B*L + 8*B*Hs + 512 bytes, each piece rounded
+ *     up to 256) must fit the array, else DOMINO_ERR_SCRATCH_LIMIT -- e.g. B=4, L=16, Hs=1024
+ *     needs 164,864 bytes and fits; B=4, L=64 needs 363,008 and does not;
  *   - every call on a device shares that device's array, and the array keeps the previous
  *     call's contents (the call clears what must start at zero).  Calls whose kernels overlap
  *     on the GPU -- on different streams, or from different host threads -- race on the array
@@ -252,7 +283,7 @@ DOMINO_API const char* domino_greedy_plan(const domino_shape_t* shape);
  *     with that device current); make that first call before any stream capture begins.
  * status_dev may be NULL (the code then lands in the array).  Returns DOMINO_OK or a negative
  * DOMINO_ERR_* code (nothing launched). */
-#define DOMINO_NOALLOC_SCRATCH_BYTES (1024u * 1024u)
+#define DOMINO_NOALLOC_SCRATCH_BYTES (256u * 1024u)
 DOMINO_API int domino_draft_greedy_noalloc(const domino_shape_t* shape, const domino_weights_t* weights,
                                            const void* base_logits, const void* hidden, const float* S0,
                                            int32_t* tokens_out, float* logits_out, float* states_out,

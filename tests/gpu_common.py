@@ -120,3 +120,73 @@ def accept_parity(draft_tokens: np.ndarray, target: np.ndarray):
     want = oracle.accept_len(np.ascontiguousarray(draft_tokens, dtype=np.int32), target)
     assert np.array_equal(got, want), f"accept length mismatch: {got} vs {want}"
     return got
+
+
+def greedy_parity_rows(data: dict, chunk: int = 16, nthreads: int = 0):
+    """Oracle replay of every row of a large greedy case, in chunks of rows.
+
+    The GPU drafts with logits and states written, and again with neither (the fused-argmax path).
+    Each chunk of rows is replayed teacher-forced on the GPU's tokens and compared element by
+    element (steps 1 and 2).  The no-logits call is replayed only on rows whose tokens differ from
+    the first call's.  Step 3 needs no separate oracle run here: where every earlier token matched
+    the replay's argmax at a margin above MARGIN, the replay of that prefix is the oracle's own
+    greedy path, so the oracle's greedy tokens equal the GPU's up to the first small margin.
+    """
+    sh = data["shape"]
+    B = sh["B"]
+    w, lb, h, S0 = device_inputs(data)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    tok, lg, st = domino.draft_greedy(w, lb, h, S0, logits_out=True, states_out=True, status=status)
+    tok2, _, _ = domino.draft_greedy(w, lb, h, S0, status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    tok = tok.cpu().numpy()
+    tok2 = tok2.cpu().numpy()
+    bl, hh, s0 = data["base_logits"], data["hidden"], data["S0"]
+    le = se = 0.0
+    ndiv = 0
+    for r0 in range(0, B, chunk):
+        rows = list(range(r0, min(B, r0 + chunk)))
+        ref = oracle.head(sh, data["weights"], bl, hh, s0, tokens=np.ascontiguousarray(tok), rows=rows,
+                          nthreads=nthreads)
+        e1, e2 = check_logits_states(lg[r0:rows[-1] + 1].cpu().numpy(), st[r0:rows[-1] + 1].cpu().numpy(), ref,
+                                     f"greedy rows {rows[0]}..{rows[-1]}")
+        le, se = max(le, e1), max(se, e2)
+        ndiv += check_tokens_against_replay(tok[rows], ref, f"greedy rows {rows[0]}..{rows[-1]}")
+        del ref
+    other = [b for b in range(B) if not np.array_equal(tok[b], tok2[b])]
+    for r0 in range(0, len(other), chunk):
+        rows = other[r0:r0 + chunk]
+        ref2 = oracle.head(sh, data["weights"], bl, hh, s0, tokens=np.ascontiguousarray(tok2), rows=rows,
+                           want_states=False, nthreads=nthreads)
+        ndiv += check_tokens_against_replay(tok2[rows], ref2, "greedy (no logits)")
+    return {"tokens": tok, "max_logit_err": le, "max_state_err": se, "small_margin_divergences": ndiv,
+            "rows_replayed_twice": len(other)}
+
+
+def tf_parity_rows(data: dict, chunk: int = 16, nthreads: int = 0, logits_dtype=torch.float32):
+    """Teacher-forced parity on every row, in chunks of rows.  With bf16 logits the bound widens by
+    the rounding of the fp32 value to bf16 (at most 2^-9 of its magnitude)."""
+    sh = data["shape"]
+    B = sh["B"]
+    w, lb, h, S0 = device_inputs(data)
+    y = torch.from_numpy(data["tokens"]).cuda()
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    lg, st = domino.teacher_forced(w, lb, h, S0, y, states_out=True, status=status, logits_dtype=logits_dtype)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    rtol = LOGIT_RTOL + (2.0 ** -9 if logits_dtype == torch.bfloat16 else 0.0)
+    le = se = 0.0
+    for r0 in range(0, B, chunk):
+        rows = list(range(r0, min(B, r0 + chunk)))
+        ref = oracle.head(sh, data["weights"], data["base_logits"], data["hidden"], data["S0"],
+                          tokens=data["tokens"], rows=rows, nthreads=nthreads)
+        gl = lg[r0:rows[-1] + 1].float().cpu().numpy().astype(np.float64)
+        err = np.abs(gl - ref["logits"])
+        bad = err > LOGIT_ATOL + rtol * np.abs(ref["logits"])
+        assert not bad.any(), f"teacher-forced rows {rows[0]}..: {bad.sum()} logits out of tolerance"
+        s = float(np.abs(st[r0:rows[-1] + 1].cpu().numpy().astype(np.float64) - ref["states"]).max())
+        assert s <= STATE_ATOL, f"teacher-forced rows {rows[0]}..: state error {s:.3e}"
+        le, se = max(le, float(err.max())), max(se, s)
+        del ref
+    return {"max_logit_err": le, "max_state_err": se}

@@ -170,7 +170,7 @@ def test_teacher_forced_ex_rejects_a_bad_logits_dtype(L):
 def test_noalloc_limits_are_checked_on_the_host(L):
     w = domino.Weights(*([0x10000] * 7))
     p = ctypes.c_void_p(0x10000)  # never dereferenced: every case fails before any launch
-    # B = 4 rows of 64 positions need more than the 1 MiB scratch array
+    # B = 4 rows of 64 positions need more than the 256 KiB scratch array
     big = domino.Shape(4, 64, 512, 256, 256, 12000, 1)
     assert L.domino_draft_greedy_noalloc(ctypes.byref(big), ctypes.byref(w), p, p, p, p, None, None, None,
                                          None) == domino.ERR_SCRATCH_LIMIT
@@ -184,6 +184,37 @@ def test_noalloc_limits_are_checked_on_the_host(L):
                                          None) == domino.ERR_INVALID_ARGUMENT
     assert L.domino_draft_greedy_noalloc(ctypes.byref(ok), ctypes.byref(w), p, p, p, None, None, None, None,
                                          None) == domino.ERR_INVALID_ARGUMENT  # tokens_out is required
+    # the optional projection table is checked like every other weight: a misaligned one is refused on
+    # the host by both greedy entry points (the fused kernels read it with vector loads)
+    wp = domino.Weights(*([0x10000] * 7 + [0x10004]))
+    assert L.domino_draft_greedy_noalloc(ctypes.byref(ok), ctypes.byref(wp), p, p, p, p, None, None, None,
+                                         None) == domino.ERR_INVALID_ARGUMENT
+    n = L.domino_workspace_bytes(ctypes.byref(ok))
+    assert L.domino_draft_greedy(ctypes.byref(ok), ctypes.byref(wp), p, p, p, p, None, None, p, n, None,
+                                 None) == domino.ERR_INVALID_ARGUMENT
+
+
+def test_accept_sample_checks_its_arguments_on_the_host(L):
+    p = ctypes.c_void_p(0x10000)  # never dereferenced: every case fails before any launch
+    n = L.domino_accept_sample_workspace_bytes(4, 16, 151936)
+    assert n > 0 and n % 256 == 0
+    assert L.domino_accept_sample_workspace_bytes(0, 16, 1000) == 0
+    assert L.domino_accept_sample_workspace_bytes(4, 65, 1000) == 0
+    assert L.domino_accept_sample_workspace_bytes(4, 16, 1001) == 0
+    ok = (4, 16, 151936)
+    # temperature must be positive and finite
+    for t in (0.0, -0.5, float("inf"), float("nan")):
+        assert L.domino_accept_sample(*ok, p, None, p, t, p, p, p, p, n, None, None) == domino.ERR_INVALID_ARGUMENT
+    # required pointers, aligned logits, the workspace
+    assert L.domino_accept_sample(*ok, None, None, p, 1.0, p, p, p, p, n, None, None) == domino.ERR_INVALID_ARGUMENT
+    assert L.domino_accept_sample(*ok, p, None, p, 1.0, None, p, p, p, n, None, None) == domino.ERR_INVALID_ARGUMENT
+    assert L.domino_accept_sample(*ok, p, ctypes.c_void_p(0x10004), p, 1.0, p, p, p, p, n, None,
+                                  None) == domino.ERR_INVALID_ARGUMENT
+    assert L.domino_accept_sample(*ok, p, None, p, 1.0, p, p, p, p, n - 256, None, None) == domino.ERR_WORKSPACE
+    assert L.domino_accept_sample(*ok, p, None, p, 1.0, p, p, p, ctypes.c_void_p(0x10010), n, None,
+                                  None) == domino.ERR_WORKSPACE
+    assert L.domino_accept_sample(5000, 16, 1000, p, None, p, 1.0, p, p, p, p, 1 << 40, None,
+                                  None) == domino.ERR_UNSUPPORTED
 
 
 def test_projection_and_debug_entry_points_check_their_arguments(L):

@@ -216,7 +216,9 @@ def test_batched_teacher_forcing_reports_bad_tokens():
 @pytest.mark.parametrize("B", [1, 8], ids=["vocabulary-major", "row-major"])
 def test_bf16_teacher_forced_logits_are_the_fp32_ones_rounded(B):
     """domino_teacher_forced_ex with bf16 logits writes exactly the fp32 logits of the same call
-    rounded to nearest even (both logits epilogues: B*L < 64 and >= 64)."""
+    rounded to nearest even (both logits epilogues: B*L < 64 and >= 64), and those bf16 logits lie
+    within the stated tolerance of the fp64 oracle, widened by the rounding to bf16 (2^-9 of the
+    value)."""
     data = _persistent_case(B=B, seed=350 + B, Hs=256)
     w, lb, h, S0 = G.device_inputs(data)
     y = torch.randint(0, data["shape"]["V"], (B, 16), dtype=torch.int32, device="cuda")
@@ -225,3 +227,14 @@ def test_bf16_teacher_forced_logits_are_the_fp32_ones_rounded(B):
     torch.cuda.synchronize()
     assert lg16.dtype == torch.bfloat16
     assert torch.equal(lg16, lg32.to(torch.bfloat16))
+    data["tokens"] = y.cpu().numpy()
+    res = G.tf_parity_rows(data, logits_dtype=torch.bfloat16)
+    print("bf16 teacher-forced logits against the oracle", res)
+
+
+def test_bf16_teacher_forced_logits_8b_b32_against_oracle():
+    """bf16 logits at the Qwen3-8B shape, B = 32 (the row-major epilogue), every row against the
+    oracle."""
+    wl = synth.workload("qwen3-8b-head-b32")
+    data = synth.make_workload(wl, with_tokens=True)
+    print(G.tf_parity_rows(data, logits_dtype=torch.bfloat16))

@@ -1,6 +1,6 @@
 """GPU parity: the CUDA path, called through the C ABI, against the fp64 oracle on the same
-seeded inputs (procedure in gpu_common).  Small cases are checked on every output; the full
-Qwen3-shaped workloads on every output of sampled rows (rows are independent)."""
+seeded inputs (procedure in gpu_common).  Every case is checked on every row and every output;
+the large ones row chunk by row chunk."""
 import numpy as np
 import pytest
 import torch
@@ -38,6 +38,12 @@ SMALL = [
     _custom(2, 5, 512, 512, 256, 3000, 1, 200),           # short block, small vocabulary
     _custom(4, 16, 2560, 1024, 256, 20000, 1, 210),       # Qwen3-4B widths, B = 4
     _custom(1, 16, 4096, 1024, 256, 7992, 1, 220, s0_std=1.0, peak=0.5),  # 8B widths, many near-ties
+    # the batched tensor-core path (B > 4) and its W2 argmax kernel: ragged 16-column units, every
+    # supported rank, two batch bands, fewer vocabulary units than SMs, a one-unit vocabulary
+    _custom(7, 5, 256, 128, 64, 1000, 1, 300),            # r = 64, V % 16 = 8
+    _custom(130, 3, 256, 256, 128, 5000, 1, 310),         # bands of 128 and 2 rows, r = 128
+    _custom(40, 16, 512, 256, 256, 2056, 1, 320, s0_std=1.0, peak=0.5),  # 129 units: 129 CTAs
+    _custom(9, 4, 128, 64, 64, 16, 1, 330),               # V = 16: one unit, one CTA
 ]
 
 
@@ -76,23 +82,26 @@ def test_greedy_and_accept_8b_b1():
     print({k: v for k, v in res.items() if k != "tokens"}, "accept", acc)
 
 
-def test_greedy_tf_accept_8b_b32_sampled_rows():
+def test_greedy_tf_accept_8b_b32_every_row():
+    """Qwen3-8B shapes at B = 32 (per-row S0 ~ N(0, 0.1)): greedy, teacher forcing and the accept
+    length against the oracle on every row and every output."""
     wl = synth.workload("qwen3-8b-head-b32")
     data = synth.make_workload(wl, with_tokens=True, with_target=True)
-    rows = [0, 13, 31]
-    res = G.greedy_parity(data, rows=rows)
+    res = G.greedy_parity_rows(data)
     print("greedy", {k: v for k, v in res.items() if k != "tokens"})
-    print("tf", G.tf_parity(data, rows=rows))
+    print("tf", G.tf_parity_rows(data))
     acc = G.accept_parity(res["tokens"], data["target_logits"])
     print("accept", acc)
 
 
-@pytest.mark.parametrize("B,peak", list(zip(synth.SWEEP_BATCHES, (1.0, 2.0, 4.0, 1.0, 2.0, 4.0))))
-def test_greedy_batch_sweep_sampled_rows(B, peak):
+@pytest.mark.parametrize("B,peak", [(B, p) for B in synth.SWEEP_BATCHES for p in synth.SWEEP_PEAKS],
+                         ids=lambda v: str(v))
+def test_greedy_batch_sweep_every_row(B, peak):
+    """The batch sweep, B in {1, 4, 16, 64, 128, 256} crossed with base-logit peaks {+1, +2, +4}:
+    every row replayed by the oracle, with and without logits written."""
     wl = synth.workload("qwen3-8b-head-sweep", B=B, peak=peak)
     data = synth.make_workload(wl)
-    rows = sorted({0, B // 2, B - 1})
-    res = G.greedy_parity(data, rows=rows)
+    res = G.greedy_parity_rows(data)
     print(B, peak, {k: v for k, v in res.items() if k != "tokens"})
 
 

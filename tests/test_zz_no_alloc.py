@@ -70,6 +70,36 @@ def test_noalloc_matches_workspace_entry_point_twice(B, L):
                 assert t[b, i] == tr[b, i], f"call {call}: row {b} position {i}"
 
 
+@pytest.mark.parametrize("B", [1, 4])
+def test_noalloc_tmem_kernel_against_oracle_twice(B):
+    """The Qwen3-8B widths (d = 4096, Hs = 1024) take the TMEM-resident fused kernel, the one behind
+    the headline shape; through the fixed scratch array its tokens, logits and states must match
+    the fp64 oracle (replayed on the GPU's tokens) on two calls in a row, and the second call must
+    repeat the first bit for bit despite the leftovers the first left in the array."""
+    from tests import gpu_common as G
+    wl = dict(B=B, L=16, d=4096, Hs=1024, r=256, V=6000, dtype=synth.BF16, weight_seed=450 + B,
+              input_seed=451 + B, s0_std=0.2, peak=2.0, name="noalloc-tmem")
+    data = synth.make_workload(wl)
+    w, lb, h, S0 = G.device_inputs(data)
+    assert "k_greedy_tmem" in domino.greedy_plan(domino.make_shape(w, B, 16))
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    first = None
+    for call in range(2):
+        tok, lg, st = domino.draft_greedy_noalloc(w, lb, h, S0, logits_out=True, states_out=True, status=status)
+        torch.cuda.synchronize()
+        assert int(status.item()) == 0, f"call {call}: {domino.status_string(int(status.item()))}"
+        t = tok.cpu().numpy()
+        ref = G.oracle.head(data["shape"], data["weights"], data["base_logits"], data["hidden"], data["S0"],
+                            tokens=np.ascontiguousarray(t))
+        G.check_logits_states(lg.cpu().numpy(), st.cpu().numpy(), ref, f"noalloc call {call}")
+        G.check_tokens_against_replay(t, ref, f"noalloc call {call}")
+        if first is None:
+            first = (tok.clone(), lg.clone(), st.clone())
+        else:
+            for x, y in zip(first, (tok, lg, st)):
+                assert torch.equal(x, y), f"call {call} differs from call 0"
+
+
 def test_noalloc_without_status_pointer_or_optional_outputs():
     w, lb, h, S0 = _case(2, 16, 420)
     t_ref, l_ref, _ = domino.draft_greedy(w, lb, h, S0, logits_out=True)
@@ -86,7 +116,7 @@ def test_noalloc_without_status_pointer_or_optional_outputs():
 
 
 def test_noalloc_long_block_that_still_fits():
-    # B = 2 rows of 64 positions: about 0.5 MiB of keys and accumulators, within the array
+    # B = 2 rows of 64 positions: about 180 KB of keys, projections and accumulators, within the array
     w, lb, h, S0 = _case(2, 64, 440)
     t_ref, l_ref, s_ref = domino.draft_greedy(w, lb, h, S0, logits_out=True, states_out=True)
     t, l, s = domino.draft_greedy_noalloc(w, lb, h, S0, logits_out=True, states_out=True)
@@ -101,7 +131,7 @@ def test_noalloc_rejects_shapes_beyond_its_scratch_and_unsupported_shapes():
     L = domino.lib()
     ws = w.c_struct()
     p = ctypes.c_void_p(lb.data_ptr())  # never dereferenced: the checks fail before any launch
-    # B = 4 rows of 64 positions need more than the 1 MiB array
+    # B = 4 rows of 64 positions need more than the 256 KiB array
     big = domino.Shape(4, 64, 512, 256, 256, 12000, 1)
     assert L.domino_draft_greedy_noalloc(ctypes.byref(big), ctypes.byref(ws), p, p, p, p, None, None,
                                          None, None) == domino.ERR_SCRATCH_LIMIT

@@ -174,12 +174,12 @@ class ClockSampler:
 class Point:
     """Device-resident inputs of one batch point plus the timed step."""
 
-    def __init__(self, wl: dict, device, proj: bool = False):
+    def __init__(self, wl: dict, device, proj: bool = False, with_target: bool = True):
         import torch
         from draft_block_causal_b200 import domino
         self.torch, self.domino = torch, domino
         self.wl = wl
-        data = synth.make_workload(wl, with_target=True)
+        data = synth.make_workload(wl, with_target=with_target)
         self.data = data
         sh = self.sh = data["shape"]
         dt = sh["dtype"]
@@ -190,7 +190,7 @@ class Point:
         self.lb = domino.to_device(data["base_logits"], dt, device)
         self.h = domino.to_device(data["hidden"], dt, device)
         self.S0 = torch.from_numpy(data["S0"]).to(device)
-        self.T = torch.from_numpy(data["target_logits"]).to(device)
+        self.T = torch.from_numpy(data["target_logits"]).to(device) if with_target else None
         B, L = sh["B"], sh["L"]
         self.ws = domino.alloc_workspace(domino.workspace_bytes(self.w, B, L), device)
         self.tok = torch.empty((B, L), dtype=torch.int32, device=device)
@@ -711,7 +711,7 @@ def profile_driver_tf(n: int, batch: int = 1):
     torch.cuda.set_device(0)
     device = torch.device("cuda", 0)
     wl = synth.workload(HEADLINE) if batch == 1 else synth.workload("qwen3-8b-head-sweep", B=batch)
-    pt = Point(wl, device)
+    pt = Point(wl, device, with_target=False)
     stream = torch.cuda.current_stream()
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
     tokens = torch.from_numpy(synth.teacher_tokens(pt.sh, 7)).to(device)
@@ -719,6 +719,28 @@ def profile_driver_tf(n: int, batch: int = 1):
     for _ in range(n):
         flush.zero_()
         pt.tf(stream, tokens, logits)
+    torch.cuda.synchronize()
+    assert int(pt.status.item()) == 0
+
+
+def profile_driver_accept(n: int, batch: int = 1):
+    """A short, fixed sequence for an external profiler: n greedy accept-length calls and n sampled
+    verifications (greedy drafts, T = 1, fixed uniforms) of one greedy draft's tokens."""
+    import torch
+    torch.cuda.set_device(0)
+    device = torch.device("cuda", 0)
+    wl = synth.workload(HEADLINE) if batch == 1 else synth.workload("qwen3-8b-head-sweep", B=batch)
+    pt = Point(wl, device)
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
+    pt.greedy(stream)
+    uni = torch.from_numpy(np.random.default_rng(0).random((pt.sh["B"], pt.sh["L"] + 1)).astype(np.float32)).to(device)
+    for _ in range(n):
+        flush.zero_()
+        pt.accept(stream)
+    for _ in range(n):
+        flush.zero_()
+        pt.domino.accept_sample(pt.tok, pt.T, 1.0, uni, status=pt.status)
     torch.cuda.synchronize()
     assert int(pt.status.item()) == 0
 
@@ -731,7 +753,7 @@ def profile_driver(n: int, batch: int = 1, trace: bool = False, proj: bool = Fal
     torch.cuda.set_device(0)
     device = torch.device("cuda", 0)
     wl = synth.workload(HEADLINE) if batch == 1 else synth.workload("qwen3-8b-head-sweep", B=batch)
-    pt = Point(wl, device, proj=proj)
+    pt = Point(wl, device, proj=proj, with_target=False)
     stream = torch.cuda.current_stream()
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
     L = pt.sh["L"]
@@ -817,7 +839,12 @@ def main():
     ap.add_argument("--trace", action="store_true", help="profiling driver: print the fused kernel's phase times")
     ap.add_argument("--proj", action="store_true", help="profiling driver: use the embedding projection table")
     ap.add_argument("--profile-tf", action="store_true", help="profiling driver: teacher-forced calls instead")
+    ap.add_argument("--profile-accept", action="store_true",
+                    help="profiling driver: accept-length and sampled-verification calls instead")
     args = ap.parse_args()
+    if args.profile and args.profile_accept:
+        profile_driver_accept(args.profile, batch=args.profile_batch)
+        return
     if args.profile and args.profile_tf:
         profile_driver_tf(args.profile, batch=args.profile_batch)
         return

@@ -13,9 +13,6 @@
 //     columns [R*d/256, (R+1)*d/256) and the W_hh rows after them (packed bf16 pairs).
 //  2. The W2 stream is register double-buffered (the next chunk's loads are issued before the
 //     current chunk is reduced) and its first chunk is issued between barrier arrival and wait.
-//     The slack of the shared memory reserved to keep one CTA per SM (about 100 KB at B = 1) holds
-//     m of every 8 of its W2 chunks for the whole call (w2_slot), so each position streams only
-//     the rest of its slice from L2.
 //  3. The W1 state-block partials are spread over kRep replicas of the accumulator, cutting the
 //     number of same-address atomics per replica from G to G/kRep.  Every partial sum that
 //     several CTAs or warps add into (these accumulators, and the GRU gate sums in shared
@@ -63,8 +60,6 @@ struct TArgs {
   const float* Xp;  // [V][3Hs] input projection of the embedding table, or null
   const int32_t* tf_tokens;  // [B][L] given tokens (teacher-forced mode), or null (greedy)
   const float* Gx;           // teacher-forced mode: [B][L-1][3Hs] W_ih . embed[y_i] precomputed, or null
-  int w2m;                   // W2 chunks kept in shared memory per aligned block of 8 (0..8)
-  unsigned w2r_off;          // byte offset of those chunks in dynamic shared memory (16-aligned)
 };
 
 __device__ __forceinline__ unsigned ld_acquire_u32(const unsigned* p) {
@@ -222,26 +217,13 @@ __device__ void tmem_rows_dot(uint32_t tbase, int col0, int cpr, int nrows, cons
     tmem_rows_dot_ch<BMAX, In, 2>(tbase, col0, cpr, nrows, in_t, B, acc_s, acc_stride, warp, lane);
 }
 
-// Shared-memory slot of chunk ch of the CTA's W2 slice, or -1 when the chunk streams from L2: m of
-// every aligned block of 8 chunks are resident, chosen by (ch ^ (ch >> 4)) & 7 < m -- a permutation
-// of each block -- so that every warp (chunks ch = warp + 16k) and every iteration k mixes resident
-// and streamed chunks.
-__device__ __forceinline__ int w2_slot(int ch, int m) {
-  const int rk = (ch ^ (ch >> 4)) & 7;
-  return rk < m ? (ch >> 3) * m + rk : -1;
-}
-
 template <int BMAX, int ROWS>
 __device__ __forceinline__ void w2_load(const TArgs& p, int v0, int v1, int ch, int lane, size_t lrow, int L,
-                                        uint4 (&q)[ROWS], float (&lb)[BMAX], const uint8_t* w2r) {
+                                        uint4 (&q)[ROWS], float (&lb)[BMAX]) {
   const int vb = v0 + ch * ROWS;
-  const int slot = w2_slot(ch, p.w2m);
-  const uint8_t* rs = w2r + (size_t)slot * ROWS * (kR2 * 2) + lane * 16;
 #pragma unroll
   for (int k = 0; k < ROWS; ++k)
-    q[k] = (vb + k < v1) ? (slot >= 0 ? *reinterpret_cast<const uint4*>(rs + k * (kR2 * 2))
-                                      : ldg16_w2(p.W2 + (size_t)(vb + k) * kR2 + lane * 8))
-                         : make_uint4(0u, 0u, 0u, 0u);
+    q[k] = (vb + k < v1) ? ldg16_w2(p.W2 + (size_t)(vb + k) * kR2 + lane * 8) : make_uint4(0u, 0u, 0u, 0u);
   const int v = vb + (lane / (32 / ROWS));
 #pragma unroll
   for (int b = 0; b < BMAX; ++b)
@@ -310,7 +292,6 @@ __global__ void __launch_bounds__(kThreads2, 1) k_greedy_tmem(TArgs p) {
   int* tok_s = reinterpret_cast<int*>(best_s + kWarps2 * BMAX);        // [BMAX]
   int* flag_s = tok_s + BMAX;
   uint32_t* tbase_s = reinterpret_cast<uint32_t*>(flag_s + 1);
-  const uint8_t* w2r = smem + p.w2r_off;  // resident W2 chunks (greedy mode)
   unsigned epoch = 0;
 
   // ---- TMEM: one allocation for the whole call ----
@@ -364,19 +345,6 @@ __global__ void __launch_bounds__(kThreads2, 1) k_greedy_tmem(TArgs p) {
     tmem_wait_st();
   }
   const bool tf = p.tf_tokens != nullptr;
-  // this CTA's resident W2 chunks, once for the call (read after the barrier below)
-  if (!tf && p.w2m > 0) {
-    const int nchunks = (v1 - v0 + ROWS - 1) / ROWS;
-    uint8_t* w2w = smem + p.w2r_off;
-    for (int t = tid; t < nchunks * ROWS * 32; t += kThreads2) {
-      const int ch = t / (ROWS * 32), k = (t / 32) % ROWS, ln = t % 32;
-      const int slot = w2_slot(ch, p.w2m);
-      const int v = v0 + ch * ROWS + k;
-      if (slot >= 0 && v < v1)
-        *reinterpret_cast<uint4*>(w2w + ((size_t)slot * ROWS + k) * (kR2 * 2) + ln * 16) =
-            ldg16(p.W2 + (size_t)v * kR2 + ln * 8);
-    }
-  }
   for (int k = tid; k < maxu * kR2 && !tf; k += kThreads2) {
     const int jj = k / kR2, kk = k % kR2;
     w1s_s[k] = (jj < nu) ? __bfloat162float(p.W1[(size_t)kk * ldw1 + d + j0 + jj]) : 0.f;
@@ -450,7 +418,7 @@ __global__ void __launch_bounds__(kThreads2, 1) k_greedy_tmem(TArgs p) {
 
   stamp(p.trace, p.ntrace, 1);
   grid_arrive(p, epoch);
-  if (!tf && warp < nch) w2_load<BMAX, ROWS>(p, v0, v1, warp, lane, 0, L, qa, lba, w2r);
+  if (!tf && warp < nch) w2_load<BMAX, ROWS>(p, v0, v1, warp, lane, 0, L, qa, lba);
   if (!grid_wait(p, epoch, flag_s)) { leave(); return; }
   stamp(p.trace, p.ntrace, 2);
 
@@ -510,10 +478,10 @@ __global__ void __launch_bounds__(kThreads2, 1) k_greedy_tmem(TArgs p) {
 #pragma unroll
       for (int b = 0; b < BMAX; ++b) best[b] = 0ull;
       for (int ch = warp; ch < nch; ch += 2 * kWarps2) {
-        if (ch + kWarps2 < nch) w2_load<BMAX, ROWS>(p, v0, v1, ch + kWarps2, lane, lrow, L, qb, lbb, w2r);
+        if (ch + kWarps2 < nch) w2_load<BMAX, ROWS>(p, v0, v1, ch + kWarps2, lane, lrow, L, qb, lbb);
         w2_chunk<BMAX, ROWS>(p, v0, v1, ch, lane, lrow, L, qa, lba, uv, best);
         if (ch + kWarps2 >= nch) break;
-        if (ch + 2 * kWarps2 < nch) w2_load<BMAX, ROWS>(p, v0, v1, ch + 2 * kWarps2, lane, lrow, L, qa, lba, w2r);
+        if (ch + 2 * kWarps2 < nch) w2_load<BMAX, ROWS>(p, v0, v1, ch + 2 * kWarps2, lane, lrow, L, qa, lba);
         w2_chunk<BMAX, ROWS>(p, v0, v1, ch + kWarps2, lane, lrow, L, qb, lbb, uv, best);
       }
 #pragma unroll
@@ -631,7 +599,7 @@ __global__ void __launch_bounds__(kThreads2, 1) k_greedy_tmem(TArgs p) {
     }
     stamp(p.trace, p.ntrace, tb + 6);
     grid_arrive(p, epoch);
-    if (!tf && warp < nch) w2_load<BMAX, ROWS>(p, v0, v1, warp, lane, lrow + V, L, qa, lba, w2r);
+    if (!tf && warp < nch) w2_load<BMAX, ROWS>(p, v0, v1, warp, lane, lrow + V, L, qa, lba);
     if (!grid_wait(p, epoch, flag_s)) { leave(); return; }
     stamp(p.trace, p.ntrace, tb + 7);
   }
@@ -644,7 +612,7 @@ __global__ void __launch_bounds__(kThreads2, 1) k_greedy_tmem(TArgs p) {
   leave();
 }
 
-// Shared memory of the kernel's working arrays (before the resident W2 chunks).
+// Shared memory of the kernel's working arrays.
 size_t smem_work_bytes(int bmax, int d, int Hs, int maxu) {
   size_t bytes = ((size_t)bmax * kR2 + (size_t)bmax * Hs) * 4 + (size_t)bmax * (d / 2) * 4;
   bytes += ((size_t)maxu * kR2 + (((size_t)bmax * maxu + 3) & ~(size_t)3)) * 4 + 6 * (size_t)bmax * maxu * 8;
@@ -702,18 +670,7 @@ cudaError_t launch_tmem_common(const Shape& s, const domino_weights_t& w, const 
   cudaError_t e = cudaMemsetAsync(ws.sync, 0, zero_bytes, st);
   if (e != cudaSuccess) return e;
   const int bmax = s.B <= 1 ? 1 : (s.B <= 2 ? 2 : 4);
-  size_t smem = smem_bytes_tmem(bmax, s.d, s.Hs, a.maxu);
-  if (!tf_tokens) {
-    // greedy: the shared memory reserved to keep one CTA per SM but not used by the working arrays
-    // holds W2 chunks for the whole call.  The reservation is not grown for them: shared memory and
-    // L1 share one array per SM, and the W2 stream needs the L1 capacity for its loads in flight.
-    const int rows = bmax == 4 ? 4 : 8;
-    const size_t work = smem_work_bytes(bmax, s.d, s.Hs, a.maxu), chunk = (size_t)rows * s.r * 2;
-    const int nblk = ((s.V + G - 1) / G + rows * 8 - 1) / (rows * 8);  // aligned blocks of 8 chunks
-    const size_t avail = smem > work ? smem - work : 0;
-    a.w2m = (int)std::min<size_t>(8, avail / (chunk * (size_t)nblk));
-    a.w2r_off = (unsigned)work;
-  }
+  const size_t smem = smem_bytes_tmem(bmax, s.d, s.Hs, a.maxu);
   if (bmax == 1) e = launch_tmem_t<1, 8>(a, G, smem, st);
   else if (bmax == 2) e = launch_tmem_t<2, 8>(a, G, smem, st);
   else e = launch_tmem_t<4, 4>(a, G, smem, st);

@@ -321,6 +321,31 @@ def full_accept_targets(pt: Point, stream):
     return logits
 
 
+def w2_kernel_phases(pt: Point, flush, stream) -> dict:
+    """Phase stamps of the last position's W2 argmax launch (k_w2_argmax), medians over CTAs, in us
+    from the moment the wait on the previous grid returned in the earliest CTA."""
+    torch, domino = pt.torch, pt.domino
+    buf = torch.zeros(148 * 16, dtype=torch.int64, device=pt.lb.device)
+    flush.zero_()
+    torch.cuda.synchronize()
+    domino.set_trace(buf)
+    try:
+        pt.greedy(stream)
+        torch.cuda.synchronize()
+    finally:
+        domino.set_trace(None)
+    t = buf.view(-1, 16).cpu().numpy().astype(np.int64)
+    t = t[(t[:, 1] != 0) & (t[:, 15] != 0)]
+    ref = t[:, 15].min()
+    names = {0: "start", 2: "first_w2_stage_issued", 3: "first_lbase_issued", 15: "prev_grid_done_in_cta",
+             4: "u_band_in_tmem", 5: "first_mma", 6: "first_acc_in_epilogue", 8: "last_mma_committed",
+             9: "last_w2_issued", 10: "last_lbase_issued", 7: "epilogue_done", 1: "end"}
+    out = {n: round(float(np.median(t[:, k] - ref)) / 1e3, 2) for k, n in names.items()}
+    out["end_max"] = round(float((t[:, 1] - ref).max()) / 1e3, 2)
+    out["tiles_median"] = int(np.median(t[:, 11]))
+    return out
+
+
 def time_tf(pt: Point, steps: int, warmup: int, flush, stream, bf16_logits: bool = False) -> list:
     """Teacher-forced calls (uniform given tokens, logits out), each after an L2 flush; per-call
     device times in ms."""
@@ -757,6 +782,13 @@ def profile_driver(n: int, batch: int = 1, trace: bool = False, proj: bool = Fal
     stream = torch.cuda.current_stream()
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
     L = pt.sh["L"]
+    if trace and batch > 4:  # the batched path: the W2 argmax launch's phases
+        for _ in range(n):
+            flush.zero_()
+            pt.greedy(stream)
+        torch.cuda.synchronize()
+        print(json.dumps({"B": batch, "w2_argmax_phases_us": w2_kernel_phases(pt, flush, stream)}), flush=True)
+        return
     buf = torch.zeros(4 + 10 * L, dtype=torch.int64, device=device)
     for k in range(n):
         flush.zero_()

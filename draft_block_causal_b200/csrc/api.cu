@@ -322,7 +322,8 @@ int domino_draft_greedy(const domino_shape_t* shape, const domino_weights_t* w, 
         float* lo = logits_out ? logits_out + row0 * s.V : nullptr;
         if (w2_argmax_supported(Mb, s.V, s.r, Ub, w->W2, Lbp, (long long)s.L * s.V))
           e = w2_argmax(Ub, (const bf*)w->W2, Mb, s.V, s.r, Lbp, (long long)s.L * s.V, ws.keys + (size_t)i * s.B + b0,
-                        lo, (long long)s.L * s.V, i == s.L - 1 && b0 + 128 >= s.B, st, spin_limit(), cs);
+                        lo, (long long)s.L * s.V, i == s.L - 1 && b0 + 128 >= s.B, ws.claim, epoch, st,
+                        spin_limit(), cs);
         else
           e = gemm_tc_argmax(Ub, (const bf*)w->W2, Mb, s.V, s.r, Lbp, (long long)s.L * s.V,
                              ws.keys + (size_t)i * s.B + b0, lo, (long long)s.L * s.V, st, spin_limit(), cs, ws.claim,
@@ -401,9 +402,13 @@ int teacher_forced_impl(const domino_shape_t* shape, const domino_weights_t* w, 
   using bf = __nv_bfloat16;
   const bool tc = s.dtype == DOMINO_DTYPE_BF16 && s.d % 64 == 0 && s.r % 64 == 0 && s.Hs % 64 == 0 &&
                   gemm_tc_supported((int)BL, s.r, s.d, hidden, w->W1);
-  cudaError_t e = tc ? gemm_tc_store_f32_t((const bf*)w->W1, (const bf*)hidden, s.r, (int)BL, s.d, 0, ws.P, s.r, st,
-                                           spin_limit(), cs, 0, s.d + s.Hs)
-                     : launch_hproj(s, w->W1, hidden, (int)BL, ws.P, cs);
+  // every check has passed: from here on work is enqueued.  The logits GEMM claims its work slots by
+  // SM (epoch 1 against words zeroed here).
+  cudaError_t e = cudaMemsetAsync(ws.claim, 0, kClaimWords * sizeof(uint32_t), cs);
+  if (e == cudaSuccess)
+    e = tc ? gemm_tc_store_f32_t((const bf*)w->W1, (const bf*)hidden, s.r, (int)BL, s.d, 0, ws.P, s.r, st,
+                                 spin_limit(), cs, 0, s.d + s.Hs)
+           : launch_hproj(s, w->W1, hidden, (int)BL, ws.P, cs);
   // Small batches whose GRU rows fit in TMEM: the whole recurrence in one fused kernel (one grid
   // barrier per update), then the activations and logits of all positions as below.
   // The input half of every update is known up front: one gather + W_ih product over all B*(L-1)
@@ -459,7 +464,7 @@ int teacher_forced_impl(const domino_shape_t* shape, const domino_weights_t* w, 
   if (e == cudaSuccess) {
     if (tc_w2)
       e = gemm_tc_logits((const __nv_bfloat16*)w->W2, ws.u16, s.V, (int)BL, s.r, (const __nv_bfloat16*)base_logits,
-                         logits_out, logits_dtype == DOMINO_DTYPE_BF16, st, spin_limit(), cs);
+                         logits_out, logits_dtype == DOMINO_DTYPE_BF16, st, spin_limit(), cs, ws.claim, 1u);
     else
       e = launch_w2(s, w->W2, ws.u, (int)BL, base_logits, 1, 0, nullptr, static_cast<float*>(logits_out), cs);
   }

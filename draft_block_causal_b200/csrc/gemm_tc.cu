@@ -37,6 +37,7 @@
 #include "common.cuh"
 #include "gemm_tc.h"
 #include "launch.cuh"
+#include "sm_affinity.cuh"
 #include "umma.cuh"
 
 #include <atomic>
@@ -151,21 +152,26 @@ struct EpiLogitsT {  // logits[n][m] = D + Lb[n][m]   (m = vocabulary row, n = (
 // 32 rows x 16 columns go to shared memory (16-byte chunks XOR-swizzled so that neither side has
 // bank conflicts) and come back so that each store instruction writes whole 64-byte (fp32) or
 // 32-byte (bf16) row segments -- 8 or 16 rows per instruction instead of 32 scattered 16-byte
-// pieces.  Every lane of the warp calls apply with the same n0.
+// pieces.  Every lane of the warp calls apply with the same n0.  Each thread also loads the L_base
+// of its next 16-column group (the next call's, within the tile) before storing this one, so that
+// the load's latency overlaps the stores.
 template <typename OutT>
 struct EpiLogitsRowT {
   static constexpr bool kSide = false;
   static constexpr bool kARes = false;
   static constexpr int kGroups = 2;  // the epilogue is the longest phase of a tile: two warps per lane quadrant
   static constexpr bool kWarpCoop = true;
-  using State = NoState;
+  struct State {
+    uint4 la, lb;  // L_base of (pm, pn .. pn + 15), loaded ahead
+    int pm, pn;
+  };
   const bf16* Lb;
   OutT* logits;
   int M;
   long long ld;
-  __device__ __forceinline__ void init(State&) const {}
+  __device__ __forceinline__ void init(State& st) const { st.pm = -1; st.pn = -1; }
   __device__ __forceinline__ void finish(State&, int) const {}
-  __device__ __forceinline__ void apply(State&, int m, int n0, const float (&v)[16], int N, const uint8_t*, int,
+  __device__ __forceinline__ void apply(State& st, int m, int n0, const float (&v)[16], int N, const uint8_t*, int,
                                         int) const {
     const int lane = threadIdx.x & 31;
     if (n0 + 16 <= N) {  // warp-uniform
@@ -175,9 +181,23 @@ struct EpiLogitsRowT {
       float z[16];
       if (m < M) {
         const bf16* lr = Lb + (size_t)m * ld + n0;
+        uint4 qa, qb;
+        if (st.pm == m && st.pn == n0) {
+          qa = st.la;
+          qb = st.lb;
+        } else {
+          qa = __ldg(reinterpret_cast<const uint4*>(lr));
+          qb = __ldg(reinterpret_cast<const uint4*>(lr) + 1);
+        }
+        if (n0 + 32 <= N) {  // the next group of this row
+          st.la = __ldg(reinterpret_cast<const uint4*>(lr + 16));
+          st.lb = __ldg(reinterpret_cast<const uint4*>(lr + 16) + 1);
+          st.pm = m;
+          st.pn = n0 + 16;
+        }
         float a[8], b[8];
-        widen(__ldg(reinterpret_cast<const uint4*>(lr)), a);
-        widen(__ldg(reinterpret_cast<const uint4*>(lr) + 1), b);
+        widen(qa, a);
+        widen(qb, b);
 #pragma unroll
         for (int j = 0; j < 8; ++j) { z[j] = v[j] + a[j]; z[8 + j] = v[8 + j] + b[j]; }
       } else {
@@ -400,53 +420,6 @@ __device__ __forceinline__ uint32_t cluster_map(uint32_t addr, int rank) {
 __device__ __forceinline__ void st_cluster_f4(uint32_t addr, float a, float b, float c, float d) {
   asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
                : "memory");
-}
-
-// ---- SM affinity of work slots ----
-// A persistent launch with one CTA per SM walks the tiles t = slot, slot + grid, ...  Choosing the
-// slot from the SM the CTA runs on (rather than from blockIdx) gives every tile the same SM at
-// every launch, so that its operand lines stay in the L2 partition next to that SM across
-// launches.  g_sm_rank maps %smid to a dense rank (filled once per device by k_sm_probe /
-// k_sm_rank); each launch claims slots with atomicExch against a per-launch epoch, so that every
-// slot is taken exactly once even when the scheduler places two CTAs on one SM.
-constexpr int kMaxSmid = 1024;
-__device__ int g_sm_of_cta[kMaxSmid];
-__device__ int g_sm_rank[kMaxSmid];
-
-__device__ __forceinline__ unsigned sm_id() {
-  unsigned s;
-  asm volatile("mov.u32 %0, %%smid;" : "=r"(s));
-  return s;
-}
-// Launched with more than half an SM's shared memory (unused): one CTA per SM.
-__global__ void k_sm_probe(int n) {
-  if (threadIdx.x == 0 && blockIdx.x < (unsigned)n) g_sm_of_cta[blockIdx.x] = (int)sm_id();
-}
-__global__ void k_sm_rank(int n) {  // one thread: dense rank of each recorded smid
-  if (threadIdx.x != 0 || blockIdx.x != 0) return;
-  for (int s = 0; s < kMaxSmid; ++s) g_sm_rank[s] = -1;
-  for (int i = 0; i < n; ++i) {
-    const int s = g_sm_of_cta[i];
-    if (s >= 0 && s < kMaxSmid) g_sm_rank[s] = 0;  // present
-  }
-  int r = 0;
-  for (int s = 0; s < kMaxSmid; ++s)
-    if (g_sm_rank[s] == 0) g_sm_rank[s] = ++r;
-  for (int s = 0; s < kMaxSmid; ++s)
-    if (g_sm_rank[s] > 0) --g_sm_rank[s];  // ranks 0 .. r-1
-}
-// Work slot of this CTA (thread 0 only).  claim == null: blockIdx.x.
-__device__ int claim_slot(uint32_t* claim, uint32_t epoch) {
-  if (!claim) return (int)blockIdx.x;
-  const int G = (int)gridDim.x;
-  const unsigned s = sm_id();
-  const int pref = s < (unsigned)kMaxSmid ? g_sm_rank[s] : -1;
-  if (pref >= 0 && pref < G && atomicExch(claim + pref, epoch) != epoch) return pref;
-  for (int k = 0; k < G; ++k) {  // taken (or no rank): the next free slot
-    const int c = ((int)blockIdx.x + k) % G;
-    if (atomicExch(claim + c, epoch) != epoch) return c;
-  }
-  return (int)blockIdx.x;  // unreachable: G CTAs, G slots
 }
 
 // Shared memory (from a 1024-aligned base): [resident A][stage ring][1024 B: mbarriers, TMEM slot]
@@ -874,24 +847,6 @@ bool tmap_bf16(CUtensorMap* tm, const void* base, uint64_t rows, uint64_t cols, 
 }
 
 
-// Fills g_sm_rank once per device (two small launches on `st`, no host synchronisation).
-cudaError_t ensure_sm_rank(cudaStream_t st) {
-  static std::atomic<uint64_t> done{0};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  const uint64_t bit = dev < 64 ? (1ull << dev) : 0;
-  if (bit && (done.load(std::memory_order_acquire) & bit)) return cudaSuccess;
-  const int n = std::min(sm_count(), kMaxSmid);
-  const int hold = 120 * 1024;  // more than half an SM's shared memory: one CTA per SM
-  cudaError_t e = cudaFuncSetAttribute(k_sm_probe, cudaFuncAttributeMaxDynamicSharedMemorySize, hold);
-  if (e != cudaSuccess) return e;
-  k_sm_probe<<<n, 32, hold, st>>>(n);
-  k_sm_rank<<<1, 32, 0, st>>>(n);
-  e = cudaGetLastError();
-  if (e == cudaSuccess && bit) done.fetch_or(bit, std::memory_order_acq_rel);
-  return e;
-}
-
 // The kernel's dynamic shared memory opt-in, set once per device.
 template <int BN, class Epi, bool SPLIT>
 cudaError_t set_smem_once(size_t smem) {
@@ -1171,21 +1126,27 @@ cudaError_t gemm_tc_store_f32_t(const bf16* A, const bf16* Bm, int M, int N, int
 
 template <typename OutT>
 cudaError_t logits_t(const bf16* W2, const bf16* U, int V, int N, int r, const bf16* Lb, OutT* logits, int32_t* status,
-                     uint64_t limit, cudaStream_t st) {
+                     uint64_t limit, cudaStream_t st, uint32_t* claim, uint32_t epoch) {
   if (N >= 64) {  // enough rows for the row-major orientation: vector loads and stores in the epilogue
-    // the row bands of one vocabulary tile run side by side, so each W2 tile is read from HBM once
+    // The row bands of one vocabulary tile run side by side on CTAs of consecutive work slots --
+    // neighbouring SMs when the slots are taken by SM (claim) -- so each W2 tile is read from HBM once.
+    if (claim) {
+      cudaError_t e = ensure_sm_rank(st);
+      if (e != cudaSuccess) return e;
+    }
     EpiLogitsRowT<OutT> e{Lb, logits, N, (long long)V};
     return launch_gemm<256>(U, W2, N, V, r, e, status, limit, st, 0, 0, 0, nullptr, 0, nullptr, 0, 0, 1, 0, 2,
-                            nullptr, 0, 1);
+                            claim, epoch, 1);
   }
   EpiLogitsT<OutT> e{Lb, logits, V};
   return launch_gemm_bn(W2, U, V, N, r, e, status, limit, st);
 }
 
 cudaError_t gemm_tc_logits(const bf16* W2, const bf16* U, int V, int N, int r, const bf16* Lb, void* logits,
-                           int out_bf16, int32_t* status, uint64_t limit, cudaStream_t st) {
-  return out_bf16 ? logits_t(W2, U, V, N, r, Lb, static_cast<bf16*>(logits), status, limit, st)
-                  : logits_t(W2, U, V, N, r, Lb, static_cast<float*>(logits), status, limit, st);
+                           int out_bf16, int32_t* status, uint64_t limit, cudaStream_t st, uint32_t* claim,
+                           uint32_t epoch) {
+  return out_bf16 ? logits_t(W2, U, V, N, r, Lb, static_cast<bf16*>(logits), status, limit, st, claim, epoch)
+                  : logits_t(W2, U, V, N, r, Lb, static_cast<float*>(logits), status, limit, st, claim, epoch);
 }
 
 }  // namespace domino

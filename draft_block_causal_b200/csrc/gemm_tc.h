@@ -45,11 +45,12 @@ cudaError_t gemm_tc_argmax(const __nv_bfloat16* U, const __nv_bfloat16* W2, int 
 // resident in TMEM, W2 kept in L2 across positions, balanced vocabulary ranges): M <= 128 rows,
 // r a multiple of 64 up to 256, U, W2 and Lb 16-byte aligned, Lb's row stride ldl (elements) a
 // multiple of 8.  w2_argmax_supported tells whether a call qualifies.  last: this is the call's last
-// read of W2 (its lines are then marked evict-first rather than evict-last).
+// read of W2 (its lines are then marked evict-first rather than evict-last).  claim / epoch: as for
+// gemm_tc_argmax (vocabulary ranges taken by the SM a CTA runs on).
 bool w2_argmax_supported(int M, int V, int r, const void* U, const void* W2, const void* Lb, long long ldl);
 cudaError_t w2_argmax(const __nv_bfloat16* U, const __nv_bfloat16* W2, int M, int V, int r, const __nv_bfloat16* Lb,
-                      long long ldl, uint64_t* keys, float* out, long long ldo, bool last, int32_t* status,
-                      uint64_t limit, cudaStream_t st);
+                      long long ldl, uint64_t* keys, float* out, long long ldo, bool last, uint32_t* claim,
+                      uint32_t epoch, int32_t* status, uint64_t limit, cudaStream_t st);
 
 // u16[n][k] = bf16(SiLU(P[n * ldp + k] + sum_j W1s[k][j] S[n][j])) for k < r, n < N, where the
 // fp32 state arrives as its two-term bf16 split S_hl [N x 2Hs] and W1s [r x Hs] has row stride ldw
@@ -84,9 +85,10 @@ cudaError_t gemm_tc_debug(const __nv_bfloat16* A, const __nv_bfloat16* Bm, int M
 void gemm_tc_skinny_plan(int M, int N, int K, int* bn, int* ks);
 
 // logits[n][v] = Lb[n][v] + sum_k W2[v][k] U[n][k]   (W2 [V x r], U [N x r], Lb [N x V] bf16); logits
-// fp32, or bf16 (round to nearest even) when out_bf16
+// fp32, or bf16 (round to nearest even) when out_bf16.  claim / epoch (optional, as for
+// gemm_tc_argmax): work slots taken by the SM a CTA runs on.
 cudaError_t gemm_tc_logits(const __nv_bfloat16* W2, const __nv_bfloat16* U, int V, int N, int r,
                            const __nv_bfloat16* Lb, void* logits, int out_bf16, int32_t* status, uint64_t limit,
-                           cudaStream_t st);
+                           cudaStream_t st, uint32_t* claim = nullptr, uint32_t epoch = 0);
 
 }  // namespace domino

@@ -85,7 +85,9 @@ __device__ __forceinline__ void stamp(unsigned long long* trace, int ntrace, int
   if (trace && k < ntrace && blockIdx.x == 0 && threadIdx.x == 0) trace[k] = clock64();
 }
 
-// Split-phase grid barrier on a monotonic counter: arrive, do independent work, then wait.
+// Split-phase grid barrier on a monotonic counter: arrive, do independent work, then wait.  (A
+// separate release flag written by the last arrival was measured slower: its extra round trip is
+// serial, while polling the counter itself costs nothing the waits can feel.)
 __device__ __forceinline__ void grid_arrive(const TArgs& p, unsigned& epoch) {
   __syncthreads();
   ++epoch;
@@ -288,7 +290,8 @@ __global__ void __launch_bounds__(kThreads2, 1) k_greedy_tmem(TArgs p) {
   unsigned long long* gh_s = reinterpret_cast<unsigned long long*>(w1s_s + (size_t)maxu * kR2);  // [BMAX][3*maxu]
   unsigned long long* gi_s = gh_s + BMAX * 3 * maxu;                    // [BMAX][3*maxu]
   float* sn_s = reinterpret_cast<float*>(gi_s + BMAX * 3 * maxu);       // [BMAX][maxu]
-  uint64_t* best_s = reinterpret_cast<uint64_t*>(sn_s + ((BMAX * maxu + 3) & ~3));  // [warps][BMAX]
+  float* bias_s = sn_s + ((BMAX * maxu + 3) & ~3);                      // [2][3][maxu] b_ih, b_hh (own units)
+  uint64_t* best_s = reinterpret_cast<uint64_t*>(bias_s + ((6 * maxu + 3) & ~3));  // [warps][BMAX]
   int* tok_s = reinterpret_cast<int*>(best_s + kWarps2 * BMAX);        // [BMAX]
   int* flag_s = tok_s + BMAX;
   uint32_t* tbase_s = reinterpret_cast<uint32_t*>(flag_s + 1);
@@ -350,6 +353,10 @@ __global__ void __launch_bounds__(kThreads2, 1) k_greedy_tmem(TArgs p) {
     w1s_s[k] = (jj < nu) ? __bfloat162float(p.W1[(size_t)kk * ldw1 + d + j0 + jj]) : 0.f;
   }
   for (int k = tid; k < BMAX * 6 * maxu; k += kThreads2) gh_s[k] = 0ull;  // gh_s and gi_s
+  for (int k = tid; k < 6 * maxu; k += kThreads2) {  // the own units' biases, read at every update
+    const int h = k / (3 * maxu), g = (k / maxu) % 3, jj = k % maxu;
+    bias_s[k] = jj < nu ? __bfloat162float((h ? p.b_hh : p.b_ih)[(size_t)g * Hs + j0 + jj]) : 0.f;
+  }
   // P[i][b][k] = W1[k, :d] . H[b, i]  for the rank rows k = c, c + G, ... (one warp per value)
   if (!tf) {
     const int nk = (kR2 - c + G - 1) / G;
@@ -538,6 +545,10 @@ __global__ void __launch_bounds__(kThreads2, 1) k_greedy_tmem(TArgs p) {
 
     // t_i; gi = W_ih . embed[t_i] for the own units: gathered from the projection table, or
     // computed from TMEM with the embedding row staged in the lane-sliced layout; GRU cell -> S_i
+    if (!tf) {  // the global argmax of each row, read once (tok_s held this CTA's own candidate)
+      if (tid < B) tok_s[tid] = min(max(key_index(__ldcg(p.keys + (size_t)i * B + tid)), 0), V - 1);
+      __syncthreads();
+    }
     if (proj) {
       for (int t = tid; t < B * 3 * nu; t += kThreads2) {
         const int b = t / (3 * nu), R = t % (3 * nu), g = R / nu, jj = R % nu;
@@ -545,17 +556,15 @@ __global__ void __launch_bounds__(kThreads2, 1) k_greedy_tmem(TArgs p) {
           gi_s[b * 3 * maxu + R] = fix_of(__ldg(p.Gx + ((size_t)b * (L - 1) + i) * 3 * Hs + (size_t)g * Hs + j0 + jj));
           continue;
         }
-        const int tok = tf ? tok_s[b] : min(max(key_index(__ldcg(p.keys + (size_t)i * B + b)), 0), V - 1);
-        gi_s[b * 3 * maxu + R] = fix_of(__ldg(p.Xp + (size_t)tok * 3 * Hs + (size_t)g * Hs + j0 + jj));
+        gi_s[b * 3 * maxu + R] = fix_of(__ldg(p.Xp + (size_t)tok_s[b] * 3 * Hs + (size_t)g * Hs + j0 + jj));
       }
       __syncthreads();
       stamp(p.trace, p.ntrace, tb + 4);
     } else {
       for (int t = tid; t < B * (d / 2); t += kThreads2) {
         const int b = t / (d / 2), w = t % (d / 2);
-        const int tok = tf ? tok_s[b] : min(max(key_index(__ldcg(p.keys + (size_t)i * B + b)), 0), V - 1);
         x_t[((size_t)b * cpri + w % cpri) * 128 + w / cpri] =
-            __ldg(reinterpret_cast<const uint32_t*>(p.embed + (size_t)tok * d) + w);
+            __ldg(reinterpret_cast<const uint32_t*>(p.embed + (size_t)tok_s[b] * d) + w);
       }
       __syncthreads();
       stamp(p.trace, p.ntrace, tb + 4);
@@ -569,8 +578,8 @@ __global__ void __launch_bounds__(kThreads2, 1) k_greedy_tmem(TArgs p) {
       float gi[3], gh[3];
 #pragma unroll
       for (int g = 0; g < 3; ++g) {
-        gi[g] = fix_value(gi_s[b * 3 * maxu + g * nu + jj]) + __bfloat162float(p.b_ih[(size_t)g * Hs + j]);
-        gh[g] = fix_value(gh_s[b * 3 * maxu + g * nu + jj]) + __bfloat162float(p.b_hh[(size_t)g * Hs + j]);
+        gi[g] = fix_value(gi_s[b * 3 * maxu + g * nu + jj]) + bias_s[g * maxu + jj];
+        gh[g] = fix_value(gh_s[b * 3 * maxu + g * nu + jj]) + bias_s[(3 + g) * maxu + jj];
         gi_s[b * 3 * maxu + g * nu + jj] = 0ull;
         gh_s[b * 3 * maxu + g * nu + jj] = 0ull;
       }
@@ -615,7 +624,8 @@ __global__ void __launch_bounds__(kThreads2, 1) k_greedy_tmem(TArgs p) {
 // Shared memory of the kernel's working arrays.
 size_t smem_work_bytes(int bmax, int d, int Hs, int maxu) {
   size_t bytes = ((size_t)bmax * kR2 + (size_t)bmax * Hs) * 4 + (size_t)bmax * (d / 2) * 4;
-  bytes += ((size_t)maxu * kR2 + (((size_t)bmax * maxu + 3) & ~(size_t)3)) * 4 + 6 * (size_t)bmax * maxu * 8;
+  bytes += ((size_t)maxu * kR2 + (((size_t)bmax * maxu + 3) & ~(size_t)3) + ((6 * (size_t)maxu + 3) & ~(size_t)3)) * 4 +
+           6 * (size_t)bmax * maxu * 8;
   bytes += (size_t)kWarps2 * bmax * 8 + (size_t)bmax * 4 + 16;
   return (bytes + 15) & ~(size_t)15;
 }

@@ -21,7 +21,8 @@
 //                   position cannot change the result (a rejection recorded for it can only follow
 //                   an earlier one, which wins the max).
 //   k_sample_finish one block per row: k = L - first[b]; the replacement at (b, k) from the residual,
-//                   recomputed from the merged statistics, with a fixed-order double-precision scan.
+//                   recomputed from the merged statistics, with coalesced tiles and a fixed-order
+//                   double-precision block scan carried across tiles.
 // Both are memory-bound on the logits they read: at most B*L*V*4 bytes of target (and as many of
 // draft) logits, plus one target (and draft) row per rejected row.
 #include "common.cuh"
@@ -150,20 +151,65 @@ __global__ void __launch_bounds__(kStatThreads) k_sample_stats(SampleArgs a) {
 }
 
 // Residual mass max(0, p(v) - q(v)) at one position from its merged statistics.
-__device__ __forceinline__ float residual_at(const SampleArgs& a, const float* trow, const float* drow, int x,
-                                             const float4& st, int v) {
-  const float p = expf((trow[v] - st.x) * a.inv_t) / st.y;
-  const float q = drow ? expf((drow[v] - st.z) * a.inv_t) / st.w : (v == x ? 1.f : 0.f);
+__device__ __forceinline__ float residual_of(const SampleArgs& a, float t, float d, bool one_hot, const float4& st) {
+  const float p = expf((t - st.x) * a.inv_t) / st.y;
+  const float q = one_hot ? 0.f : expf((d - st.z) * a.inv_t) / st.w;
   return fmaxf(p - q, 0.f);
 }
 
+// The four residuals of columns v .. v + 3 (v a multiple of 4; V is a multiple of 8).
+__device__ __forceinline__ void residual4(const SampleArgs& a, const float* trow, const float* drow, int x,
+                                          const float4& st, int v, float (&r)[4]) {
+  const float4 t = __ldcs(reinterpret_cast<const float4*>(trow + v));
+  const float4 d = drow ? __ldcs(reinterpret_cast<const float4*>(drow + v)) : make_float4(0.f, 0.f, 0.f, 0.f);
+  r[0] = residual_of(a, t.x, d.x, !drow, st);
+  r[1] = residual_of(a, t.y, d.y, !drow, st);
+  r[2] = residual_of(a, t.z, d.z, !drow, st);
+  r[3] = residual_of(a, t.w, d.w, !drow, st);
+  if (!drow) {  // the one-hot draft removes the draft token's whole mass: res(x) = max(0, p(x) - 1)
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+      if (v + e == x) r[e] = fmaxf(expf((((const float*)&t)[e] - st.x) * a.inv_t) / st.y - 1.f, 0.f);
+  }
+}
+
+// Block-wide inclusive scan of one double per thread in thread order (fixed): within each warp, then
+// over the warp totals.  Returns the inclusive prefix; *excl receives the exclusive one -- equal, bit
+// for bit, to the inclusive prefix of the previous thread -- and *total the block total.
+__device__ __forceinline__ double block_scan(double v, double* wsum, double* excl, double* total) {
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  double inc = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const double t = __shfl_up_sync(0xffffffffu, inc, o);
+    if (lane >= o) inc += t;
+  }
+  double exc = __shfl_up_sync(0xffffffffu, inc, 1);
+  if (lane == 0) exc = 0.0;
+  __syncthreads();  // wsum is free (its previous use has been read)
+  if (lane == 31) wsum[wid] = inc;
+  __syncthreads();
+  double before = 0.0, tot = 0.0;
+  for (int w = 0; w < (int)(blockDim.x >> 5); ++w) {
+    if (w == wid) before = tot;
+    tot += wsum[w];
+  }
+  *excl = before + exc;
+  *total = tot;
+  return before + inc;
+}
+
+// One block per row.  Pass 1: the residual's total Z (fixed-order sum).  Pass 2: walk the row in
+// tiles of 4 columns per thread, coalesced; a block scan of the per-thread sums gives every thread an
+// interval [lo, hi) of the running sum that tiles the row exactly (the tile base carries over
+// bit-exactly); the thread whose interval holds u * Z finds the column among its four.
 __global__ void __launch_bounds__(kFinThreads) k_sample_finish(SampleArgs a, int32_t* __restrict__ accept_out,
                                                                 int32_t* __restrict__ next_out) {
   pdl_wait();
   pdl_trigger();
   __shared__ double wsum[kFinThreads / 32];
-  __shared__ int y_s, last_s;
-  const int b = blockIdx.x, tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  __shared__ int y_s, last_s, done_s;
+  const int b = blockIdx.x, tid = threadIdx.x;
   const uint32_t f = __ldcg(a.count + (size_t)a.B * a.L + b);
   const int k = a.L - (int)f;
   if (k >= a.L) {
@@ -175,52 +221,54 @@ __global__ void __launch_bounds__(kFinThreads) k_sample_finish(SampleArgs a, int
   const float4 st = __ldcg(a.stats + n);
   const float* trow = a.T + n * a.V;
   const float* drow = a.D ? a.D + n * a.V : nullptr;
-  const int per = (a.V + kFinThreads - 1) / kFinThreads;
-  const int v0 = min(a.V, tid * per), v1 = min(a.V, v0 + per);
+  constexpr int kTile = 4 * kFinThreads;
+  if (tid == 0) { y_s = -1; last_s = -1; done_s = 0; }
+  // pass 1: the total, and the last column with mass
   double own = 0.0;
   int lastpos = -1;
-  for (int v = v0; v < v1; ++v) {
-    const float r = residual_at(a, trow, drow, x, st, v);
-    own += (double)r;
-    if (r > 0.f) lastpos = v;
-  }
-  // Inclusive scan of the per-thread sums in thread order (fixed): within each warp, then over the
-  // warp totals.  Thread t's interval is [lo, hi) with lo equal -- bit for bit -- to the hi of thread
-  // t - 1 (the same additions), so the intervals tile [0, total) and exactly one thread holds a draw.
-  double inc = own;
+  for (int v = 4 * tid; v < a.V; v += kTile) {
+    float r[4];
+    residual4(a, trow, drow, x, st, v, r);
 #pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const double t = __shfl_up_sync(0xffffffffu, inc, o);
-    if (lane >= o) inc += t;
-  }
-  double exc = __shfl_up_sync(0xffffffffu, inc, 1);
-  if (lane == 0) exc = 0.0;
-  if (lane == 31) wsum[wid] = inc;
-  if (tid == 0) { y_s = -1; last_s = -1; }
-  __syncthreads();
-  double before = 0.0, total = 0.0;
-  for (int w = 0; w < kFinThreads / 32; ++w) {
-    if (w == wid) before = total;
-    total += wsum[w];
-  }
-  const double lo = before + exc, hi = before + inc;
-  const double target = (double)a.uni[(size_t)b * (a.L + 1) + a.L] * total;
-  if (lo <= target && target < hi) {  // this thread's columns hold the draw
-    double run = lo;
-    int y = -1;
-    for (int v = v0; v < v1; ++v) {
-      const float r = residual_at(a, trow, drow, x, st, v);
-      run += (double)r;
-      if (run > target && r > 0.f) { y = v; break; }
+    for (int e = 0; e < 4; ++e) {
+      own += (double)r[e];
+      if (r[e] > 0.f) lastpos = v + e;
     }
-    if (y < 0) y = lastpos;  // rounding at the chunk's end
-    atomicMax(&y_s, y);
   }
+  double excl, total;
+  block_scan(own, wsum, &excl, &total);
   if (lastpos >= 0) atomicMax(&last_s, lastpos);
+  const double target = (double)a.uni[(size_t)b * (a.L + 1) + a.L] * total;
+  // pass 2: the tile and column where the running sum first exceeds the target
+  double base = 0.0;
+  for (int v0 = 0; v0 < a.V; v0 += kTile) {
+    const int v = v0 + 4 * tid;
+    float r[4] = {0.f, 0.f, 0.f, 0.f};
+    if (v < a.V) residual4(a, trow, drow, x, st, v, r);
+    const double s4 = (((double)r[0] + (double)r[1]) + (double)r[2]) + (double)r[3];
+    double ex, tile_total;
+    const double inc = block_scan(s4, wsum, &ex, &tile_total);
+    const double lo = base + ex, hi = base + inc;
+    if (lo <= target && target < hi) {  // exactly one thread of one tile
+      double run = lo;
+      int y = -1, lp = -1;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        run += (double)r[e];
+        if (r[e] > 0.f) lp = v + e;
+        if (y < 0 && run > target && r[e] > 0.f) y = v + e;
+      }
+      y_s = y >= 0 ? y : lp;  // rounding within the four: the last of them with mass
+      done_s = 1;
+    }
+    base = base + tile_total;
+    __syncthreads();
+    if (done_s) break;  // block-uniform
+  }
   __syncthreads();
   if (tid == 0) {
     accept_out[b] = k;
-    next_out[b] = y_s >= 0 ? y_s : last_s;  // the draw lies past the total: the last v with mass
+    next_out[b] = y_s >= 0 ? y_s : last_s;  // the draw lies past the running total: the last v with mass
   }
 }
 

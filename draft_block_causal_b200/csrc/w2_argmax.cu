@@ -8,7 +8,9 @@
 //
 // One CTA per SM owns one contiguous range of the vocabulary -- 16-column units, balanced to within
 // one unit -- and walks it in tiles of up to 128 columns (the last tile of a range may be narrower:
-// its MMA and loads shrink to its width).  Roles:
+// its MMA and loads shrink to its width).  The range is chosen by the SM the CTA runs on
+// (sm_affinity.cuh), so that at every position of the block the same SM reads the same W2 rows and
+// finds them in the L2 of its own die.  Roles:
 //   - the activation band u [128 x r] sits in TMEM as the A operand of tcgen05.mma for the whole
 //     launch (lane = batch row; 32-bit column c holds k = 2c and 2c + 1), so shared memory holds only
 //     the streamed operands;
@@ -32,6 +34,7 @@
 #include "common.cuh"
 #include "gemm_tc.h"
 #include "launch.cuh"
+#include "sm_affinity.cuh"
 #include "umma.cuh"
 
 #include <algorithm>
@@ -63,9 +66,14 @@ struct W2Args {
   long long ldo;
   int M, V, r;
   int last;            // the call's last read of W2: evict-first instead of evict-last
+  uint32_t* claim;     // work-slot claim words (one per SM, zero before the call's first launch), or null
+  uint32_t epoch;      // nonzero, distinct for every launch that shares the claim words
   int32_t* status;
   unsigned long long limit;
-  unsigned long long* trace;  // [gridDim.x][16] globaltimer stamps, or null
+  unsigned long long* trace;  // [gridDim.x][16] globaltimer stamps (ns), or null -- slots:
+  // 0 start, 1 end, 2 first W2 stage issued, 3 first L_base tile issued, 4 u band in TMEM (MMA side),
+  // 5 first MMA issued, 6 first accumulator in the epilogue, 7 epilogue done, 8 last MMA committed,
+  // 9 last W2 stage issued, 10 last L_base tile issued, 11 tiles, 15 wait on the previous grid done
 };
 
 __device__ __forceinline__ void tstamp(unsigned long long* trace, int k, unsigned long long v) {
@@ -95,9 +103,12 @@ __global__ void __launch_bounds__(kW2Threads, 1)
   uint64_t* best_s = mma_done + 1;  // [128] the second column group's best key per row
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(best_s + 128);
   volatile int* abort_s = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* slot_s = reinterpret_cast<volatile int*>(tmem_slot + 2);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int G = gridDim.x, c = blockIdx.x;
+  if (threadIdx.x == 0) *slot_s = claim_slot(p.claim, p.epoch);
+  __syncthreads();
+  const int G = gridDim.x, c = *slot_s;  // this CTA's vocabulary range (by the SM it runs on)
   const int nunits = (p.V + kUnit - 1) / kUnit;
   const int u0 = (int)((long long)nunits * c / G), u1 = (int)((long long)nunits * (c + 1) / G);
   const int ntiles = (u1 - u0 + kTileUnits - 1) / kTileUnits;
@@ -147,8 +158,10 @@ __global__ void __launch_bounds__(kW2Threads, 1)
             for (int j = 0; j < w; ++j)
               tma_load_2d_hint(dst + j * (kUnit * 128), &tmWn, &full[s], kb * 64, n0 + j * kUnit, pol);
           }
+          if (it == 0) tstamp(p.trace, 2, globaltimer_ns());
         }
       }
+      tstamp(p.trace, 9, globaltimer_ns());
       if (!ok) *abort_s = 1;
       int never = 0;  // no copy may be in flight when the CTA exits
       for (uint32_t j = (it > (uint32_t)kStages ? it - kStages : 0u); j < it; ++j)
@@ -167,13 +180,16 @@ __global__ void __launch_bounds__(kW2Threads, 1)
         for (int bx = 0; bx < nb; ++bx)
           tma_load_2d_hint(side_ring + (size_t)sl * kSideBytes + bx * kBoxBytes, &tmL, &sfull[sl], n0 + bx * 64, 0,
                            pol);
+        if (t == 0) tstamp(p.trace, 3, globaltimer_ns());
       }
+      tstamp(p.trace, 10, globaltimer_ns());
       int never = 0;
       for (int j = max(0, t - kSide); j < t; ++j) mbar_wait_bounded(&sfull[j % kSide], (j / kSide) & 1, limit, &never);
     }
   } else if (warp == 1) {
     if (lane == 0) {  // ---- MMA issuer ----
       bool ok = mbar_wait_bounded(a_ready, 0u, limit, abort_s);
+      tstamp(p.trace, 4, globaltimer_ns());
       tmem_fence_after_sync();
       uint32_t it = 0;
       for (int t = 0; t < ntiles && ok; ++t) {
@@ -193,10 +209,13 @@ __global__ void __launch_bounds__(kW2Threads, 1)
             umma_bf16_ta(d_tmem, tbase + (uint32_t)(kb * 32 + k * 8), sw128_desc(b_addr + 32 * k), idesc,
                          (kb | k) != 0);
           umma_commit(&empty[s]);
+          if (it == 0) tstamp(p.trace, 5, globaltimer_ns());
         }
         if (!ok) break;
         umma_commit(&accf[a]);
       }
+      tstamp(p.trace, 8, globaltimer_ns());
+      tstamp(p.trace, 11, (unsigned long long)ntiles);
       if (!ok) *abort_s = 1;
       int never = 0;  // TMEM may be freed only once every issued MMA has finished
       umma_commit(mma_done);
@@ -234,6 +253,7 @@ __global__ void __launch_bounds__(kW2Threads, 1)
       const uint32_t a = t & 1, aph = (t >> 1) & 1;
       const int sl = t % kSide;
       if (!mbar_wait_warp(&accf[a], aph, limit, abort_s)) { *abort_s = 1; break; }
+      if (t == 0 && warp == 4 && lane == 0) tstamp(p.trace, 6, globaltimer_ns());
       if (!mbar_wait_warp(&sfull[sl], (t / kSide) & 1, limit, abort_s)) { *abort_s = 1; break; }
       tmem_fence_after_sync();
       const int cb = g * 64;
@@ -303,6 +323,7 @@ __global__ void __launch_bounds__(kW2Threads, 1)
         mbar_arrive(&sempty[sl]);
       }
     }
+    if (warp == 4 && lane == 0) tstamp(p.trace, 7, globaltimer_ns());
     // the two column groups of a row meet in shared memory; one atomicMax per row and CTA
     const uint64_t key = idx >= 0 ? argmax_key(best, idx) : 0ull;
     if (g == 1) best_s[row] = key;
@@ -343,9 +364,13 @@ bool w2_argmax_supported(int M, int V, int r, const void* U, const void* W2, con
 }
 
 cudaError_t w2_argmax(const bf16* U, const bf16* W2, int M, int V, int r, const bf16* Lb, long long ldl,
-                      uint64_t* keys, float* out, long long ldo, bool last, int32_t* status, uint64_t limit,
-                      cudaStream_t st) {
+                      uint64_t* keys, float* out, long long ldo, bool last, uint32_t* claim, uint32_t epoch,
+                      int32_t* status, uint64_t limit, cudaStream_t st) {
   if (!w2_argmax_supported(M, V, r, U, W2, Lb, ldl)) return cudaErrorInvalidValue;
+  if (claim) {
+    cudaError_t e = ensure_sm_rank(st);
+    if (e != cudaSuccess) return e;
+  }
   CUtensorMap tw, twn, tl;
   if (!tmap_bf16_tiles(&tw, W2, (uint64_t)V, (uint64_t)r, 128) || !tmap_bf16_tiles(&twn, W2, (uint64_t)V, (uint64_t)r, kUnit) ||
       !tmap_bf16_tiles(&tl, Lb, (uint64_t)M, (uint64_t)V, 128, (uint64_t)ldl))
@@ -354,7 +379,8 @@ cudaError_t w2_argmax(const bf16* U, const bf16* W2, int M, int V, int r, const 
   if (e != cudaSuccess) return e;
   const int nunits = (V + kUnit - 1) / kUnit;
   const int grid = std::max(1, std::min(sm_count(), nunits));
-  W2Args a{U, keys, out, ldo, M, V, r, last ? 1 : 0, status, (unsigned long long)limit, nullptr};
+  W2Args a{U, keys, out, ldo, M, V, r, last ? 1 : 0, grid == sm_count() ? claim : nullptr, epoch, status,
+           (unsigned long long)limit, nullptr};
   int ntrace = 0;
   debug_trace(&a.trace, &ntrace);
   if (a.trace && ntrace < grid * 16) a.trace = nullptr;

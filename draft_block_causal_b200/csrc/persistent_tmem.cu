@@ -13,6 +13,8 @@
 //     columns [R*d/256, (R+1)*d/256) and the W_hh rows after them (packed bf16 pairs).
 //  2. The W2 stream is register double-buffered (the next chunk's loads are issued before the
 //     current chunk is reduced) and its first chunk is issued between barrier arrival and wait.
+//     (Staging it through shared memory -- a ring of 1-D bulk copies, or of cp.async chunks three
+//     ahead per warp -- measured slower: 198 and 191 us for the W2 pass against 129 us.)
 //  3. The W1 state-block partials are spread over kRep replicas of the accumulator, cutting the
 //     number of same-address atomics per replica from G to G/kRep.  Every partial sum that
 //     several CTAs or warps add into (these accumulators, and the GRU gate sums in shared

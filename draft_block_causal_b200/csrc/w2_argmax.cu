@@ -13,7 +13,10 @@
 // finds them in the L2 of its own die.  Roles:
 //   - the activation band u [128 x r] sits in TMEM as the A operand of tcgen05.mma for the whole
 //     launch (lane = batch row; 32-bit column c holds k = 2c and 2c + 1), so shared memory holds only
-//     the streamed operands;
+//     the streamed operands.  It arrives by one TMA load into two L_base ring slots that have not
+//     been filled yet, and each epilogue thread moves its row from there into its TMEM lane (one
+//     16-byte shared-memory read per chunk, where loading it from global memory row by row took
+//     one L2 request per row and chunk: 4.6 us for 128 rows against the MMAs' 15);
 //   - warp 0 streams W2 tiles (K-major, 128-byte swizzle) through a ring of kStages k-block stages
 //     with an L2 evict-last policy: W2 (77.8 MB at V = 151936) is re-read at every position of the
 //     block and should stay in B200's 126 MB L2 while the operands streamed beside it pass through.
@@ -60,9 +63,11 @@ constexpr size_t kRingBytes = (size_t)kStages * kStageBytes + (size_t)kSide * kS
 constexpr size_t kMiscBytes = 1280;     // mbarriers, TMEM slot, flags, the cross-group argmax
 constexpr size_t kSmemBytes = kRingBytes + kMiscBytes + 1024;  // + alignment slack
 static_assert(kSmemBytes <= 232448, "shared memory budget");
+// The u band (128 rows x r <= 256, bf16: at most four 128 x 64 boxes) is staged through L_base ring
+// slots 1 and 2 before their first L_base tile.
+static_assert(kSide >= 3 && 2 * kSideBytes >= 4 * kBoxBytes, "u band staging space");
 
 struct W2Args {
-  const bf16* U;       // [M][r] activations (bf16), row-major
   uint64_t* keys;      // [M] argmax keys (atomicMax)
   float* out;          // optional z: out[m * ldo + v]
   long long ldo;
@@ -90,7 +95,7 @@ __device__ __forceinline__ const uint4* side_at(const uint8_t* side, int row, in
 
 __global__ void __launch_bounds__(kW2Threads, 1)
     k_w2_argmax(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmWn,
-                const __grid_constant__ CUtensorMap tmL, W2Args p) {
+                const __grid_constant__ CUtensorMap tmL, const __grid_constant__ CUtensorMap tmU, W2Args p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   uint8_t* side_ring = ring + (size_t)kStages * kStageBytes;
@@ -102,7 +107,8 @@ __global__ void __launch_bounds__(kW2Threads, 1)
   uint64_t* acce = accf + 2;
   uint64_t* a_ready = acce + 2;
   uint64_t* mma_done = a_ready + 1;
-  uint64_t* best_s = mma_done + 1;  // [128] the second column group's best key per row
+  uint64_t* u_full = mma_done + 1;
+  uint64_t* best_s = u_full + 1;  // [128] the second column group's best key per row
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(best_s + 128);
   volatile int* abort_s = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* slot_s = reinterpret_cast<volatile int*>(tmem_slot + 2);
@@ -124,11 +130,13 @@ __global__ void __launch_bounds__(kW2Threads, 1)
     for (int a = 0; a < 2; ++a) { mbar_init(&accf[a], 1); mbar_init(&acce[a], kEpiWarps); }
     mbar_init(a_ready, kEpiWarps);
     mbar_init(mma_done, 1);
+    mbar_init(u_full, 1);
     *abort_s = 0;
     mbar_fence_init();
     tma_prefetch_desc(&tmW);
     tma_prefetch_desc(&tmWn);
     tma_prefetch_desc(&tmL);
+    tma_prefetch_desc(&tmU);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, kTmemCols);
@@ -176,6 +184,8 @@ __global__ void __launch_bounds__(kW2Threads, 1)
       for (; t < ntiles; ++t) {
         const int sl = t % kSide;
         if (!mbar_wait_bounded(&sempty[sl], ((t / kSide) & 1) ^ 1, limit, abort_s)) { *abort_s = 1; break; }
+        // slots 1 and 2 hold the u band until the epilogue has moved it into TMEM
+        if ((t == 1 || t == 2) && !mbar_wait_bounded(a_ready, 0u, limit, abort_s)) { *abort_s = 1; break; }
         const int ut = u0 + t * kTileUnits, w = min(kTileUnits, u1 - ut);
         const int n0 = ut * kUnit, nb = (w * kUnit + 63) / 64;
         mbar_arrive_expect_tx(&sfull[sl], (uint32_t)nb * kBoxBytes);
@@ -229,15 +239,23 @@ __global__ void __launch_bounds__(kW2Threads, 1)
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
     pdl_wait();  // u comes from the previous kernel; keys and logits may be read by earlier ones
     if (warp == 4 && lane == 0) tstamp(p.trace, 15, globaltimer_ns());
-    {  // u band into TMEM columns [0, r/2): the two warps of a lane quadrant take half the columns
-      // each; every load is issued before the first TMEM store (the stores are ordered with memory
-      // operations, so interleaving them would serialise one L2 round trip per load)
+    {  // u band into TMEM columns [0, r/2): one TMA load of 128 rows x r into ring slots 1 and 2
+      // (rows past M read as zeros), then each thread moves its row (= TMEM lane) out of the
+      // swizzled boxes, the two warps of a lane quadrant half of the columns each
+      uint8_t* ubuf = side_ring + kSideBytes;
+      const int nbox = p.r / 64;
+      if (warp == 4 && lane == 0) {
+        mbar_arrive_expect_tx(u_full, (uint32_t)nbox * kBoxBytes);
+        for (int bx = 0; bx < nbox; ++bx) tma_load_2d(ubuf + bx * kBoxBytes, &tmU, u_full, bx * 64, 0);
+      }
+      if (!mbar_wait_warp(u_full, 0u, limit, abort_s)) *abort_s = 1;
       const int half = p.r / 4;  // 32-bit words per warp: a multiple of 16 (r is a multiple of 64)
-      const uint4* src = reinterpret_cast<const uint4*>(p.U + (size_t)row * p.r) + g * half / 4;
       uint4 v[16];
 #pragma unroll
-      for (int i = 0; i < 16; ++i)
-        v[i] = (4 * i < half && row < p.M) ? __ldg(src + i) : make_uint4(0u, 0u, 0u, 0u);
+      for (int i = 0; i < 16; ++i) {
+        const int k0 = g * (p.r / 2) + 8 * i;  // first of the chunk's 8 k values
+        v[i] = 4 * i < half ? *side_at(ubuf, row, k0) : make_uint4(0u, 0u, 0u, 0u);
+      }
 #pragma unroll
       for (int i = 0; i < 16; ++i)
         if (4 * i < half) tmem_st4(tbase + lane_off + (uint32_t)(g * half + 4 * i), v[i]);
@@ -336,6 +354,10 @@ __global__ void __launch_bounds__(kW2Threads, 1)
     }
   }
 
+  if (warp == 4 && lane == 0) {  // no u copy may be in flight when the CTA exits (a timed-out wait)
+    int never = 0;
+    mbar_wait_bounded(u_full, 0u, limit, &never);
+  }
   tmem_fence_before_sync();
   __syncthreads();
   tmem_fence_after_sync();
@@ -373,20 +395,21 @@ cudaError_t w2_argmax(const bf16* U, const bf16* W2, int M, int V, int r, const 
     cudaError_t e = ensure_sm_rank(st);
     if (e != cudaSuccess) return e;
   }
-  CUtensorMap tw, twn, tl;
+  CUtensorMap tw, twn, tl, tu;
   if (!tmap_bf16_tiles(&tw, W2, (uint64_t)V, (uint64_t)r, 128) || !tmap_bf16_tiles(&twn, W2, (uint64_t)V, (uint64_t)r, kUnit) ||
-      !tmap_bf16_tiles(&tl, Lb, (uint64_t)M, (uint64_t)V, 128, (uint64_t)ldl))
+      !tmap_bf16_tiles(&tl, Lb, (uint64_t)M, (uint64_t)V, 128, (uint64_t)ldl) ||
+      !tmap_bf16_tiles(&tu, U, (uint64_t)M, (uint64_t)r, 128))
     return cudaErrorInvalidValue;
   cudaError_t e = set_smem_w2_once();
   if (e != cudaSuccess) return e;
   const int nunits = (V + kUnit - 1) / kUnit;
   const int grid = std::max(1, std::min(sm_count(), nunits));
-  W2Args a{U, keys, out, ldo, M, V, r, last ? 1 : 0, grid == sm_count() ? claim : nullptr, epoch, status,
+  W2Args a{keys, out, ldo, M, V, r, last ? 1 : 0, grid == sm_count() ? claim : nullptr, epoch, status,
            (unsigned long long)limit, nullptr};
   int ntrace = 0;
   debug_trace(&a.trace, &ntrace);
   if (a.trace && ntrace < grid * 16) a.trace = nullptr;
-  return note_launch(launch_pdl(k_w2_argmax, dim3(grid), dim3(kW2Threads), kSmemBytes, st, tw, twn, tl, a));
+  return note_launch(launch_pdl(k_w2_argmax, dim3(grid), dim3(kW2Threads), kSmemBytes, st, tw, twn, tl, tu, a));
 }
 
 }  // namespace domino

@@ -309,6 +309,49 @@ def w2_kernel_us(pt: Point, flush, stream) -> float:
     return float((t[:, 1].max() - t[:, 15].min()) / 1e3)
 
 
+def batched_phases(pt: Point, flush, stream) -> dict:
+    """Phase times of the persistent batched greedy kernel (k_greedy_batched) in one greedy call, from
+    CTA 0's stamps: its start, the moment it passed each grid barrier (every CTA had finished the
+    phase before it) and its end.  Phases in launch order: C0, D0, E0, then per position A (W2
+    argmax), B (W_ih product; absent with the projection table), C (cell), D (W_hh|W1 product), E
+    (next activations); the last position runs A only."""
+    torch, domino = pt.torch, pt.domino
+    buf = torch.zeros(1024, dtype=torch.int64, device=pt.lb.device)
+    flush.zero_()
+    torch.cuda.synchronize()
+    domino.set_trace(buf)
+    try:
+        pt.greedy(stream)
+        torch.cuda.synchronize()
+    finally:
+        domino.set_trace(None)
+    t = buf.cpu().numpy().astype(np.int64)
+    L, proj = pt.sh["L"], pt.w.embed_proj is not None
+    names = ["C", "D", "E"]
+    for i in range(L):
+        names.append("A")
+        if i < L - 1:
+            names += (["C"] if proj else ["B", "C"]) + ["D", "E"]
+    dur = [(t[j + 1] - t[j]) / 1e3 for j in range(len(names))]
+    out = {"kernel_us": round(float(t[len(names)] - t[0]) / 1e3, 2), "phases_us_summed": {}}
+    for n in "ABCDE":
+        out["phases_us_summed"][n] = round(sum(d for d, m in zip(dur, names) if m == n), 2)
+    a = [d for d, m in zip(dur, names) if m == "A"]
+    out["w2_phase_us_median"] = round(float(np.median(a)), 2)
+    return out
+
+
+def w2_us_of(pt: Point, flush, stream):
+    """(µs, note) of one position's W2 product with the fused argmax on the batched path."""
+    if "k_greedy_batched" in pt.domino.greedy_plan(pt.domino.make_shape(pt.w, pt.sh["B"], pt.sh["L"])):
+        ph = batched_phases(pt, flush, stream)
+        return ph["w2_phase_us_median"], ("phase A (W2 product, L_base, argmax) of the persistent batched kernel, "
+                                          "median over the positions, from CTA 0's grid-barrier stamps (the "
+                                          "slowest CTA and the barrier included)"), ph
+    return w2_kernel_us(pt, flush, stream), ("last position's W2 GEMM with fused argmax, one launch, from its own "
+                                             "device clock stamps"), None
+
+
 def full_accept_targets(pt: Point, stream):
     """Target logits on which every draft token of the point's greedy call is the argmax: the
     draft's own final logits (one greedy call with logits written, untimed)."""
@@ -604,7 +647,7 @@ def run_ours(args):
                 psh = p.sh
                 ga = statistics.mean(g_ms)
                 fl = greedy_flops(psh)
-                w2_us = w2_kernel_us(p, flush, stream)
+                w2_us, w2_note, phases = w2_us_of(p, flush, stream)
                 w2_flops = 2.0 * psh["B"] * psh["V"] * psh["r"]
                 points[str(pb)] = {
                     "blocks_per_s": round(pb * len(s_ms) / (sum(s_ms) * 1e-3), 1),
@@ -618,9 +661,13 @@ def run_ours(args):
                     "greedy_tflops": round(fl / (ga * 1e-3) / 1e12, 2),
                     "w2_argmax_gemm": {"us": round(w2_us, 2), "tflops": round(w2_flops / (w2_us * 1e-6) / 1e12, 1),
                                        "tensor_frac": round(w2_flops / (w2_us * 1e-6) / 1e12 / peaks["bf16_tflops"], 4),
-                                       "note": "last position's W2 GEMM with fused argmax, one launch, from its "
-                                               "own device clock stamps"},
+                                       # the W2 phase streams W2 and the L_base rows from HBM at every position
+                                       "hbm_frac": round(2.0 * psh["V"] * (psh["r"] + psh["B"]) / (w2_us * 1e-6) / 1e9
+                                                         / peaks["hbm_gbs"], 4),
+                                       "note": w2_note},
                 }
+                if phases:
+                    points[str(pb)]["batched_kernel_phases"] = phases
                 # The synthetic targets (base + N(0, 0.5)) reject most drafts within two positions, so
                 # the early-exit accept length skips most target reads.  For a step whose accept
                 # length is the whole block -- every target row read, as with drafts that mostly
@@ -689,8 +736,8 @@ def run_ours(args):
                        "accept_mean": round(float(p.acc.float().mean().item()), 3),
                        "hbm_frac": round(greedy_bytes(psh) / (ga * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
                        "tensor_frac": round(greedy_flops(psh) / (ga * 1e-3) / 1e12 / peaks["bf16_tflops"], 4)}
-                if pb > 4:  # the batched path: one W2 argmax launch from its own clock stamps
-                    w2_us = w2_kernel_us(p, flush, stream)
+                if pb > 4:  # the batched path: the W2 product of one position
+                    w2_us, _, _ = w2_us_of(p, flush, stream)
                     w2_flops = 2.0 * min(pb, 128) * psh["V"] * psh["r"]
                     ent["w2_argmax_us"] = round(w2_us, 2)
                     ent["w2_tensor_frac"] = round(w2_flops / (w2_us * 1e-6) / 1e12 / peaks["bf16_tflops"], 4)
@@ -782,12 +829,15 @@ def profile_driver(n: int, batch: int = 1, trace: bool = False, proj: bool = Fal
     stream = torch.cuda.current_stream()
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
     L = pt.sh["L"]
-    if trace and batch > 4:  # the batched path: the W2 argmax launch's phases
+    if trace and batch > 4:  # the batched path: the persistent kernel's phases, or the W2 launch's
         for _ in range(n):
             flush.zero_()
             pt.greedy(stream)
         torch.cuda.synchronize()
-        print(json.dumps({"B": batch, "w2_argmax_phases_us": w2_kernel_phases(pt, flush, stream)}), flush=True)
+        if "k_greedy_batched" in pt.domino.greedy_plan(pt.domino.make_shape(pt.w, batch, L)):
+            print(json.dumps({"B": batch, "batched_kernel_phases": batched_phases(pt, flush, stream)}), flush=True)
+        else:
+            print(json.dumps({"B": batch, "w2_argmax_phases_us": w2_kernel_phases(pt, flush, stream)}), flush=True)
         return
     buf = torch.zeros(4 + 10 * L, dtype=torch.int64, device=device)
     for k in range(n):

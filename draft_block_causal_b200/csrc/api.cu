@@ -120,6 +120,7 @@ Workspace layout_workspace(const Shape& s, void* base) {
   w.Gx = reinterpret_cast<float*>(take(3 * (size_t)s.Hs * BL * sizeof(float)));
   w.Gh = reinterpret_cast<float*>(take(3 * (size_t)s.Hs * s.B * sizeof(float)));
   w.S_hl = reinterpret_cast<__nv_bfloat16*>(take(2 * BL * s.Hs * sizeof(__nv_bfloat16)));
+  w.part = reinterpret_cast<float*>(take(batched_partial_floats(s) * sizeof(float)));
   w.bytes = off;
   return w;
 }
@@ -160,6 +161,7 @@ const char* domino_greedy_plan(const domino_shape_t* shape) {
   if (check_shape(shape) != DOMINO_OK) return "invalid shape";
   const Shape s = to_shape(shape);
   if (use_persistent_greedy(s)) return persistent_plan(s);
+  if (batched_shape_ok(s)) return batched_plan();
   if (s.dtype == DOMINO_DTYPE_BF16 && s.d % 64 == 0 && s.r % 64 == 0) {
     if (s.Hs % 64 != 0)
       return "per-phase kernels: tcgen05 H-projection GEMM, then per position k_u + tcgen05 W2 GEMM with the argmax "
@@ -275,6 +277,18 @@ int domino_draft_greedy(const domino_shape_t* shape, const domino_weights_t* w, 
   if (use_persistent_greedy(s)) return cuda_rc(launch_persistent_greedy(s, *w, base_logits, hidden, S0, tokens_out,
                                                                          logits_out, states_out, ws, st,
                                                                          spin_limit(), cs));
+  if (use_greedy_batched(s, *w, base_logits)) {
+    // the barrier counter, the work-slot claims and the argmax keys are adjacent: one memset
+    cudaError_t e =
+        cudaMemsetAsync(ws.sync, 0, (char*)(ws.keys + (size_t)s.B * s.L) - (char*)ws.sync, cs);
+    if (e == cudaSuccess)  // P[n][k] = sum_c W1[k][c] H[n][c] for every (row, position) n
+      e = gemm_tc_store_f32_t((const __nv_bfloat16*)w->W1, (const __nv_bfloat16*)hidden, s.r, s.B * s.L, s.d, 0,
+                              ws.P, s.r, st, spin_limit(), cs, 0, s.d + s.Hs);
+    if (e == cudaSuccess)
+      e = launch_greedy_batched(s, *w, base_logits, S0, logits_out, states_out, ws, st, spin_limit(), cs);
+    if (e == cudaSuccess) e = launch_tokens_from_keys(ws.keys, s.B, s.L, tokens_out, cs);
+    return cuda_rc(e);
+  }
 
   const size_t BL = (size_t)s.B * s.L;
   // Batches the fused kernel does not take: one launch per phase and position.  With bf16 storage

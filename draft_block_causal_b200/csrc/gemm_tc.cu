@@ -698,20 +698,28 @@ __global__ void __launch_bounds__(EpiWarps<Epi>::kThreads, 1)
           cluster_wait();  // every CTA of the cluster is running
           waited_first = true;
         }
+        // up to 64 columns of TMEM loads in flight per wait: one load latency per batch rather than
+        // one per 16-column unit
+        constexpr int kCh = BN >= 64 ? 64 : BN;
 #pragma unroll 1
-        for (int c0 = 0; c0 < BN; c0 += 16) {
-          uint32_t r[16];
-          tmem_ld16(taddr + c0, r);
-          tmem_wait_ld();
-          const int u = (c0 >> 4) * kBM + row;
-          const int o = unit_owner(u, ksplit, U);
-          const int li = u - unit_first(o, ksplit, U);
-          const uint32_t base = cluster_map(recv, o);
+        for (int c0 = 0; c0 < BN; c0 += kCh) {
+          uint32_t r[kCh];
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            reg_fence(r[4 * j]); reg_fence(r[4 * j + 1]); reg_fence(r[4 * j + 2]); reg_fence(r[4 * j + 3]);
-            st_cluster_f4(base + slot_offset(piece * nmax + li, li, j), __uint_as_float(r[4 * j]),
-                          __uint_as_float(r[4 * j + 1]), __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3]));
+          for (int h = 0; h < kCh / 16; ++h) tmem_ld16(taddr + c0 + 16 * h, &r[16 * h]);
+          tmem_wait_ld();
+#pragma unroll
+          for (int h = 0; h < kCh / 16; ++h) {
+            const int u = ((c0 + 16 * h) >> 4) * kBM + row;
+            const int o = unit_owner(u, ksplit, U);
+            const int li = u - unit_first(o, ksplit, U);
+            const uint32_t base = cluster_map(recv, o);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              uint32_t* q4 = &r[16 * h + 4 * j];
+              reg_fence(q4[0]); reg_fence(q4[1]); reg_fence(q4[2]); reg_fence(q4[3]);
+              st_cluster_f4(base + slot_offset(piece * nmax + li, li, j), __uint_as_float(q4[0]),
+                            __uint_as_float(q4[1]), __uint_as_float(q4[2]), __uint_as_float(q4[3]));
+            }
           }
         }
         tmem_fence_before_sync();
@@ -1045,6 +1053,18 @@ cudaError_t launch_gemm_skinny(const void* A, const void* Bm, int M, int N, int 
 
 bool tmap_bf16_tiles(CUtensorMap* tm, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows, uint64_t ld) {
   return tmap_bf16(tm, base, rows, cols, box_rows, ld);
+}
+
+bool tmap_bf16_3d(CUtensorMap* tm, const void* base, uint64_t n0, uint64_t n1, uint64_t n2, uint32_t box2) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn || n0 % 8 != 0) return false;
+  cuuint64_t dims[3] = {n0, n1, n2};
+  cuuint64_t strides[2] = {n0 * 2, n0 * n1 * 2};
+  cuuint32_t box[3] = {(cuuint32_t)kBK, 1, box2};
+  cuuint32_t es[3] = {1, 1, 1};
+  return fn(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 int sm_count() {

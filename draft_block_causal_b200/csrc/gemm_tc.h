@@ -16,6 +16,10 @@ namespace domino {
 // of this library expect.  False when the driver's encoder is missing or refuses the map.
 bool tmap_bf16_tiles(CUtensorMap* tm, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows,
                      uint64_t ld = 0);
+// bf16 tensor [n2][n1][n0] (contiguous, n0 innermost) seen as boxes of 64 x 1 x box2 with 128-byte
+// swizzling: one box is box2 rows of 64 elements at one index of the middle dimension, laid out in
+// shared memory as a box_rows x 64 tile of tmap_bf16_tiles.  n0 must be a multiple of 8.
+bool tmap_bf16_3d(CUtensorMap* tm, const void* base, uint64_t n0, uint64_t n1, uint64_t n2, uint32_t box2);
 // SM count of the current device.
 int sm_count();
 

@@ -38,6 +38,7 @@ struct Workspace {
   __nv_bfloat16* S_hl; // [B*L][2Hs] two-term bf16 split of states
   unsigned long long* a_acc;  // [2][kAccReplicas][B][r] W1 state-block sums of the fused kernels
                               // (fixed point, see fix_add; ping-pong over positions)
+  float* part;         // partial sums of the persistent batched kernel (batched_partial_floats)
   size_t bytes;
 };
 constexpr int kSyncWords = 64;

@@ -36,4 +36,16 @@ cudaError_t launch_persistent_greedy(const Shape& s, const domino_weights_t& w, 
                                      float* states_out, const Workspace& ws, int32_t* status, uint64_t spin_limit,
                                      cudaStream_t st);
 
+// The persistent batched kernel (persistent_batched.cu): greedy drafting of 5..128 rows in one
+// cooperative launch, bf16 storage.  The caller computes ws.P (W1[:, :d] . H for every position)
+// and zeroes ws.sync, ws.claim and ws.keys before the launch, and turns the keys into tokens after.
+bool batched_shape_ok(const Shape& s);
+bool use_greedy_batched(const Shape& s, const domino_weights_t& w, const void* base_logits);
+const char* batched_plan();
+// Floats of ws.part the kernel needs for shape s (0 when the kernel does not take the shape).
+size_t batched_partial_floats(const Shape& s);
+cudaError_t launch_greedy_batched(const Shape& s, const domino_weights_t& w, const void* base_logits,
+                                  const float* S0, float* logits_out, float* states_out, const Workspace& ws,
+                                  int32_t* status, uint64_t spin, cudaStream_t st);
+
 }  // namespace domino

@@ -294,7 +294,10 @@ DOMINO_API int domino_draft_greedy_noalloc(const domino_shape_t* shape, const do
  * [0] start, [1] prologue done, [2] first barrier passed, [3] end, and for position i at
  * 4 + 10*i + {0: inputs staged, 1: W_hh products done, 2: W2 pass + CTA argmax done,
  * 3: argmax barrier passed, 4: embedding row staged, 5: W_ih products done, 6: state and W1
- * partials done, 7: state barrier passed}.  NULL turns it off.  Process-wide. */
+ * partials done, 7: state barrier passed}.  The persistent batched kernel (5..128 rows) records the
+ * globaltimer (ns) of CTA 0: [0] start, [e] when it passed grid barrier e (phases C0, D, E, then per
+ * position A, B, C, D, E -- B absent with a projection table -- and A alone at the last position),
+ * then its end.  NULL turns it off.  Process-wide. */
 DOMINO_API int domino_debug_set_trace(void* device_buf, int32_t n_entries);
 
 /* Test and tuning hook for the tensor-core GEMM engine behind the batched paths:

@@ -92,12 +92,13 @@ def _persistent_case(B=1, seed=300, Hs=256):
     return synth.make_workload(wl)
 
 
-def test_plan_names_the_fused_kernel_for_small_batches():
+def test_plan_names_the_kernel_of_each_batch_size():
     data = _persistent_case()
     w, lb, h, S0 = G.device_inputs(data)
     assert "k_greedy_persistent" in domino.greedy_plan(domino.make_shape(w, 1, 16))
     assert "k_greedy_persistent" in domino.greedy_plan(domino.make_shape(w, 4, 16))
-    assert "per-phase" in domino.greedy_plan(domino.make_shape(w, 32, 16))
+    assert "k_greedy_batched" in domino.greedy_plan(domino.make_shape(w, 32, 16))
+    assert "per-phase" in domino.greedy_plan(domino.make_shape(w, 200, 16))
     data = _persistent_case(Hs=512)
     w, lb, h, S0 = G.device_inputs(data)
     assert "k_greedy_tmem" in domino.greedy_plan(domino.make_shape(w, 2, 16))

@@ -29,7 +29,8 @@ CASES = [  # (B, L, d, Hs, V, plan substring)
     (1, 16, 4096, 1024, 20000, "k_greedy_tmem"),
     (3, 16, 1024, 512, 9000, "k_greedy_tmem"),
     (4, 16, 2560, 1024, 20000, "k_greedy_tmem"),
-    (32, 16, 1024, 512, 9000, "per-phase"),
+    (32, 16, 1024, 512, 9000, "k_greedy_batched"),
+    (136, 4, 512, 256, 3000, "per-phase"),
 ]
 
 

@@ -44,6 +44,10 @@ SMALL = [
     _custom(130, 3, 256, 256, 128, 5000, 1, 310),         # bands of 128 and 2 rows, r = 128
     _custom(40, 16, 512, 256, 256, 2056, 1, 320, s0_std=1.0, peak=0.5),  # 129 units: 129 CTAs
     _custom(9, 4, 128, 64, 64, 16, 1, 330),               # V = 16: one unit, one CTA
+    # the persistent batched kernel (5 <= B <= 128, Hs a multiple of 128): its smallest batch with a
+    # short block, a single position (no GRU update), r = 128 and a vocabulary of 65 units
+    _custom(5, 2, 256, 128, 128, 1000, 1, 340),
+    _custom(100, 1, 256, 128, 128, 1040, 1, 350),
 ]
 
 

@@ -313,10 +313,11 @@ def batched_phases(pt: Point, flush, stream) -> dict:
     """Phase times of the persistent batched greedy kernel (k_greedy_batched) in one greedy call, from
     CTA 0's stamps: its start, the moment it passed each grid barrier (every CTA had finished the
     phase before it) and its end.  Phases in launch order: C0, D0, E0, then per position A (W2
-    argmax), B (W_ih product; absent with the projection table), C (cell), D (W_hh|W1 product), E
-    (next activations); the last position runs A only."""
+    argmax), X (gather of the drafted rows) and B (W_ih product) -- both absent with the projection
+    table --, C (cell), D (W_hh|W1 product), E (next activations); the last position runs A only."""
     torch, domino = pt.torch, pt.domino
-    buf = torch.zeros(1024, dtype=torch.int64, device=pt.lb.device)
+    G = torch.cuda.get_device_properties(pt.lb.device).multi_processor_count
+    buf = torch.zeros(256 + 128 * G + 16 * G, dtype=torch.int64, device=pt.lb.device)
     flush.zero_()
     torch.cuda.synchronize()
     domino.set_trace(buf)
@@ -326,18 +327,37 @@ def batched_phases(pt: Point, flush, stream) -> dict:
     finally:
         domino.set_trace(None)
     t = buf.cpu().numpy().astype(np.int64)
+    arr = t[256:256 + 128 * G].reshape(128, G)  # [barrier - 1][CTA] arrival stamps
+    det = t[256 + 128 * G:].reshape(2, 8, G)     # phases B, D of position 1: per-CTA milestones
     L, proj = pt.sh["L"], pt.w.embed_proj is not None
     names = ["C", "D", "E"]
     for i in range(L):
         names.append("A")
         if i < L - 1:
-            names += (["C"] if proj else ["B", "C"]) + ["D", "E"]
+            names += (["C"] if proj else ["X", "B", "C"]) + ["D", "E"]
     dur = [(t[j + 1] - t[j]) / 1e3 for j in range(len(names))]
     out = {"kernel_us": round(float(t[len(names)] - t[0]) / 1e3, 2), "phases_us_summed": {}}
-    for n in "ABCDE":
+    for n in "AXBCDE":
         out["phases_us_summed"][n] = round(sum(d for d, m in zip(dur, names) if m == n), 2)
     a = [d for d, m in zip(dur, names) if m == "A"]
     out["w2_phase_us_median"] = round(float(np.median(a)), 2)
+    # per phase (all but the last): the slowest CTA's work (its arrival at the closing barrier) and
+    # the barrier itself (last arrival to CTA 0's release), summed by phase kind
+    work, sync = {}, {}
+    for j, m in enumerate(names[:-1]):
+        last = int(arr[j].max())
+        work[m] = work.get(m, 0.0) + (last - t[j]) / 1e3
+        sync[m] = sync.get(m, 0.0) + (t[j + 1] - last) / 1e3
+    out["slowest_cta_work_us_summed"] = {k: round(v, 2) for k, v in work.items()}
+    out["barrier_us_summed"] = {k: round(v, 2) for k, v in sync.items()}
+    for ph, name in ((0, "B"), (1, "D")):
+        d = det[ph]
+        ok = d[0] != 0
+        if ok.any():  # medians over the CTAs with an item, µs from each CTA's own phase start
+            out[f"phase_{name}_pos1_milestones_us"] = {
+                lab: round(float(np.median((d[k][ok & (d[k] != 0)] - d[0][ok & (d[k] != 0)]))) / 1e3, 2)
+                for k, lab in ((1, "producer_done"), (2, "gather_done"), (3, "mmas_issued"), (4, "acc_in_epilogue"),
+                               (5, "epilogue_done")) if (ok & (d[k] != 0)).any()}
     return out
 
 

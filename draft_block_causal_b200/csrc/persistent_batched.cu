@@ -5,15 +5,15 @@
 // is computed for every position before the launch), z = L_base[i] + W2 . u, t_i = argmax z (lowest
 // index on ties), S_i = GRUCell(embed[t_i], S_{i-1}) in the PyTorch gate form.
 //
-// Every position runs five phases, separated by bounded grid barriers:
+// Every position runs six phases, separated by bounded grid barriers:
 //   A  W2 argmax.  The u band (rows = batch, bf16) arrives by TMA into two L_base ring slots and moves
 //      into TMEM as the A operand of tcgen05.mma; W2 tiles (warp 0) and L_base tiles (warp 2) stream
 //      by TMA into shared-memory rings; warp 1 issues the MMAs into two 128 x 128 accumulators; warps
 //      4..11 add L_base, fold the argmax (u64 keys, atomicMax per row and CTA) and write the logits
 //      when asked.  Each CTA owns the vocabulary range of the SM it runs on, as in k_w2_argmax.
-//   B  gate inputs W_ih . embed[t_i].  Item = (128-row tile of W_ih, K slice): one item per CTA.
-//      Warp 0 streams the W_ih tile by TMA, warps 2..3 gather the embedding rows of the drafted
-//      tokens into the same stages with cp.async (128-byte swizzle), warp 1 issues the MMAs into one
+//   X  every thread copies a share of the embedding rows of the drafted tokens into a row buffer.
+//   B  gate inputs W_ih . x.  Item = (128-row tile of W_ih, K slice): one item per CTA.  Warp 0
+//      streams the W_ih tile and the rows' K slice by TMA, warp 1 issues the MMAs into one
 //      accumulator (rows = gate rows, columns = batch rows), warps 4..11 store the item's partial sums
 //      into its own slot of a global buffer -- plain stores, no atomics.
 //   C  the GRU cell: each (row, unit) adds its partial sums in a fixed order (bit-reproducible),
@@ -23,7 +23,8 @@
 //   D  W_hh . S_i and W1's state block . S_i as one stacked product (3Hs + r rows) against the
 //      split state (K = 2Hs: the weights repeated along K), items and partial slots as in phase B.
 //   E  u_{i+1} = SiLU(P_{i+1} + the W1 partial sums), rounded to bf16 for phase A.
-// The last position runs phase A only.  Before position 0: C0 (the split of S0), D and E.
+// The last position runs phase A only.  Before position 0: C0 (the split of S0), D and E.  With
+// the embedding projection table phases X and B are skipped.
 //
 // Roles keep running counters of the stages, tiles and phases they have gone through, so the
 // mbarriers are initialised once.  Every mbarrier wait and every grid barrier is bounded: a role
@@ -44,8 +45,6 @@ namespace {
 
 constexpr int kThreads = 384;           // 12 warps
 constexpr int kEpiWarps = 8;            // warps 4..11
-constexpr int kLsuThreads = 64;         // warps 2..3 in phase B
-constexpr int kLsuAhead = 3;            // cp.async groups each gathering thread keeps in flight
 constexpr int kTmemCols = 512;
 constexpr uint32_t kBox = 128 * 64 * 2; // one 128 x 64 bf16 box, 128-byte swizzle: 16 KB
 // phase A: W2 ring of kStagesA boxes, L_base ring of kSide tiles (two boxes each)
@@ -61,6 +60,10 @@ static_assert(kStagesG * kStageG <= kRegion, "phase B/D ring");
 constexpr int kUnit = 16;               // vocabulary columns per work unit
 constexpr int kTileUnits = 8;           // units per vocabulary tile (128 columns)
 constexpr int kMaxKs = 8;               // K slices of phases B and D
+constexpr int kTraceArrive = 256;       // first per-CTA arrival stamp of the optional trace
+// then, from kTraceArrive + 128 * G: per CTA, milestones of phases B and D at position 1 --
+// [(phase * 8 + k) * G + c], k: 0 start, 1 producer done, 3 MMAs issued,
+// 4 accumulator in the epilogue, 5 epilogue done
 // Poll limit of the waits for a role's own copies and MMAs at the end of a phase: independent of the
 // caller's spin limit (which may be tiny in a test), so that a role that gave up still lets its
 // copies land before the CTA moves on; the 2-second cap of mbar_wait_bounded bounds it in time.
@@ -75,7 +78,7 @@ enum : int {
   kMmaA = 28, kFullB = 29, kEmptyB = 36, kAccB = 43, kMmaB = 44, kFullD = 45, kEmptyD = 52, kAccD = 59, kMmaD = 60,
   kNumBars = 61
 };
-// misc block: kBarSlots mbarriers, best_s [128] u64, tok_s [128] int, four int flags
+// misc block: kBarSlots mbarriers, best_s [128] u64, 512 spare bytes, four int flags
 constexpr int kBarSlots = 62;
 static_assert(kNumBars <= kBarSlots && kBarSlots * 8 + 128 * 8 + 128 * 4 + 16 <= (int)kMisc, "misc block");
 
@@ -92,6 +95,7 @@ struct BArgs {
   uint64_t* keys;         // [L][B] argmax keys (zero before the launch)
   bf16* u16;              // [B][r] activations of the current position
   bf16* S_hl;             // [B][2Hs] two-term split of the current state
+  bf16* X;                // [B][d] embedding rows of the tokens drafted at the current position
   float* partx;           // [ksx][B][3Hs] phase B partial sums
   float* parth;           // [ksd][B][3Hs + r] phase D partial sums
   uint32_t* claim;        // per-SM work-slot claims (zero before the launch)
@@ -100,8 +104,9 @@ struct BArgs {
   int B, L, d, Hs, r, V;
   int ksx, ksd;           // K slices of phases B and D
   unsigned long long limit;
-  unsigned long long* trace;  // optional: [0] CTA 0's start, [e] when CTA 0 passed grid barrier e,
-  int ntrace;                 // then its end (globaltimer, ns); entries past ntrace are not written
+  unsigned long long* trace;  // optional (globaltimer, ns): [0] CTA 0's start, [e] when CTA 0 passed
+  int ntrace;                 // grid barrier e, then its end; [kTraceArrive + (e-1) * G + c] when
+                              // CTA c arrived at barrier e.  Entries past ntrace are not written.
 };
 
 __device__ __forceinline__ void tma_load_3d_hint(void* smem_dst, const CUtensorMap* tmap, uint64_t* bar, int x, int y,
@@ -137,14 +142,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                      const __grid_constant__ CUtensorMap tmL, const __grid_constant__ CUtensorMap tmU,
                      const __grid_constant__ CUtensorMap tmWih, const __grid_constant__ CUtensorMap tmWhh,
                      const __grid_constant__ CUtensorMap tmW1s, const __grid_constant__ CUtensorMap tmShl,
-                     BArgs p) {
+                     const __grid_constant__ CUtensorMap tmX, BArgs p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   uint8_t* side_ring = ring + (size_t)kStagesA * kBox;
   uint64_t* bars = reinterpret_cast<uint64_t*>(ring + kRegion);
   uint64_t* best_s = bars + kBarSlots;                             // [128]
-  int* tok_s = reinterpret_cast<int*>(best_s + 128);               // [128]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tok_s + 128);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(best_s + 128 + 64);
   volatile int* abort_s = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* slot_s = reinterpret_cast<volatile int*>(tmem_slot + 2);
   volatile int* flag_s = reinterpret_cast<volatile int*>(tmem_slot + 3);
@@ -163,7 +167,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&bars[kUFull], 1);
     mbar_init(&bars[kMmaA], 1);
     for (int s = 0; s < kStagesG; ++s) {
-      mbar_init(&bars[kFullB + s], 1 + kLsuThreads);
+      mbar_init(&bars[kFullB + s], 1);
       mbar_init(&bars[kEmptyB + s], 1);
       mbar_init(&bars[kFullD + s], 1);
       mbar_init(&bars[kEmptyD + s], 1);
@@ -182,6 +186,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tma_prefetch_desc(&tmWhh);
     tma_prefetch_desc(&tmW1s);
     tma_prefetch_desc(&tmShl);
+    tma_prefetch_desc(&tmX);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, kTmemCols);
@@ -214,6 +219,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     if (threadIdx.x == 0) {
       ++epoch;
+      if (p.trace) {
+        const long long k = kTraceArrive + (long long)(epoch - 1) * G + blockIdx.x;
+        if (k < p.ntrace) p.trace[k] = globaltimer_ns();
+      }
       __threadfence();
       atomicAdd(p.bar, 1u);
       const unsigned target = epoch * (unsigned)G;
@@ -466,21 +475,24 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t* empty = &bars[isB ? kEmptyB : kEmptyD];
     uint64_t* accb = &bars[isB ? kAccB : kAccD];
     uint64_t* mmab = &bars[isB ? kMmaB : kMmaD];
-    uint32_t& itG = isB ? itB : itD;
+    const uint32_t it0 = isB ? itB : itD;
     const uint32_t nph = (isB ? nB : nD) & 1u;
-    const uint32_t it0 = itG;
     const int nst = has ? kb1 - kb0 : 0;
     float* part = isB ? p.partx : p.parth;
     const int ldp = isB ? H3 : HD;
-    if (isB && threadIdx.x < 128) {  // tokens of position i (the keys are complete after phase A)
-      const int b = threadIdx.x;
-      int tok = b < B ? key_index(p.keys[(size_t)i * B + b]) : 0;
-      tok_s[b] = (tok >= 0 && tok < V) ? tok : 0;
-    }
-    __syncthreads();
+    const long long det = (p.trace && i == 1) ? kTraceArrive + 128LL * G + (isB ? 0 : 8) * (long long)G : -1;
+    auto mark = [&](int k) {
+      if (det >= 0 && det + (long long)k * G + blockIdx.x < p.ntrace) p.trace[det + (long long)k * G + blockIdx.x] =
+          globaltimer_ns();
+    };
+    if (threadIdx.x == 0) mark(0);
     if (warp == 0) {
       if (lane == 0 && has) {  // TMA producer: the weight tile (and, in phase D, the split state)
         const uint64_t pol = l2_policy_evict_first();
+        // phase B: the W_ih boxes past the ring's depth are requested from memory at once, so that
+        // their loads meet L2 when ring slots free up (the first kStagesG go straight to the ring)
+        if (isB)
+          for (int kb = kb0 + kStagesG; kb < kb1; ++kb) tma_prefetch_l2_hint(&tmWih, kb * 64, mt * 128, pol);
         bool ok = true;
         uint32_t it = it0;
         for (int kb = kb0; kb < kb1; ++kb, ++it) {
@@ -488,8 +500,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!mbar_wait_bounded(&empty[s], ((it / kStagesG) & 1u) ^ 1u, limit, abort_s)) { ok = false; break; }
           uint8_t* st = ring + (size_t)s * kStageG;
           if (isB) {
-            mbar_arrive_expect_tx(&full[s], kBox);
+            mbar_arrive_expect_tx(&full[s], 2 * kBox);
             tma_load_2d_hint(st, &tmWih, &full[s], kb * 64, mt * 128, pol);
+            tma_load_2d(st + kBox, &tmX, &full[s], kb * 64, 0);
           } else {
             mbar_arrive_expect_tx(&full[s], 2 * kBox);
             const int kx = (kb * 64) % Hs;
@@ -499,38 +512,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         if (!ok) *abort_s = 1;
+        mark(1);
         int never = 0;
         for (uint32_t j = (it - it0 > (uint32_t)kStagesG ? it - kStagesG : it0); j < it; ++j)
           mbar_wait_bounded(&full[j % kStagesG], (j / kStagesG) & 1u, kDrain, &never);
-      }
-    } else if (warp == 2 || warp == 3) {
-      if (isB && has) {  // gather: the K slice of each drafted token's embedding row, 16 bytes per copy
-        const int pt = (warp - 2) * 32 + lane;
-        bool ok = true;
-        uint32_t it = it0;
-        int issued = 0;
-        for (int kb = kb0; kb < kb1; ++kb, ++it, ++issued) {
-          const int s = it % kStagesG;
-          if (!mbar_wait_bounded(&empty[s], ((it / kStagesG) & 1u) ^ 1u, limit, abort_s)) { ok = false; break; }
-          uint8_t* dst = ring + (size_t)s * kStageG + kBox;
-          for (int c = pt; c < 128 * 8; c += kLsuThreads) {
-            const int rw = c >> 3, ch = c & 7;
-            const bf16* src = p.embed + (size_t)tok_s[rw] * p.d + kb * 64 + ch * 8;
-            const uint32_t da = smem_u32(dst + rw * 128 + ((ch ^ (rw & 7)) << 4));
-            const uint32_t sz = rw < B ? 16u : 0u;  // rows past the batch land as zeros
-            asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(da), "l"(src), "r"(sz) : "memory");
-          }
-          asm volatile("cp.async.commit_group;" ::: "memory");
-          if (issued >= kLsuAhead) {  // stage it - kLsuAhead has landed
-            asm volatile("cp.async.wait_group %0;" ::"n"(kLsuAhead) : "memory");
-            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-            mbar_arrive(&full[(it - kLsuAhead) % kStagesG]);
-          }
-        }
-        asm volatile("cp.async.wait_group 0;" ::: "memory");
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        for (uint32_t j = (issued > kLsuAhead ? it - kLsuAhead : it0); j < it; ++j) mbar_arrive(&full[j % kStagesG]);
-        if (!ok) *abort_s = 1;
       }
     } else if (warp == 1) {
       if (lane == 0 && has) {  // MMA issuer: one 128 x 128 accumulator at TMEM column 0
@@ -548,36 +533,52 @@ __global__ void __launch_bounds__(kThreads, 1)
           umma_commit(&empty[s]);
         }
         if (!ok) *abort_s = 1;
+        mark(3);
         umma_commit(accb);  // completes when every MMA issued above has finished
         int never = 0;
         umma_commit(mmab);
         mbar_wait_bounded(mmab, nph, kDrain, &never);
       }
-    } else if (warp >= 4 && has) {  // epilogue: partial sums of this item -> part[kq][n][row]
-      const int q = warp & 3, g = (warp - 4) >> 2;
-      const int row = q * 32 + lane;
-      if (mbar_wait_warp(accb, nph, limit, abort_s)) {
-        tmem_fence_after_sync();
-        const uint32_t taddr = tbase + ((uint32_t)(q * 32) << 16) + (uint32_t)(g * 64);
-        uint32_t rr[64];
-        tmem_ld16(taddr, &rr[0]);
-        tmem_ld16(taddr + 16, &rr[16]);
-        tmem_ld16(taddr + 32, &rr[32]);
-        tmem_ld16(taddr + 48, &rr[48]);
-        tmem_wait_ld();
-        float* dst = part + (size_t)kq * B * ldp + (size_t)mt * 128 + row;
+    } else if (has) {  // warps 2..11
+      if (warp >= 4) {  // epilogue: the item's partial sums -> part[kq][n][tile row]
+        const int q = warp & 3, g = (warp - 4) >> 2;
+        const int row = q * 32 + lane;
+        if (mbar_wait_warp(accb, nph, limit, abort_s)) {
+          if (warp == 4 && lane == 0) mark(4);
+          tmem_fence_after_sync();
+          const uint32_t taddr = tbase + ((uint32_t)(q * 32) << 16) + (uint32_t)(g * 64);
+          uint32_t rr[64];
+          tmem_ld16(taddr, &rr[0]);
+          tmem_ld16(taddr + 16, &rr[16]);
+          tmem_ld16(taddr + 32, &rr[32]);
+          tmem_ld16(taddr + 48, &rr[48]);
+          tmem_wait_ld();
+          float* dst = part + (size_t)kq * B * ldp + (size_t)mt * 128 + row;
 #pragma unroll
-        for (int c = 0; c < 64; ++c) {
-          reg_fence(rr[c]);
-          const int n = g * 64 + c;
-          if (n < B) dst[(size_t)n * ldp] = __uint_as_float(rr[c]);
+          for (int c = 0; c < 64; ++c) {
+            reg_fence(rr[c]);
+            const int n = g * 64 + c;
+            if (n < B) dst[(size_t)n * ldp] = __uint_as_float(rr[c]);
+          }
+          if (warp == 4 && lane == 0) mark(5);
+        } else {
+          *abort_s = 1;
         }
-      } else {
-        *abort_s = 1;
       }
     }
-    itG = it0 + (uint32_t)nst;
-    if (isB) ++nB; else ++nD;
+    if (isB) { itB = it0 + (uint32_t)nst; ++nB; } else { itD = it0 + (uint32_t)nst; ++nD; }
+  };
+
+  // ---- phase X: the embedding rows of the tokens drafted at position i into the row buffer ----
+  auto phase_x = [&](int i) {
+    const int q8 = p.d / 8;  // 16-byte chunks per row
+    const size_t gtid = (size_t)blockIdx.x * blockDim.x + threadIdx.x, gstride = (size_t)G * blockDim.x;
+    for (size_t c = gtid; c < (size_t)B * q8; c += gstride) {
+      const int b = (int)(c / q8), q = (int)(c % q8);
+      const int tok = key_index(p.keys[(size_t)i * B + b]);
+      const int tk = (tok >= 0 && tok < V) ? tok : 0;
+      reinterpret_cast<uint4*>(p.X)[c] = ldg16(p.embed + (size_t)tk * p.d + (size_t)q * 8);
+    }
   };
 
   // ---- phase C: the GRU cell of position i (i = -1: the split of S0) ----
@@ -594,20 +595,32 @@ __global__ void __launch_bounds__(kThreads, 1)
       } else {
         const int tok = key_index(p.keys[(size_t)i * B + b]);
         const int tk = (tok >= 0 && tok < V) ? tok : 0;
-        float gi[3], gh[3];
+        // every load of the element is issued before the first add (independent loads, one L2 round
+        // trip); the partial sums are then added in slice order, so the result does not depend on it
+        float xs[3][kMaxKs], hs[3][kMaxKs], bi[3], bh[3];
 #pragma unroll
         for (int gt = 0; gt < 3; ++gt) {
           const int rw = gt * Hs + j;
-          float x = 0.f;
-          if (p.Xp) {
-            x = p.Xp[(size_t)tk * H3 + rw];
-          } else {
-            for (int kq = 0; kq < p.ksx; ++kq) x += p.partx[((size_t)kq * B + b) * H3 + rw];
+#pragma unroll
+          for (int kq = 0; kq < kMaxKs; ++kq)
+            xs[gt][kq] = p.Xp ? (kq == 0 ? p.Xp[(size_t)tk * H3 + rw] : 0.f)
+                              : (kq < p.ksx ? p.partx[((size_t)kq * B + b) * H3 + rw] : 0.f);
+#pragma unroll
+          for (int kd = 0; kd < kMaxKs; ++kd) hs[gt][kd] = kd < p.ksd ? p.parth[((size_t)kd * B + b) * HD + rw] : 0.f;
+          bi[gt] = to_f32(p.b_ih[rw]);
+          bh[gt] = to_f32(p.b_hh[rw]);
+        }
+        float gi[3], gh[3];
+#pragma unroll
+        for (int gt = 0; gt < 3; ++gt) {
+          float x = xs[gt][0], h = hs[gt][0];
+#pragma unroll
+          for (int k = 1; k < kMaxKs; ++k) {
+            x += xs[gt][k];  // slices past ks add zeros: the sum is unchanged
+            h += hs[gt][k];
           }
-          float h = 0.f;
-          for (int kd = 0; kd < p.ksd; ++kd) h += p.parth[((size_t)kd * B + b) * HD + rw];
-          gi[gt] = x + to_f32(p.b_ih[rw]);
-          gh[gt] = h + to_f32(p.b_hh[rw]);
+          gi[gt] = x + bi[gt];
+          gh[gt] = h + bh[gt];
         }
         const float rg = sigmoidf_(gi[0] + gh[0]);
         const float zg = sigmoidf_(gi[1] + gh[1]);
@@ -624,11 +637,36 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   // ---- phase E: activations of position pos ----
   auto phase_e = [&](int pos) {
-    const size_t gtid = (size_t)blockIdx.x * blockDim.x + threadIdx.x, gstride = (size_t)G * blockDim.x;
+    if (warp == 0) {  // meanwhile: the first tiles of the coming phase A into L2 (W2 and L_base)
+      if (lane == 0) {
+        const uint64_t pol = l2_policy_evict_last();
+        for (int t = 0; t < min(ntiles, 2); ++t) {
+          const int ut = vu0 + t * kTileUnits, w = min(kTileUnits, vu1 - ut);
+          const int n0 = ut * kUnit;
+          for (int kb = 0; kb < kbA; ++kb) {
+            if (w == kTileUnits) tma_prefetch_l2_hint(&tmW, kb * 64, n0, pol);
+            else
+              for (int j = 0; j < w; ++j) tma_prefetch_l2_hint(&tmWn, kb * 64, n0 + j * kUnit, pol);
+          }
+          if (t == 0)
+            for (int bx = 0; bx < (w * kUnit + 63) / 64; ++bx)
+              asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(&tmL),
+                           "r"(n0 + bx * 64), "r"(pos), "r"(0)
+                           : "memory");
+        }
+      }
+      return;
+    }
+    const int nt = blockDim.x - 32;
+    const size_t gtid = (size_t)blockIdx.x * nt + (threadIdx.x - 32), gstride = (size_t)G * nt;
     for (size_t t = gtid; t < (size_t)B * r; t += gstride) {
       const int b = (int)(t / r), k = (int)(t % r);
+      float hs[kMaxKs];
+#pragma unroll
+      for (int kd = 0; kd < kMaxKs; ++kd) hs[kd] = kd < p.ksd ? p.parth[((size_t)kd * B + b) * HD + H3 + k] : 0.f;
       float a = p.P[((size_t)b * L + pos) * r + k];
-      for (int kd = 0; kd < p.ksd; ++kd) a += p.parth[((size_t)kd * B + b) * HD + H3 + k];
+#pragma unroll
+      for (int kd = 0; kd < kMaxKs; ++kd) a += hs[kd];
       p.u16[(size_t)b * r + k] = __float2bfloat16_rn(siluf_(a));
     }
   };
@@ -642,6 +680,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     phase_a(i);
     if (i == L - 1) break;
     ok = grid_sync();
+    if (ok && !p.Xp) { phase_x(i); ok = grid_sync(); }
     if (ok && !p.Xp) { phase_g(true, i); ok = grid_sync(); }
     if (ok) { phase_c(i); ok = grid_sync(); }
     if (ok) { phase_g(false, i); ok = grid_sync(); }
@@ -715,7 +754,7 @@ cudaError_t launch_greedy_batched(const Shape& s, const domino_weights_t& w, con
   const int G = sm_count();
   cudaError_t e = ensure_sm_rank(st);
   if (e != cudaSuccess) return e;
-  CUtensorMap tW, tWn, tL, tU, tWih, tWhh, tW1s, tShl;
+  CUtensorMap tW, tWn, tL, tU, tWih, tWhh, tW1s, tShl, tX;
   const bf* W1s = (const bf*)w.W1 + s.d;
   // base logits [B][L][V] as a 3-D tensor (v, position, row): one 128-row box per position
   bool okm = tmap_bf16_tiles(&tW, w.W2, (uint64_t)s.V, (uint64_t)s.r, 128) &&
@@ -725,12 +764,13 @@ cudaError_t launch_greedy_batched(const Shape& s, const domino_weights_t& w, con
              tmap_bf16_tiles(&tWhh, w.W_hh, 3 * (uint64_t)s.Hs, (uint64_t)s.Hs, 128) &&
              tmap_bf16_tiles(&tW1s, W1s, (uint64_t)s.r, (uint64_t)s.Hs, 128, (uint64_t)(s.d + s.Hs)) &&
              tmap_bf16_tiles(&tShl, ws.S_hl, (uint64_t)s.B, 2 * (uint64_t)s.Hs, 128) &&
+             tmap_bf16_tiles(&tX, ws.X, (uint64_t)s.B, (uint64_t)s.d, 128) &&
              tmap_bf16_3d(&tL, base_logits, (uint64_t)s.V, (uint64_t)s.L, (uint64_t)s.B, 128);
   if (!okm) return cudaErrorInvalidValue;
   BArgs a{};
   a.embed = (const bf*)w.embed; a.Xp = w.embed_proj; a.b_ih = (const bf*)w.b_ih; a.b_hh = (const bf*)w.b_hh;
   a.P = ws.P; a.S0 = S0; a.S = ws.S; a.states = states_out; a.logits = logits_out; a.keys = ws.keys;
-  a.u16 = ws.u16; a.S_hl = ws.S_hl; a.partx = ws.part;
+  a.u16 = ws.u16; a.S_hl = ws.S_hl; a.X = ws.X; a.partx = ws.part;
   a.parth = ws.part + (size_t)kMaxKs * s.B * 3 * s.Hs;
   a.claim = ws.claim; a.bar = ws.sync; a.status = status;
   a.B = s.B; a.L = s.L; a.d = s.d; a.Hs = s.Hs; a.r = s.r; a.V = s.V;
@@ -738,7 +778,7 @@ cudaError_t launch_greedy_batched(const Shape& s, const domino_weights_t& w, con
   a.ksd = ks_for((3 * s.Hs + s.r) / 128, 2 * s.Hs / 64, G);
   a.limit = spin;
   debug_trace(&a.trace, &a.ntrace);
-  void* params[] = {&tW, &tWn, &tL, &tU, &tWih, &tWhh, &tW1s, &tShl, &a};
+  void* params[] = {&tW, &tWn, &tL, &tU, &tWih, &tWhh, &tW1s, &tShl, &tX, &a};
   e = cudaLaunchCooperativeKernel((const void*)k_greedy_batched, dim3(G), dim3(kThreads), params, kSmem, st);
   return note_launch(e);
 }

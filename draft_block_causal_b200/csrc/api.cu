@@ -444,8 +444,11 @@ int teacher_forced_impl(const domino_shape_t* shape, const domino_weights_t* w, 
     if (e == cudaSuccess)
       e = launch_tf_recurrence_tmem(s, *w, S0, tokens, gx, SB, ws, st, spin_limit(), persistent_grid(), cs);
   } else {
-  if (e == cudaSuccess) e = launch_copy_rows(S0, s.Hs, SB, row, s.B, s.Hs, cs);
-  if (e == cudaSuccess && tc) e = launch_split_state(S0, s.Hs, s.B, s.Hs, ws.S_hl, cs);
+  // 5..128 rows: the recurrence in one launch of the persistent batched kernel (it writes the
+  // states' first position and the split of S0 itself); otherwise one gh GEMM + cell per update
+  const bool batched = tc && use_greedy_batched(s, *w, base_logits);
+  if (e == cudaSuccess && !batched) e = launch_copy_rows(S0, s.Hs, SB, row, s.B, s.Hs, cs);
+  if (e == cudaSuccess && tc && !batched) e = launch_split_state(S0, s.Hs, s.B, s.Hs, ws.S_hl, cs);
   // The GRU input half for every given token at once (one GEMM over B*(L-1) gathered rows), unless
   // the projection table already holds it.
   const int NX = s.B * (s.L - 1);
@@ -455,7 +458,12 @@ int teacher_forced_impl(const domino_shape_t* shape, const domino_weights_t* w, 
       e = gemm_tc_store_f32_t((const bf*)w->W_ih, ws.X, 3 * s.Hs, NX, s.d, 0, ws.Gx, 3 * s.Hs, st, spin_limit(), cs,
                               1);
   }
-  for (int i = 0; i + 1 < s.L && e == cudaSuccess; ++i) {
+  if (batched) {
+    if (e == cudaSuccess) e = cudaMemsetAsync(ws.sync, 0, kSyncWords * sizeof(uint32_t), cs);
+    if (e == cudaSuccess)
+      e = launch_tf_batched(s, *w, base_logits, S0, tokens, ws.Gx, SB, ws, st, spin_limit(), cs);
+  }
+  for (int i = 0; i + 1 < s.L && e == cudaSuccess && !batched; ++i) {
     if (tc)
       e = gru_step_tc(s, *w, ws, SB + (size_t)i * s.Hs, row, nullptr, tokens, s.L, i, ws.Gx, 3 * s.Hs, s.L - 1, i, false,
                       SB + (size_t)(i + 1) * s.Hs, row, nullptr, 0, st, cs);

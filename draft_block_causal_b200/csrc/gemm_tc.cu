@@ -1055,6 +1055,18 @@ bool tmap_bf16_tiles(CUtensorMap* tm, const void* base, uint64_t rows, uint64_t 
   return tmap_bf16(tm, base, rows, cols, box_rows, ld);
 }
 
+bool tmap_f32_3d(CUtensorMap* tm, void* base, uint64_t n0, uint64_t n1, uint64_t n2, uint32_t box0, uint32_t box1) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn || n0 % 4 != 0) return false;
+  cuuint64_t dims[3] = {n0, n1, n2};
+  cuuint64_t strides[2] = {n0 * 4, n0 * n1 * 4};
+  cuuint32_t box[3] = {box0, box1, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return fn(tm, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, base, dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
 bool tmap_bf16_3d(CUtensorMap* tm, const void* base, uint64_t n0, uint64_t n1, uint64_t n2, uint32_t box2) {
   EncodeTiledFn fn = encode_fn();
   if (!fn || n0 % 8 != 0) return false;

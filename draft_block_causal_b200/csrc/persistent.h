@@ -47,5 +47,12 @@ size_t batched_partial_floats(const Shape& s);
 cudaError_t launch_greedy_batched(const Shape& s, const domino_weights_t& w, const void* base_logits,
                                   const float* S0, float* logits_out, float* states_out, const Workspace& ws,
                                   int32_t* status, uint64_t spin, cudaStream_t st);
+// Its teacher-forced recurrence: states [B][L][Hs] (states[b][0] = S0) for the given tokens [B][L];
+// Gx: [B * (L - 1)][3Hs] fp32 W_ih . embed[y_i] (row b * (L - 1) + i), unless the weights carry the
+// projection table.  Out-of-range tokens set DOMINO_STATUS_BAD_TOKEN and read token 0.  The caller
+// zeroes ws.sync and ws.claim first.
+cudaError_t launch_tf_batched(const Shape& s, const domino_weights_t& w, const void* base_logits, const float* S0,
+                              const int32_t* tokens, const float* Gx, float* states, const Workspace& ws,
+                              int32_t* status, uint64_t spin, cudaStream_t st);
 
 }  // namespace domino

@@ -26,6 +26,11 @@
 // The last position runs phase A only.  Before position 0: C0 (the split of S0), D and E.  With
 // the embedding projection table phases X and B are skipped.
 //
+// Teacher forcing (given tokens) runs the recurrence only: C0, then per update D (W_hh . S, the
+// 3Hs gate rows alone) and C (the cell, with the gate inputs precomputed for every given token or
+// read from the projection table); the caller computes the activations and logits of all positions
+// afterwards in two tensor-core GEMMs.
+//
 // Roles keep running counters of the stages, tiles and phases they have gone through, so the
 // mbarriers are initialised once.  Every mbarrier wait and every grid barrier is bounded: a role
 // that gives up raises the CTA's abort flag, waits (bounded) for its copies and MMAs in flight, and
@@ -98,12 +103,17 @@ struct BArgs {
   bf16* X;                // [B][d] embedding rows of the tokens drafted at the current position
   float* partx;           // [ksx][B][3Hs] phase B partial sums
   float* parth;           // [ksd][B][3Hs + r] phase D partial sums
-  uint32_t* claim;        // per-SM work-slot claims (zero before the launch)
+  uint32_t* claim;        // per-SM work-slot claims, all different from epoch before the launch
+  uint32_t epoch;
   unsigned* bar;          // grid barrier counter (zero before the launch)
   int32_t* status;
   int B, L, d, Hs, r, V;
   int ksx, ksd;           // K slices of phases B and D
   unsigned long long limit;
+  // teacher forcing: the given tokens [B][L] and, unless the projection table is given, their gate
+  // inputs W_ih . embed[y] as rows b * (L - 1) + i of Gx [B * (L - 1)][3Hs]; null in greedy drafting
+  const int32_t* tokens;
+  const float* Gx;
   unsigned long long* trace;  // optional (globaltimer, ns): [0] CTA 0's start, [e] when CTA 0 passed
   int ntrace;                 // grid barrier e, then its end; [kTraceArrive + (e-1) * G + c] when
                               // CTA c arrived at barrier e.  Entries past ntrace are not written.
@@ -142,7 +152,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                      const __grid_constant__ CUtensorMap tmL, const __grid_constant__ CUtensorMap tmU,
                      const __grid_constant__ CUtensorMap tmWih, const __grid_constant__ CUtensorMap tmWhh,
                      const __grid_constant__ CUtensorMap tmW1s, const __grid_constant__ CUtensorMap tmShl,
-                     const __grid_constant__ CUtensorMap tmX, BArgs p) {
+                     const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmPx,
+                     const __grid_constant__ CUtensorMap tmPh, BArgs p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   uint8_t* side_ring = ring + (size_t)kStagesA * kBox;
@@ -159,7 +170,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const unsigned long long limit = p.limit;
 
   if (threadIdx.x == 0) {
-    *slot_s = claim_slot(p.claim, 1u);
+    *slot_s = claim_slot(p.claim, p.epoch);
     for (int s = 0; s < kStagesA; ++s) { mbar_init(&bars[kFullA + s], 1); mbar_init(&bars[kEmptyA + s], 1); }
     for (int s = 0; s < kSide; ++s) { mbar_init(&bars[kSFull + s], 1); mbar_init(&bars[kSEmpty + s], kEpiWarps); }
     for (int a = 0; a < 2; ++a) { mbar_init(&bars[kAccFA + a], 1); mbar_init(&bars[kAccEA + a], kEpiWarps); }
@@ -187,6 +198,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     tma_prefetch_desc(&tmW1s);
     tma_prefetch_desc(&tmShl);
     tma_prefetch_desc(&tmX);
+    tma_prefetch_desc(&tmPx);
+    tma_prefetch_desc(&tmPh);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, kTmemCols);
@@ -464,7 +477,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // isB: A = W_ih (rows [mt*128, +128), columns = k), B = the embedding rows of the drafted tokens;
   // else A = [W_hh ; W1 state block] (k wraps at Hs), B = the split state S_hl.
   auto phase_g = [&](bool isB, int i) {
-    const int ntile = isB ? H3 / 128 : HD / 128;
+    const int ntile = (isB || p.tokens) ? H3 / 128 : HD / 128;
     const int ks = isB ? p.ksx : p.ksd;
     const int KB = isB ? p.d / 64 : 2 * Hs / 64;
     const int item = blockIdx.x;
@@ -478,8 +491,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t it0 = isB ? itB : itD;
     const uint32_t nph = (isB ? nB : nD) & 1u;
     const int nst = has ? kb1 - kb0 : 0;
-    float* part = isB ? p.partx : p.parth;
-    const int ldp = isB ? H3 : HD;
     const long long det = (p.trace && i == 1) ? kTraceArrive + 128LL * G + (isB ? 0 : 8) * (long long)G : -1;
     auto mark = [&](int k) {
       if (det >= 0 && det + (long long)k * G + blockIdx.x < p.ntrace) p.trace[det + (long long)k * G + blockIdx.x] =
@@ -540,10 +551,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_wait_bounded(mmab, nph, kDrain, &never);
       }
     } else if (has) {  // warps 2..11
-      if (warp >= 4) {  // epilogue: the item's partial sums -> part[kq][n][tile row]
+      if (warp >= 4) {  // epilogue: the item's partial sums -> part[kq][n][tile row], by one TMA store
         const int q = warp & 3, g = (warp - 4) >> 2;
         const int row = q * 32 + lane;
-        if (mbar_wait_warp(accb, nph, limit, abort_s)) {
+        const bool got = mbar_wait_warp(accb, nph, limit, abort_s);
+        if (got) {
           if (warp == 4 && lane == 0) mark(4);
           tmem_fence_after_sync();
           const uint32_t taddr = tbase + ((uint32_t)(q * 32) << 16) + (uint32_t)(g * 64);
@@ -553,16 +565,30 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_ld16(taddr + 32, &rr[32]);
           tmem_ld16(taddr + 48, &rr[48]);
           tmem_wait_ld();
-          float* dst = part + (size_t)kq * B * ldp + (size_t)mt * 128 + row;
+          // the MMAs are done, so the ring is free: stage the tile there as [batch row][gate row]
+          // (a warp writes 32 consecutive floats per store: no bank conflict)
+          float* stg = reinterpret_cast<float*>(ring);
 #pragma unroll
           for (int c = 0; c < 64; ++c) {
             reg_fence(rr[c]);
-            const int n = g * 64 + c;
-            if (n < B) dst[(size_t)n * ldp] = __uint_as_float(rr[c]);
+            stg[(g * 64 + c) * 128 + row] = __uint_as_float(rr[c]);
           }
-          if (warp == 4 && lane == 0) mark(5);
         } else {
           *abort_s = 1;
+        }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        asm volatile("bar.sync 1, %0;" ::"r"(kEpiWarps * 32) : "memory");
+        if (warp == 4 && lane == 0) {
+          if (got) {  // rows past B fall outside the tensor and are not written
+            asm volatile(
+                "cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%1, %2, %3}], [%4];" ::"l"(
+                    isB ? &tmPx : &tmPh),
+                "r"(mt * 128), "r"(0), "r"(kq), "r"(smem_u32(ring))
+                : "memory");
+            asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+            asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");  // written before the barrier
+          }
+          mark(5);
         }
       }
     }
@@ -593,8 +619,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         hn = p.S0[t];
         if (p.states) p.states[(size_t)b * L * Hs + j] = hn;
       } else {
-        const int tok = key_index(p.keys[(size_t)i * B + b]);
-        const int tk = (tok >= 0 && tok < V) ? tok : 0;
+        const int tok = p.tokens ? p.tokens[(size_t)b * L + i] : key_index(p.keys[(size_t)i * B + b]);
+        const bool valid = tok >= 0 && tok < V;
+        if (!valid && j == 0) set_status(p.status, DOMINO_STATUS_BAD_TOKEN);
+        const int tk = valid ? tok : 0;
         // every load of the element is issued before the first add (independent loads, one L2 round
         // trip); the partial sums are then added in slice order, so the result does not depend on it
         float xs[3][kMaxKs], hs[3][kMaxKs], bi[3], bh[3];
@@ -603,8 +631,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int rw = gt * Hs + j;
 #pragma unroll
           for (int kq = 0; kq < kMaxKs; ++kq)
-            xs[gt][kq] = p.Xp ? (kq == 0 ? p.Xp[(size_t)tk * H3 + rw] : 0.f)
-                              : (kq < p.ksx ? p.partx[((size_t)kq * B + b) * H3 + rw] : 0.f);
+            xs[gt][kq] = p.Xp     ? (kq == 0 ? p.Xp[(size_t)tk * H3 + rw] : 0.f)
+                         : p.Gx   ? (kq == 0 ? p.Gx[((size_t)b * (L - 1) + i) * H3 + rw] : 0.f)
+                                  : (kq < p.ksx ? p.partx[((size_t)kq * B + b) * H3 + rw] : 0.f);
 #pragma unroll
           for (int kd = 0; kd < kMaxKs; ++kd) hs[gt][kd] = kd < p.ksd ? p.parth[((size_t)kd * B + b) * HD + rw] : 0.f;
           bi[gt] = to_f32(p.b_ih[rw]);
@@ -637,28 +666,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   // ---- phase E: activations of position pos ----
   auto phase_e = [&](int pos) {
-    if (warp == 0) {  // meanwhile: the first tiles of the coming phase A into L2 (W2 and L_base)
-      if (lane == 0) {
-        const uint64_t pol = l2_policy_evict_last();
-        for (int t = 0; t < min(ntiles, 2); ++t) {
-          const int ut = vu0 + t * kTileUnits, w = min(kTileUnits, vu1 - ut);
-          const int n0 = ut * kUnit;
-          for (int kb = 0; kb < kbA; ++kb) {
-            if (w == kTileUnits) tma_prefetch_l2_hint(&tmW, kb * 64, n0, pol);
-            else
-              for (int j = 0; j < w; ++j) tma_prefetch_l2_hint(&tmWn, kb * 64, n0 + j * kUnit, pol);
-          }
-          if (t == 0)
-            for (int bx = 0; bx < (w * kUnit + 63) / 64; ++bx)
-              asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(&tmL),
-                           "r"(n0 + bx * 64), "r"(pos), "r"(0)
-                           : "memory");
-        }
-      }
-      return;
-    }
-    const int nt = blockDim.x - 32;
-    const size_t gtid = (size_t)blockIdx.x * nt + (threadIdx.x - 32), gstride = (size_t)G * nt;
+    const size_t gtid = (size_t)blockIdx.x * blockDim.x + threadIdx.x, gstride = (size_t)G * blockDim.x;
     for (size_t t = gtid; t < (size_t)B * r; t += gstride) {
       const int b = (int)(t / r), k = (int)(t % r);
       float hs[kMaxKs];
@@ -672,6 +680,22 @@ __global__ void __launch_bounds__(kThreads, 1)
   };
 
   bool ok = true;
+  if (p.tokens) {  // teacher forcing: the recurrence over the given tokens
+    phase_c(-1);
+    for (int i = 0; i + 1 < L; ++i) {
+      if (!(ok = grid_sync())) break;
+      phase_g(false, i);
+      if (!(ok = grid_sync())) break;
+      phase_c(i);
+    }
+    tmem_fence_before_sync();
+    __syncthreads();
+    tmem_fence_after_sync();
+    if (warp == 1) tmem_dealloc(tbase, kTmemCols);
+    if (threadIdx.x == 0 && *abort_s) set_status(p.status, DOMINO_STATUS_DEVICE_TIMEOUT);
+    if (tracer && (int)epoch + 1 < p.ntrace) p.trace[epoch + 1] = globaltimer_ns();
+    return;
+  }
   phase_c(-1);
   ok = grid_sync();
   if (ok) { phase_g(false, 0); ok = grid_sync(); }
@@ -747,14 +771,35 @@ const char* batched_plan() {
          "grid barriers";
 }
 
+namespace {
+cudaError_t launch_batched(const Shape& s, const domino_weights_t& w, const void* base_logits, const float* S0,
+                           float* logits_out, float* states_out, const int32_t* tokens, const float* Gx,
+                           const Workspace& ws, int32_t* status, uint64_t spin, cudaStream_t st);
+}  // namespace
+
 cudaError_t launch_greedy_batched(const Shape& s, const domino_weights_t& w, const void* base_logits,
                                   const float* S0, float* logits_out, float* states_out, const Workspace& ws,
                                   int32_t* status, uint64_t spin, cudaStream_t st) {
+  return launch_batched(s, w, base_logits, S0, logits_out, states_out, nullptr, nullptr, ws, status, spin, st);
+}
+
+cudaError_t launch_tf_batched(const Shape& s, const domino_weights_t& w, const void* base_logits, const float* S0,
+                              const int32_t* tokens, const float* Gx, float* states, const Workspace& ws,
+                              int32_t* status, uint64_t spin, cudaStream_t st) {
+  if (!tokens || !states || (!Gx && !w.embed_proj && s.L > 1)) return cudaErrorInvalidValue;
+  return launch_batched(s, w, base_logits, S0, nullptr, states, tokens, w.embed_proj ? nullptr : Gx, ws, status,
+                        spin, st);
+}
+
+namespace {
+cudaError_t launch_batched(const Shape& s, const domino_weights_t& w, const void* base_logits, const float* S0,
+                           float* logits_out, float* states_out, const int32_t* tokens, const float* Gx,
+                           const Workspace& ws, int32_t* status, uint64_t spin, cudaStream_t st) {
   using bf = __nv_bfloat16;
   const int G = sm_count();
   cudaError_t e = ensure_sm_rank(st);
   if (e != cudaSuccess) return e;
-  CUtensorMap tW, tWn, tL, tU, tWih, tWhh, tW1s, tShl, tX;
+  CUtensorMap tW, tWn, tL, tU, tWih, tWhh, tW1s, tShl, tX, tPx, tPh;
   const bf* W1s = (const bf*)w.W1 + s.d;
   // base logits [B][L][V] as a 3-D tensor (v, position, row): one 128-row box per position
   bool okm = tmap_bf16_tiles(&tW, w.W2, (uint64_t)s.V, (uint64_t)s.r, 128) &&
@@ -765,6 +810,9 @@ cudaError_t launch_greedy_batched(const Shape& s, const domino_weights_t& w, con
              tmap_bf16_tiles(&tW1s, W1s, (uint64_t)s.r, (uint64_t)s.Hs, 128, (uint64_t)(s.d + s.Hs)) &&
              tmap_bf16_tiles(&tShl, ws.S_hl, (uint64_t)s.B, 2 * (uint64_t)s.Hs, 128) &&
              tmap_bf16_tiles(&tX, ws.X, (uint64_t)s.B, (uint64_t)s.d, 128) &&
+             tmap_f32_3d(&tPx, ws.part, 3 * (uint64_t)s.Hs, (uint64_t)s.B, kMaxKs, 128, 128) &&
+             tmap_f32_3d(&tPh, ws.part + (size_t)kMaxKs * s.B * 3 * s.Hs, 3 * (uint64_t)s.Hs + s.r, (uint64_t)s.B,
+                         kMaxKs, 128, 128) &&
              tmap_bf16_3d(&tL, base_logits, (uint64_t)s.V, (uint64_t)s.L, (uint64_t)s.B, 128);
   if (!okm) return cudaErrorInvalidValue;
   BArgs a{};
@@ -775,12 +823,18 @@ cudaError_t launch_greedy_batched(const Shape& s, const domino_weights_t& w, con
   a.claim = ws.claim; a.bar = ws.sync; a.status = status;
   a.B = s.B; a.L = s.L; a.d = s.d; a.Hs = s.Hs; a.r = s.r; a.V = s.V;
   a.ksx = ks_for(3 * s.Hs / 128, s.d / 64, G);
-  a.ksd = ks_for((3 * s.Hs + s.r) / 128, 2 * s.Hs / 64, G);
+  a.ksd = tokens ? ks_for(3 * s.Hs / 128, 2 * s.Hs / 64, G) : ks_for((3 * s.Hs + s.r) / 128, 2 * s.Hs / 64, G);
+  a.tokens = tokens;
+  a.Gx = Gx;
+  // greedy drafting claims against words zeroed just before; teacher forcing against the words its
+  // logits GEMM (epoch 1) will claim after it, so it takes epoch 2
+  a.epoch = tokens ? 2u : 1u;
   a.limit = spin;
   debug_trace(&a.trace, &a.ntrace);
-  void* params[] = {&tW, &tWn, &tL, &tU, &tWih, &tWhh, &tW1s, &tShl, &tX, &a};
+  void* params[] = {&tW, &tWn, &tL, &tU, &tWih, &tWhh, &tW1s, &tShl, &tX, &tPx, &tPh, &a};
   e = cudaLaunchCooperativeKernel((const void*)k_greedy_batched, dim3(G), dim3(kThreads), params, kSmem, st);
   return note_launch(e);
 }
+}  // namespace
 
 }  // namespace domino

@@ -23,8 +23,15 @@ def _small(B=2, L=6, dtype=1, seed=200):
     return synth.make_workload(wl, with_tokens=True)
 
 
-def test_bad_teacher_forcing_token_sets_status():
-    data = _small()
+@pytest.mark.parametrize("shape", ["per-phase", "batched"])
+def test_bad_teacher_forcing_token_sets_status(shape):
+    if shape == "per-phase":
+        data = _small()
+    else:  # the persistent batched kernel's recurrence (5 <= B <= 128, Hs a multiple of 128)
+        data = synth.make_workload(dict(B=8, L=6, d=256, Hs=128, r=128, V=2000, dtype=1, weight_seed=260,
+                                        input_seed=261, s0_std=0.2, peak=2.0, name="bad-token"), with_tokens=True)
+        w, _, _, _ = G.device_inputs(data)
+        assert "k_greedy_batched" in domino.greedy_plan(domino.make_shape(w, 8, 6))
     w, lb, h, S0 = G.device_inputs(data)
     y = torch.from_numpy(data["tokens"]).cuda()
     y[1, 2] = 5000  # V = 2000
@@ -58,10 +65,15 @@ def test_calls_are_asynchronous_and_ordered_on_the_callers_stream():
     s = torch.cuda.Stream()
     lb2 = torch.zeros_like(lb)
     with torch.cuda.stream(s):
+        # outputs and workspace allocated up front: a first allocation on a new stream may wait for
+        # the device inside the caching allocator, which is not the library's call
+        tok_out = torch.empty_like(ref_tok)
+        ws = domino.alloc_workspace(domino.workspace_bytes(w, 4, 8))
+        torch.cuda.synchronize()
         torch.cuda._sleep(200_000_000)  # ~0.1 s of GPU time on this stream
         lb2.copy_(lb)                   # the inputs only become valid after the sleep
         t0 = time.perf_counter()
-        tok, _, _ = domino.draft_greedy(w, lb2, h, S0, stream=s)
+        tok, _, _ = domino.draft_greedy(w, lb2, h, S0, tokens_out=tok_out, workspace=ws, stream=s)
         host_s = time.perf_counter() - t0
     s.synchronize()
     assert host_s < 0.05, f"call blocked the host for {host_s:.3f} s"

@@ -796,13 +796,14 @@ def run_ours(args):
     return result
 
 
-def profile_driver_tf(n: int, batch: int = 1):
+def profile_driver_tf(n: int, batch: int = 1, workload: str = ""):
     """A short, fixed sequence of teacher-forced calls (uniform given tokens, logits out) for an
     external profiler."""
     import torch
     torch.cuda.set_device(0)
     device = torch.device("cuda", 0)
-    wl = synth.workload(HEADLINE) if batch == 1 else synth.workload("qwen3-8b-head-sweep", B=batch)
+    wl = (synth.workload(workload) if workload else
+          synth.workload(HEADLINE) if batch == 1 else synth.workload("qwen3-8b-head-sweep", B=batch))
     pt = Point(wl, device, with_target=False)
     stream = torch.cuda.current_stream()
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
@@ -837,14 +838,15 @@ def profile_driver_accept(n: int, batch: int = 1):
     assert int(pt.status.item()) == 0
 
 
-def profile_driver(n: int, batch: int = 1, trace: bool = False, proj: bool = False):
+def profile_driver(n: int, batch: int = 1, trace: bool = False, proj: bool = False, workload: str = ""):
     """A short, fixed sequence of greedy calls for an external profiler (ncu -k ... -s ... -c ...).
     With `trace`, the last call records the fused kernel's phase clock stamps (CTA 0) and the
     per-phase totals are printed as one JSON line."""
     import torch
     torch.cuda.set_device(0)
     device = torch.device("cuda", 0)
-    wl = synth.workload(HEADLINE) if batch == 1 else synth.workload("qwen3-8b-head-sweep", B=batch)
+    wl = (synth.workload(workload) if workload else
+          synth.workload(HEADLINE) if batch == 1 else synth.workload("qwen3-8b-head-sweep", B=batch))
     pt = Point(wl, device, proj=proj, with_target=False)
     stream = torch.cuda.current_stream()
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
@@ -941,6 +943,8 @@ def main():
     ap.add_argument("--trace", action="store_true", help="profiling driver: print the fused kernel's phase times")
     ap.add_argument("--proj", action="store_true", help="profiling driver: use the embedding projection table")
     ap.add_argument("--profile-tf", action="store_true", help="profiling driver: teacher-forced calls instead")
+    ap.add_argument("--profile-workload", default="", metavar="NAME",
+                    help="profiling driver: a named synthetic workload instead of the batch-selected one")
     ap.add_argument("--profile-accept", action="store_true",
                     help="profiling driver: accept-length and sampled-verification calls instead")
     args = ap.parse_args()
@@ -948,10 +952,11 @@ def main():
         profile_driver_accept(args.profile, batch=args.profile_batch)
         return
     if args.profile and args.profile_tf:
-        profile_driver_tf(args.profile, batch=args.profile_batch)
+        profile_driver_tf(args.profile, batch=args.profile_batch, workload=args.profile_workload)
         return
     if args.profile:
-        profile_driver(args.profile, batch=args.profile_batch, trace=args.trace, proj=args.proj)
+        profile_driver(args.profile, batch=args.profile_batch, trace=args.trace, proj=args.proj,
+                       workload=args.profile_workload)
         return
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3

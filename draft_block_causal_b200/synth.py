@@ -56,6 +56,10 @@ WORKLOADS = {
     # Qwen3-4B-shaped head, the same batch sweep
     "qwen3-4b-head-sweep": dict(B=1, L=16, d=2560, Hs=1024, r=256, V=151936, dtype=BF16,
                                 weight_seed=0, input_seed=5, s0_std=0.1, peak=4.0),
+    # a narrower head (d = 512, Hs = 256) over the full vocabulary, two rows: the GRU rows do not fill
+    # TMEM's layout, so the fused kernel streams them from L2 (profiling of that variant)
+    "narrow-head-b2": dict(B=2, L=16, d=512, Hs=256, r=256, V=151936, dtype=BF16,
+                           weight_seed=0, input_seed=6, s0_std=0.1, peak=4.0),
 }
 SWEEP_BATCHES = (1, 4, 16, 64, 128, 256)
 SWEEP_PEAKS = (1.0, 2.0, 4.0)

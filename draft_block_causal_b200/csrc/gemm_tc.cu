@@ -599,8 +599,8 @@ __global__ void __launch_bounds__(EpiWarps<Epi>::kThreads, 1)
       // no copy may be in flight when the CTA exits: wait for the last S issued stages (and A)
       int never = 0;
       for (uint32_t j = (it > (uint32_t)S ? it - S : 0u); j < it; ++j)
-        mbar_wait_bounded(&full[j % S], (j / S) & 1u, limit, &never);
-      if constexpr (Epi::kARes) mbar_wait_bounded(a_full, 0u, limit, &never);
+        mbar_wait_bounded(&full[j % S], (j / S) & 1u, kDrainPolls, &never);
+      if constexpr (Epi::kARes) mbar_wait_bounded(a_full, 0u, kDrainPolls, &never);
     }
   } else if (warp == 1) {
     if (lane == 0) {  // ---- MMA issuer ----
@@ -642,7 +642,7 @@ __global__ void __launch_bounds__(EpiWarps<Epi>::kThreads, 1)
       // TMEM may only be freed once every issued MMA has finished
       int never = 0;
       umma_commit(mma_done);
-      mbar_wait_bounded(mma_done, 0u, limit, &never);
+      mbar_wait_bounded(mma_done, 0u, kDrainPolls, &never);
     }
   } else {  // ---- epilogue: warps 2 .. 2 + 4 * kGroups - 1 ----
     pdl_wait();
@@ -772,7 +772,7 @@ __global__ void __launch_bounds__(EpiWarps<Epi>::kThreads, 1)
     if (Epi::kSide && side_issuer) {
       int never = 0;
       for (uint32_t k = (side_issued > 2u ? side_issued - 2u : 0u); k < side_issued; ++k)
-        mbar_wait_bounded(&sidef[k & 1u], (k >> 1) & 1u, limit, &never);
+        mbar_wait_bounded(&sidef[k & 1u], (k >> 1) & 1u, kDrainPolls, &never);
     }
   }
 

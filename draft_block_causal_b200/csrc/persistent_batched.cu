@@ -69,10 +69,8 @@ constexpr int kTraceArrive = 256;       // first per-CTA arrival stamp of the op
 // then, from kTraceArrive + 128 * G: per CTA, milestones of phases B and D at position 1 --
 // [(phase * 8 + k) * G + c], k: 0 start, 1 producer done, 3 MMAs issued,
 // 4 accumulator in the epilogue, 5 epilogue done
-// Poll limit of the waits for a role's own copies and MMAs at the end of a phase: independent of the
-// caller's spin limit (which may be tiny in a test), so that a role that gave up still lets its
-// copies land before the CTA moves on; the 2-second cap of mbar_wait_bounded bounds it in time.
-constexpr unsigned long long kDrain = 1ull << 26;
+// Poll limit of the waits for a role's own copies and MMAs at the end of a phase (umma.cuh).
+constexpr unsigned long long kDrain = kDrainPolls;
 constexpr size_t kMisc = 2048;          // mbarriers, the cross-group argmax, tokens, flags
 constexpr size_t kSmem = kRegion + kMisc + 1024;
 static_assert(kSmem <= 232448, "shared memory budget");

@@ -53,6 +53,12 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
   return false;
 }
 
+// Poll limit of the waits with which a role lets its own copies land and its MMAs finish before
+// the CTA moves on or exits.  Independent of the caller's spin limit (which a test may set to one
+// poll): a role that gave up waiting for others must still drain what it issued.  The two-second
+// cap of mbar_wait_bounded bounds it in time.
+constexpr unsigned long long kDrainPolls = 1ull << 26;
+
 // Warp-uniform bounded wait: every lane polls, and the warp succeeds only if every lane did.
 __device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, uint64_t limit, volatile int* abort) {
   const bool ok = mbar_wait_bounded(bar, parity, limit, abort);

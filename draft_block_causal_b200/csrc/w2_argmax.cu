@@ -175,7 +175,7 @@ __global__ void __launch_bounds__(kW2Threads, 1)
       if (!ok) *abort_s = 1;
       int never = 0;  // no copy may be in flight when the CTA exits
       for (uint32_t j = (it > (uint32_t)kStages ? it - kStages : 0u); j < it; ++j)
-        mbar_wait_bounded(&full[j % kStages], (j / kStages) & 1u, limit, &never);
+        mbar_wait_bounded(&full[j % kStages], (j / kStages) & 1u, kDrainPolls, &never);
     }
   } else if (warp == 2) {
     if (lane == 0) {  // ---- L_base producer (an input of the call: no wait either) ----
@@ -196,7 +196,7 @@ __global__ void __launch_bounds__(kW2Threads, 1)
       }
       tstamp(p.trace, 10, globaltimer_ns());
       int never = 0;
-      for (int j = max(0, t - kSide); j < t; ++j) mbar_wait_bounded(&sfull[j % kSide], (j / kSide) & 1, limit, &never);
+      for (int j = max(0, t - kSide); j < t; ++j) mbar_wait_bounded(&sfull[j % kSide], (j / kSide) & 1, kDrainPolls, &never);
     }
   } else if (warp == 1) {
     if (lane == 0) {  // ---- MMA issuer ----
@@ -231,7 +231,7 @@ __global__ void __launch_bounds__(kW2Threads, 1)
       if (!ok) *abort_s = 1;
       int never = 0;  // TMEM may be freed only once every issued MMA has finished
       umma_commit(mma_done);
-      mbar_wait_bounded(mma_done, 0u, limit, &never);
+      mbar_wait_bounded(mma_done, 0u, kDrainPolls, &never);
     }
   } else if (warp >= 4) {  // ---- epilogue ----
     const int q = warp & 3, g = (warp - 4) >> 2;
@@ -356,7 +356,7 @@ __global__ void __launch_bounds__(kW2Threads, 1)
 
   if (warp == 4 && lane == 0) {  // no u copy may be in flight when the CTA exits (a timed-out wait)
     int never = 0;
-    mbar_wait_bounded(u_full, 0u, limit, &never);
+    mbar_wait_bounded(u_full, 0u, kDrainPolls, &never);
   }
   tmem_fence_before_sync();
   __syncthreads();

@@ -116,13 +116,16 @@ def test_plan_names_the_kernel_of_each_batch_size():
     assert "k_greedy_tmem" in domino.greedy_plan(domino.make_shape(w, 2, 16))
 
 
-@pytest.mark.parametrize("Hs", [256, 512], ids=["l2-streamed", "tmem-resident"])
-def test_bounded_barrier_gives_up_with_status_and_the_context_survives(Hs):
-    """A spin limit of one poll makes the grid barriers give up at once: the kernel must report
-    DOMINO_STATUS_DEVICE_TIMEOUT and return (the TMEM variant freeing its tensor memory first);
-    the next call with the default limit is correct."""
-    data = _persistent_case(B=2, Hs=Hs)
+@pytest.mark.parametrize("B,Hs,plan", [(2, 256, "k_greedy_persistent"), (2, 512, "k_greedy_tmem"),
+                                       (8, 128, "k_greedy_batched")],
+                         ids=["l2-streamed", "tmem-resident", "batched"])
+def test_bounded_barrier_gives_up_with_status_and_the_context_survives(B, Hs, plan):
+    """A spin limit of one poll makes the waits give up at once: the kernels must report
+    DOMINO_STATUS_DEVICE_TIMEOUT and return (letting their own copies and MMAs finish and freeing
+    their tensor memory first); the next call with the default limit is correct."""
+    data = _persistent_case(B=B, Hs=Hs)
     w, lb, h, S0 = G.device_inputs(data)
+    assert plan in domino.greedy_plan(domino.make_shape(w, B, 16))
     good, _, _ = domino.draft_greedy(w, lb, h, S0)
     torch.cuda.synchronize()
     status = torch.zeros(1, dtype=torch.int32, device="cuda")

@@ -14,8 +14,9 @@
 //   X  every thread copies a share of the embedding rows of the drafted tokens into a row buffer.
 //   B  gate inputs W_ih . x.  Item = (128-row tile of W_ih, K slice): one item per CTA.  Warp 0
 //      streams the W_ih tile and the rows' K slice by TMA, warp 1 issues the MMAs into one
-//      accumulator (rows = gate rows, columns = batch rows), warps 4..11 store the item's partial sums
-//      into its own slot of a global buffer -- plain stores, no atomics.
+//      accumulator (rows = gate rows, columns = batch rows), warps 4..11 stage the item's partial
+//      sums in shared memory and one TMA store writes them into the item's own slot of a global
+//      buffer -- no atomics.
 //   C  the GRU cell: each (row, unit) adds its partial sums in a fixed order (bit-reproducible),
 //      applies the gates and writes S_i, its two-term bf16 split (hi, lo) for phase D and, when
 //      asked, the states output.  With the embedding projection table phase B is skipped and the

@@ -182,6 +182,27 @@ const char* domino_greedy_plan(const domino_shape_t* shape) {
   return "per-phase kernels: k_hproj, then per position k_u + k_w2 (fused argmax) + k_gru, then k_tokens";
 }
 
+const char* domino_teacher_forced_plan(const domino_shape_t* shape) {
+  if (check_shape(shape) != DOMINO_OK) return "invalid shape";
+  const Shape s = to_shape(shape);
+  const bool tc = s.dtype == DOMINO_DTYPE_BF16 && s.d % 64 == 0 && s.r % 64 == 0 && s.Hs % 64 == 0;
+  if (tc && use_persistent_greedy(s) && tmem_plan_fits(s, persistent_grid(), true) &&
+      (s.L > 1 || tmem_plan_fits(s, persistent_grid(), false)))
+    return "embedding gather + tcgen05 W_ih GEMM over all given tokens, k_greedy_tmem in teacher-forced mode (the "
+           "recurrence), then tcgen05 GEMMs for the activations and the logits of all positions";
+  if (tc && batched_shape_ok(s))
+    return tf_units_ok(s) ? "embedding gather + tcgen05 W_ih GEMM over all given tokens, k_tf_units (the recurrence: "
+                            "each CTA owns eight state units, one grid barrier per update), then tcgen05 GEMMs for the "
+                            "activations and the logits of all positions"
+                          : "embedding gather + tcgen05 W_ih GEMM over all given tokens, k_greedy_batched in "
+                            "teacher-forced mode (the recurrence), then tcgen05 GEMMs for the activations and the "
+                            "logits of all positions";
+  if (tc)
+    return "embedding gather + tcgen05 W_ih GEMM over all given tokens, per update a tcgen05 gh GEMM + k_cell, then "
+           "tcgen05 GEMMs for the activations and the logits of all positions";
+  return "CUDA-core kernels: k_hproj, k_gru per update, then k_u + k_w2 for the logits";
+}
+
 int domino_debug_gemm(const void* A, const void* Bm, int32_t M, int32_t N, int32_t K, int32_t a_kwrap, float* out,
                       int64_t ldo, int32_t trans, int32_t bn, int32_t ks, int32_t* status_dev,
                       domino_stream_t stream) {
@@ -461,7 +482,8 @@ int teacher_forced_impl(const domino_shape_t* shape, const domino_weights_t* w, 
   if (batched) {
     if (e == cudaSuccess) e = cudaMemsetAsync(ws.sync, 0, kSyncWords * sizeof(uint32_t), cs);
     if (e == cudaSuccess)
-      e = launch_tf_batched(s, *w, base_logits, S0, tokens, ws.Gx, SB, ws, st, spin_limit(), cs);
+      e = tf_units_ok(s) ? launch_tf_units(s, *w, S0, tokens, ws.Gx, SB, ws, st, spin_limit(), cs)
+                         : launch_tf_batched(s, *w, base_logits, S0, tokens, ws.Gx, SB, ws, st, spin_limit(), cs);
   }
   for (int i = 0; i + 1 < s.L && e == cudaSuccess && !batched; ++i) {
     if (tc)

@@ -68,6 +68,13 @@ template <class Epi, class = void> struct WarpCoop {
 template <class Epi> struct WarpCoop<Epi, std::void_t<decltype(Epi::kWarpCoop)>> {
   static constexpr bool value = Epi::kWarpCoop;
 };
+// Static shared memory an epilogue declares (kStaticSmem), which the stage ring must leave room for.
+template <class Epi, class = void> struct StaticSmemOf {
+  static constexpr size_t value = 0;
+};
+template <class Epi> struct StaticSmemOf<Epi, std::void_t<decltype(Epi::kStaticSmem)>> {
+  static constexpr size_t value = Epi::kStaticSmem;
+};
 template <class Epi> struct EpiWarps {
   static constexpr int kGroups = GroupsOf<Epi>::value;
   static constexpr int kThreads = 64 + 128 * kGroups;
@@ -152,27 +159,24 @@ struct EpiLogitsT {  // logits[n][m] = D + Lb[n][m]   (m = vocabulary row, n = (
 // 32 rows x 16 columns go to shared memory (16-byte chunks XOR-swizzled so that neither side has
 // bank conflicts) and come back so that each store instruction writes whole 64-byte (fp32) or
 // 32-byte (bf16) row segments -- 8 or 16 rows per instruction instead of 32 scattered 16-byte
-// pieces.  Every lane of the warp calls apply with the same n0.  Each thread also loads the L_base
-// of its next 16-column group (the next call's, within the tile) before storing this one, so that
-// the load's latency overlaps the stores.
+// pieces.  Every lane of the warp calls apply with the same n0.  L_base arrives as the side tile
+// (rows m, columns n of the output tile, by TMA one tile ahead), so the epilogue issues no loads.
 template <typename OutT>
 struct EpiLogitsRowT {
-  static constexpr bool kSide = false;
+  static constexpr bool kSide = true;
   static constexpr bool kARes = false;
   static constexpr int kGroups = 2;  // the epilogue is the longest phase of a tile: two warps per lane quadrant
   static constexpr bool kWarpCoop = true;
-  struct State {
-    uint4 la, lb;  // L_base of (pm, pn .. pn + 15), loaded ahead
-    int pm, pn;
-  };
+  static constexpr size_t kStaticSmem = 8 * 32 * 16 * 4;  // the staging buffers below
+  using State = NoState;
   const bf16* Lb;
   OutT* logits;
   int M;
   long long ld;
-  __device__ __forceinline__ void init(State& st) const { st.pm = -1; st.pn = -1; }
+  __device__ __forceinline__ void init(State&) const {}
   __device__ __forceinline__ void finish(State&, int) const {}
-  __device__ __forceinline__ void apply(State& st, int m, int n0, const float (&v)[16], int N, const uint8_t*, int,
-                                        int) const {
+  __device__ __forceinline__ void apply(State&, int m, int n0, const float (&v)[16], int N, const uint8_t* side,
+                                        int row, int c0) const {
     const int lane = threadIdx.x & 31;
     if (n0 + 16 <= N) {  // warp-uniform
       // per epilogue warp: 32 rows x 16 values (fp32: 64 B a row, four 16-byte chunks)
@@ -180,24 +184,9 @@ struct EpiLogitsRowT {
       uint32_t* sw = stage[((threadIdx.x >> 5) - 2) & 7];
       float z[16];
       if (m < M) {
-        const bf16* lr = Lb + (size_t)m * ld + n0;
-        uint4 qa, qb;
-        if (st.pm == m && st.pn == n0) {
-          qa = st.la;
-          qb = st.lb;
-        } else {
-          qa = __ldg(reinterpret_cast<const uint4*>(lr));
-          qb = __ldg(reinterpret_cast<const uint4*>(lr) + 1);
-        }
-        if (n0 + 32 <= N) {  // the next group of this row
-          st.la = __ldg(reinterpret_cast<const uint4*>(lr + 16));
-          st.lb = __ldg(reinterpret_cast<const uint4*>(lr + 16) + 1);
-          st.pm = m;
-          st.pn = n0 + 16;
-        }
         float a[8], b[8];
-        widen(qa, a);
-        widen(qb, b);
+        widen(*side_chunk(side, row, c0), a);
+        widen(*side_chunk(side, row, c0 + 8), b);
 #pragma unroll
         for (int j = 0; j < 8; ++j) { z[j] = v[j] + a[j]; z[8 + j] = v[8 + j] + b[j]; }
       } else {
@@ -426,7 +415,7 @@ __device__ __forceinline__ void st_cluster_f4(uint32_t addr, float a, float b, f
 // [two side tiles][split-K receive buffer], plus 1024 bytes of slack for the alignment.  With a
 // resident A (K <= 256, one 128-row band of M) each stage carries two k-blocks of B; otherwise one
 // k-block of A and B.
-template <int BN, bool SIDE, bool ARES, bool SPLIT = false> struct Cfg {
+template <int BN, bool SIDE, bool ARES, bool SPLIT = false, size_t STATIC = 0> struct Cfg {
   static constexpr uint32_t kBBytes = BN * kBK * 2;
   static constexpr int kKBS = ARES ? 2 : 1;
   static constexpr uint32_t kStage = ARES ? kKBS * kBBytes : kABytes + kBBytes;
@@ -435,7 +424,8 @@ template <int BN, bool SIDE, bool ARES, bool SPLIT = false> struct Cfg {
   static constexpr int kUnits = kBM * BN / 16;
   // ks * ceil(kUnits / ks) slots of 64 bytes, for any ks <= 8
   static constexpr size_t kRecvBytes = SPLIT ? (size_t)(kUnits + 8) * 64 : 0;
-  static constexpr size_t kBudget = 232448 - 2048 - 2 * kSideBytes - kAResBytes - kRecvBytes;  // 227 KB per CTA
+  // 227 KB per CTA, less the epilogue's static shared memory (STATIC)
+  static constexpr size_t kBudget = 232448 - STATIC - 2048 - 2 * kSideBytes - kAResBytes - kRecvBytes;
   static constexpr int kStagesFit = (int)(kBudget / kStage);
   static constexpr int kStages = kStagesFit > 8 ? 8 : kStagesFit;
   static constexpr int kTmemCols = (2 * BN) <= 32 ? 32 : ((2 * BN) <= 64 ? 64 : ((2 * BN) <= 128 ? 128 : ((2 * BN) <= 256 ? 256 : 512)));
@@ -451,7 +441,7 @@ __global__ void __launch_bounds__(EpiWarps<Epi>::kThreads, 1)
               int a_stream, int indep, uint32_t* __restrict__ claim, uint32_t epoch,
               unsigned long long* __restrict__ trace, int mfirst) {
   static_assert(!SPLIT || (!Epi::kSide && !Epi::kARes), "split-K needs a plain epilogue");
-  using C = Cfg<BN, Epi::kSide, Epi::kARes, SPLIT>;
+  using C = Cfg<BN, Epi::kSide, Epi::kARes, SPLIT, StaticSmemOf<Epi>::value>;
   constexpr int S = C::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* ares = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
@@ -924,7 +914,7 @@ cudaError_t launch_gemm(const void* A, const void* Bm, int M, int N, int K, cons
   }
   if (ksplit > 1) return cudaErrorInvalidValue;
   auto kern = k_gemm_tc<BN, Epi, false>;
-  const size_t smem = Cfg<BN, Epi::kSide, Epi::kARes>::kSmem;
+  const size_t smem = Cfg<BN, Epi::kSide, Epi::kARes, false, StaticSmemOf<Epi>::value>::kSmem;
   cudaError_t e = set_smem_once<BN, Epi, false>(smem);
   if (e != cudaSuccess) return e;
   const int grid = (int)grid_ctas;
@@ -1079,6 +1069,19 @@ bool tmap_bf16_3d(CUtensorMap* tm, const void* base, uint64_t n0, uint64_t n1, u
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+bool tmap_bf16_chunks(CUtensorMap* tm, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows,
+                      uint32_t box_chunks) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn || cols % kBK != 0) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)kBK, rows, cols / kBK};
+  cuuint64_t strides[2] = {cols * 2, (cuuint64_t)kBK * 2};
+  cuuint32_t box[3] = {(cuuint32_t)kBK, box_rows, box_chunks};
+  cuuint32_t es[3] = {1, 1, 1};
+  return fn(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 int sm_count() {
   int dev = 0, n = 0;
   cudaGetDevice(&dev);
@@ -1167,7 +1170,7 @@ cudaError_t logits_t(const bf16* W2, const bf16* U, int V, int N, int r, const b
       if (e != cudaSuccess) return e;
     }
     EpiLogitsRowT<OutT> e{Lb, logits, N, (long long)V};
-    return launch_gemm<256>(U, W2, N, V, r, e, status, limit, st, 0, 0, 0, nullptr, 0, nullptr, 0, 0, 1, 0, 2,
+    return launch_gemm<128>(U, W2, N, V, r, e, status, limit, st, 0, 0, 0, Lb, (uint64_t)V, nullptr, 0, 0, 1, 0, 2,
                             claim, epoch, 1);
   }
   EpiLogitsT<OutT> e{Lb, logits, V};

@@ -20,6 +20,11 @@ bool tmap_bf16_tiles(CUtensorMap* tm, const void* base, uint64_t rows, uint64_t 
 // swizzling: one box is box2 rows of 64 elements at one index of the middle dimension, laid out in
 // shared memory as a box_rows x 64 tile of tmap_bf16_tiles.  n0 must be a multiple of 8.
 bool tmap_bf16_3d(CUtensorMap* tm, const void* base, uint64_t n0, uint64_t n1, uint64_t n2, uint32_t box2);
+// bf16 matrix [rows][cols] (row-major, cols a multiple of 64) seen as 64-column chunks: one box is
+// box_chunks consecutive chunks of box_rows rows, laid out in shared memory chunk by chunk, each a
+// box_rows x 64 tile of tmap_bf16_tiles (128-byte swizzle).
+bool tmap_bf16_chunks(CUtensorMap* tm, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows,
+                      uint32_t box_chunks);
 // fp32 tensor [n2][n1][n0] (contiguous, n0 innermost, a multiple of 4) seen as boxes of
 // box0 x box1 x 1, no swizzle: a box is box1 rows of box0 elements in shared memory.
 bool tmap_f32_3d(CUtensorMap* tm, void* base, uint64_t n0, uint64_t n1, uint64_t n2, uint32_t box0, uint32_t box1);

@@ -55,4 +55,14 @@ cudaError_t launch_tf_batched(const Shape& s, const domino_weights_t& w, const v
                               const int32_t* tokens, const float* Gx, float* states, const Workspace& ws,
                               int32_t* status, uint64_t spin, cudaStream_t st);
 
+// The unit-owned teacher-forced recurrence (tf_units.cu): every CTA owns eight state units and
+// keeps their W_hh rows in shared memory; one grid barrier per update.  Same contract as
+// launch_tf_batched (ws.S_hl's first 2B rows serve as its two split-state buffers); the caller
+// zeroes ws.sync first.
+bool tf_units_ok(const Shape& s);
+const char* tf_units_plan();
+cudaError_t launch_tf_units(const Shape& s, const domino_weights_t& w, const float* S0, const int32_t* tokens,
+                            const float* Gx, float* states, const Workspace& ws, int32_t* status, uint64_t spin,
+                            cudaStream_t st);
+
 }  // namespace domino

@@ -35,7 +35,7 @@ _TORCH_DTYPE = {DTYPE_F32: torch.float32, DTYPE_BF16: torch.bfloat16}
 EXPORTS = ("domino_workspace_bytes", "domino_draft_greedy", "domino_teacher_forced",
            "domino_accept_workspace_bytes", "domino_accept_len", "domino_status_string",
            "domino_abi_version", "domino_debug_set_spin_limit", "domino_launch_count",
-           "domino_greedy_plan", "domino_draft_greedy_noalloc", "domino_debug_set_trace",
+           "domino_greedy_plan", "domino_teacher_forced_plan", "domino_draft_greedy_noalloc", "domino_debug_set_trace",
            "domino_embed_proj_bytes", "domino_project_embeddings", "domino_arena_bytes",
            "domino_pack_weights", "domino_set_l2_persistence", "domino_debug_gemm",
            "domino_debug_read_passes", "domino_teacher_forced_ex", "domino_accept_sample_workspace_bytes",
@@ -98,6 +98,8 @@ def lib(path: str = LIB_PATH) -> ctypes.CDLL:
         L.domino_debug_set_trace.restype = ctypes.c_int
         L.domino_greedy_plan.argtypes = [ctypes.POINTER(Shape)]
         L.domino_greedy_plan.restype = ctypes.c_char_p
+        L.domino_teacher_forced_plan.argtypes = [ctypes.POINTER(Shape)]
+        L.domino_teacher_forced_plan.restype = ctypes.c_char_p
         L.domino_arena_bytes.argtypes = [ctypes.POINTER(Shape)]
         L.domino_arena_bytes.restype = sz
         L.domino_pack_weights.argtypes = [ctypes.POINTER(Shape), ctypes.POINTER(Weights), vp, sz,
@@ -136,6 +138,11 @@ def launch_count() -> int:
 def greedy_plan(shape: Shape) -> str:
     """Which kernels draft_greedy runs for this shape."""
     return lib().domino_greedy_plan(ctypes.byref(shape)).decode()
+
+
+def teacher_forced_plan(shape: Shape) -> str:
+    """Which kernels teacher_forced runs for this shape (weights without the projection table)."""
+    return lib().domino_teacher_forced_plan(ctypes.byref(shape)).decode()
 
 
 def set_trace(buf) -> None:

@@ -258,6 +258,10 @@ DOMINO_API uint64_t domino_launch_count(void);
  * (e.g. which fused kernel, or the per-phase kernels), or "invalid shape". */
 DOMINO_API const char* domino_greedy_plan(const domino_shape_t* shape);
 
+/* The same for domino_teacher_forced and domino_teacher_forced_ex (weights without the embedding
+ * projection table). */
+DOMINO_API const char* domino_teacher_forced_plan(const domino_shape_t* shape);
+
 /* Greedy drafting without a workspace, for callers that cannot allocate device memory.
  *
  * The pages have no counterpart: this is a deployment convenience of this library.  Callers

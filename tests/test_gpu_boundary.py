@@ -23,15 +23,15 @@ def _small(B=2, L=6, dtype=1, seed=200):
     return synth.make_workload(wl, with_tokens=True)
 
 
-@pytest.mark.parametrize("shape", ["per-phase", "batched"])
+@pytest.mark.parametrize("shape", ["per-phase", "unit-owned"])
 def test_bad_teacher_forcing_token_sets_status(shape):
     if shape == "per-phase":
         data = _small()
-    else:  # the persistent batched kernel's recurrence (5 <= B <= 128, Hs a multiple of 128)
+    else:  # the unit-owned recurrence (5 <= B <= 128, Hs a multiple of 128 up to 1024)
         data = synth.make_workload(dict(B=8, L=6, d=256, Hs=128, r=128, V=2000, dtype=1, weight_seed=260,
                                         input_seed=261, s0_std=0.2, peak=2.0, name="bad-token"), with_tokens=True)
         w, _, _, _ = G.device_inputs(data)
-        assert "k_greedy_batched" in domino.greedy_plan(domino.make_shape(w, 8, 6))
+        assert "k_tf_units" in domino.teacher_forced_plan(domino.make_shape(w, 8, 6))
     w, lb, h, S0 = G.device_inputs(data)
     y = torch.from_numpy(data["tokens"]).cuda()
     y[1, 2] = 5000  # V = 2000
@@ -141,6 +141,33 @@ def test_bounded_barrier_gives_up_with_status_and_the_context_survives(B, Hs, pl
     torch.cuda.synchronize()
     assert int(status.item()) == 0
     assert torch.equal(again, good)
+
+
+@pytest.mark.parametrize("Hs,plan", [(128, "k_tf_units"), (1280, "k_greedy_batched")], ids=["unit-owned", "batched"])
+def test_teacher_forced_bounded_waits_give_up_with_status(Hs, plan):
+    """The teacher-forced recurrence kernels under a spin limit of one poll: the call reports
+    DOMINO_STATUS_DEVICE_TIMEOUT, and the next call with the default limit repeats the first
+    call's logits and states bit for bit."""
+    data = synth.make_workload(dict(B=8, L=6, d=256, Hs=Hs, r=128, V=2000, dtype=1, weight_seed=270,
+                                    input_seed=271, s0_std=0.2, peak=2.0, name="tf-timeout"), with_tokens=True)
+    w, lb, h, S0 = G.device_inputs(data)
+    assert plan in domino.teacher_forced_plan(domino.make_shape(w, 8, 6))
+    y = torch.from_numpy(data["tokens"]).cuda()
+    good, good_s = domino.teacher_forced(w, lb, h, S0, y, states_out=True)
+    torch.cuda.synchronize()
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    domino.set_spin_limit(1)
+    try:
+        domino.teacher_forced(w, lb, h, S0, y, status=status)
+        torch.cuda.synchronize()
+    finally:
+        domino.set_spin_limit(0)
+    assert int(status.item()) == domino.STATUS_DEVICE_TIMEOUT
+    status.zero_()
+    again, again_s = domino.teacher_forced(w, lb, h, S0, y, states_out=True, status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    assert torch.equal(again, good) and torch.equal(again_s, good_s)
 
 
 def test_persistent_and_per_phase_paths_agree():

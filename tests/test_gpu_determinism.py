@@ -63,7 +63,7 @@ def test_greedy_with_projection_table_repeats_bit_for_bit(B):
         assert torch.equal(x, y)
 
 
-@pytest.mark.parametrize("B,d,Hs", [(1, 4096, 1024), (4, 1024, 512), (2, 512, 256)])
+@pytest.mark.parametrize("B,d,Hs", [(1, 4096, 1024), (4, 1024, 512), (2, 512, 256), (32, 1024, 1024), (100, 512, 256)])
 def test_teacher_forced_repeats_bit_for_bit(B, d, Hs):
     data = _case(B, 16, d, Hs, 9000, 660 + B)
     w, lb, h, S0 = G.device_inputs(data)

@@ -61,12 +61,29 @@ def test_greedy_small(wl):
 TF_CASES = SMALL[1:4] + [
     _custom(20, 16, 512, 256, 256, 3000, 1, 230),   # B*L = 320: two column tiles, ragged vocabulary tile
     _custom(1, 7, 256, 256, 128, 1024, 1, 240),     # exactly 8 vocabulary tiles, 7 positions
+    # the unit-owned recurrence (k_tf_units): four, two and one row groups per A tile, a W_hh chunk
+    # count that halves the row groups (Hs = 128), a single update, a single position
+    _custom(5, 9, 256, 256, 128, 2000, 1, 250),
+    _custom(40, 6, 256, 256, 128, 3000, 1, 252),
+    _custom(100, 5, 256, 512, 128, 2000, 1, 254),
+    _custom(30, 4, 128, 128, 128, 1504, 1, 256),
+    _custom(12, 2, 256, 256, 128, 1000, 1, 258),
+    _custom(12, 1, 256, 256, 128, 1000, 1, 260),
+    # Hs above the unit-owned kernel's limit: the batched kernel's teacher-forced mode
+    _custom(9, 4, 256, 1280, 128, 2000, 1, 262),
 ]
+TF_PLANS = {250: "k_tf_units", 252: "k_tf_units", 254: "k_tf_units", 256: "k_tf_units", 258: "k_tf_units",
+            260: "k_tf_units", 262: "k_greedy_batched", 230: "k_tf_units"}
 
 
 @pytest.mark.parametrize("wl", TF_CASES, ids=lambda w: w["name"] + f"-B{w['B']}")
 def test_teacher_forced_small(wl):
     data = synth.make_workload(wl, with_tokens=True)
+    seed = wl["weight_seed"]
+    if seed in TF_PLANS:
+        from draft_block_causal_b200 import domino
+        w, _, _, _ = G.device_inputs(data)
+        assert TF_PLANS[seed] in domino.teacher_forced_plan(domino.make_shape(w, wl["B"], wl["L"]))
     res = G.tf_parity(data)
     print(wl["name"], res)
 

@@ -71,9 +71,11 @@ TF_CASES = SMALL[1:4] + [
     _custom(12, 1, 256, 256, 128, 1000, 1, 260),
     # Hs above the unit-owned kernel's limit: the batched kernel's teacher-forced mode
     _custom(9, 4, 256, 1280, 128, 2000, 1, 262),
+    # logits GEMM with three row bands over more vocabulary tiles than SMs (a CTA meets several bands)
+    _custom(20, 16, 256, 256, 256, 24008, 1, 264),
 ]
 TF_PLANS = {250: "k_tf_units", 252: "k_tf_units", 254: "k_tf_units", 256: "k_tf_units", 258: "k_tf_units",
-            260: "k_tf_units", 262: "k_greedy_batched", 230: "k_tf_units"}
+            260: "k_tf_units", 262: "k_greedy_batched", 230: "k_tf_units", 264: "k_tf_units"}
 
 
 @pytest.mark.parametrize("wl", TF_CASES, ids=lambda w: w["name"] + f"-B{w['B']}")

@@ -128,6 +128,19 @@ def test_greedy_batch_sweep_every_row(B, peak):
     print(B, peak, {k: v for k, v in res.items() if k != "tokens"})
 
 
+@pytest.mark.parametrize("B", [16, 64, 128])
+def test_teacher_forced_sweep_every_row(B):
+    """Teacher forcing at the Qwen3-8B widths with four, two and one row groups per A tile of the
+    unit-owned recurrence: every row's logits and states against the oracle."""
+    from draft_block_causal_b200 import domino
+    wl = synth.workload("qwen3-8b-head-sweep", B=B, peak=2.0)
+    data = synth.make_workload(wl, with_tokens=True)
+    w, _, _, _ = G.device_inputs(data)
+    assert "k_tf_units" in domino.teacher_forced_plan(domino.make_shape(w, B, wl["L"]))
+    res = G.tf_parity_rows(data)
+    print(B, res)
+
+
 def test_accept_length_constructed_prefixes():
     rng = np.random.default_rng(7)
     B, L, V = 40, 16, 151936

@@ -192,7 +192,7 @@ const char* domino_teacher_forced_plan(const domino_shape_t* shape) {
            "recurrence), then tcgen05 GEMMs for the activations and the logits of all positions";
   if (tc && batched_shape_ok(s))
     return tf_units_ok(s) ? "embedding gather + tcgen05 W_ih GEMM over all given tokens, k_tf_units (the recurrence: "
-                            "each CTA owns eight state units, one grid barrier per update), then tcgen05 GEMMs for the "
+                            "each CTA owns eight state units, loads gated by a write counter), then tcgen05 GEMMs for the "
                             "activations and the logits of all positions"
                           : "embedding gather + tcgen05 W_ih GEMM over all given tokens, k_greedy_batched in "
                             "teacher-forced mode (the recurrence), then tcgen05 GEMMs for the activations and the "

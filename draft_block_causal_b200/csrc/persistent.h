@@ -56,7 +56,7 @@ cudaError_t launch_tf_batched(const Shape& s, const domino_weights_t& w, const v
                               int32_t* status, uint64_t spin, cudaStream_t st);
 
 // The unit-owned teacher-forced recurrence (tf_units.cu): every CTA owns eight state units and
-// keeps their W_hh rows in shared memory; one grid barrier per update.  Same contract as
+// keeps their W_hh rows in shared memory; no grid barrier (a write counter).  Same contract as
 // launch_tf_batched (ws.S_hl's first 2B rows serve as its two split-state buffers); the caller
 // zeroes ws.sync first.
 bool tf_units_ok(const Shape& s);

@@ -1,5 +1,6 @@
 // tf_units.cu -- the teacher-forced GRU recurrence for 5..128 batch rows in one cooperative launch
-// in which every CTA owns eight state units, so that an update costs one grid barrier.
+// in which every CTA owns eight state units, so that an update needs no partial sums in global
+// memory and no grid barrier.
 //
 // Domino review page, section 二 ("Teacher Forcing"): with the tokens y given, every state follows
 // from the previous one, S_i = GRUCell(embed[y_i], S_{i-1}), in the PyTorch gate form
@@ -15,8 +16,12 @@
 //   warp 1      issues tcgen05.mma: D[row][gate row] += S_hl[row][k] . W_hh[gate row][k mod Hs];
 //   warps 4..7  read the accumulator (TMEM lane = batch row), apply the cell to the CTA's units and
 //               write the new states, the states output and their split for every CTA's next update.
-// The split state is double-buffered (update i reads buffer i & 1 and writes the other), so one
-// grid barrier per update orders every write before every read.
+// The split state is double-buffered (update i reads buffer i & 1 and writes the other).  Instead of
+// a grid barrier, every CTA counts its writes of the state on one ready counter, and only the
+// producer thread waits (bounded) for the count before loading; the other roles wait on their
+// mbarriers as usual.  A CTA writes a buffer only after it has read the other one whole, which
+// needs every CTA's previous cell, which came after that CTA's last read of the buffer being
+// written: no write can overtake a read.
 //
 // Small batches fill the 128-row A tile with K: at B <= 32 (64) a tile carries four (two) K chunks
 // of the state, one per row group of 32 (64) rows, and the B operand stacks the matching W_hh chunks
@@ -24,7 +29,7 @@
 // accumulator are discarded, and the epilogue adds the groups' blocks in group order, so the result
 // does not depend on timing.
 //
-// Every mbarrier wait and the grid barrier are bounded: a role that gives up raises the CTA's abort
+// Every mbarrier wait and every counter wait is bounded: a role that gives up raises the CTA's abort
 // flag, waits (bounded) for its copies and MMAs in flight, and the kernel reports
 // DOMINO_STATUS_DEVICE_TIMEOUT.
 #include "common.cuh"
@@ -65,13 +70,13 @@ struct TfArgs {
   const bf16* b_hh;       // [3Hs]
   float* states;          // [B][L][Hs]
   bf16* S_hl;             // [2][B][2Hs] split state, double-buffered
-  unsigned* bar;          // grid barrier counter (zero before the launch)
+  unsigned* ready;        // the CTAs' state writes, counted (zero before the launch)
   int32_t* status;
   int B, L, Hs, V;
   int chunks3d;           // the split-state map is tmap_bf16_chunks (one box per A tile), else 2-D
   unsigned long long limit;
-  unsigned long long* trace;  // optional (globaltimer, ns): [0] CTA 0's start, [e] when CTA 0 passed
-  int ntrace;                 // grid barrier e, then its end; from kTfTraceMarks, per CTA c the
+  unsigned long long* trace;  // optional (globaltimer, ns): [0] CTA 0's start, [e] when CTA 0 ended
+  int ntrace;                 // update e - 1 (e = 1: its set-up), then its end; from kTfTraceMarks, per CTA c the
                               // milestones k of update 1 at [kTfTraceMarks + k * G + c] (k: 0 start,
                               // 1 copies issued, 2 copies landed, 3 MMAs issued, 4 accumulator in the
                               // epilogue, 5 epilogue done).  Entries past ntrace are not written.
@@ -157,7 +162,6 @@ __global__ void __launch_bounds__(kTfThreads, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(red) + kTfRed);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kTBars);
   volatile int* abort_s = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  volatile int* flag_s = reinterpret_cast<volatile int*>(tmem_slot + 2);  // [2]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int B = p.B, L = p.L, Hs = p.Hs, H3 = 3 * Hs, G = gridDim.x;
@@ -217,42 +221,31 @@ __global__ void __launch_bounds__(kTfThreads, 1)
                   p.S_hl + (size_t)b * 2 * Hs + Hs + j0 + u0);
   }
 
-  unsigned epoch = 0;
-  // Grid barrier over a monotonic counter (the e-th waits for e * G arrivals).  The split state is
-  // written by the epilogue warps (generic proxy) and read by the next update's TMA copies, which
-  // thread 0 issues: the writers fence towards the async proxy before arriving, thread 0 after
-  // passing.  The pass flag alternates between two words, so one CTA barrier suffices after it.
-  auto grid_sync = [&]() -> bool {
-    tmem_fence_before_sync();
-    if (warp >= 4) tf_fence_proxy_global();
-    __syncthreads();
-    ++epoch;
-    if (threadIdx.x == 0) {
+  // The CTA's units of the new state are written (epilogue warps): count them on the ready counter.
+  // The writers fence towards the async proxy (the readers load by TMA), the epilogue warps meet,
+  // and one thread publishes with release semantics.
+  auto signal_written = [&]() {
+    tf_fence_proxy_global();
+    asm volatile("bar.sync 2, %0;" ::"r"(128) : "memory");
+    if (warp == 4 && lane == 0) {
       __threadfence();
-      atomicAdd(p.bar, 1u);
-      const unsigned target = epoch * (unsigned)G;
-      bool ok = *abort_s == 0;
-      if (ok) {
-        ok = false;
-        for (unsigned long long it = 0; it < limit; ++it) {
-          if (tf_ld_acquire(p.bar) >= target) { ok = true; break; }
-          if ((it & 31) == 31 && tf_ld_relaxed(p.status) == DOMINO_STATUS_DEVICE_TIMEOUT) break;
-        }
-      }
-      if (!ok) set_status(p.status, DOMINO_STATUS_DEVICE_TIMEOUT);
-      __threadfence();
-      tf_fence_proxy_global();
-      flag_s[epoch & 1u] = ok ? 1 : 0;
-      if (tracer && (int)epoch < p.ntrace) p.trace[epoch] = globaltimer_ns();
+      atomicAdd(p.ready, 1u);
     }
-    __syncthreads();
-    tmem_fence_after_sync();
-    return flag_s[epoch & 1u] != 0;
   };
+  // Producer: the state holds the writes of update i - 1 (the set-up counts as update -1) once every
+  // CTA has counted i + 1 writes.
+  auto wait_ready = [&](unsigned target) -> bool {
+    for (unsigned long long it = 0; it < limit; ++it) {
+      if (tf_ld_acquire(p.ready) >= target) return true;
+      if ((it & 31) == 31 && (*abort_s || tf_ld_relaxed(p.status) == DOMINO_STATUS_DEVICE_TIMEOUT)) break;
+    }
+    set_status(p.status, DOMINO_STATUS_DEVICE_TIMEOUT);
+    return false;
+  };
+  if (warp >= 4) signal_written();
 
-  bool ok = grid_sync();
   uint32_t it0 = 0;  // A tiles gone through the ring before this update
-  for (int i = 0; i + 1 < L && ok; ++i) {
+  for (int i = 0; i + 1 < L; ++i) {
     const int rb = (i & 1) * B;  // first row of the buffer this update reads
     auto mark = [&](int k) {
       const long long e = kTfTraceMarks + (long long)k * G + blockIdx.x;
@@ -261,9 +254,12 @@ __global__ void __launch_bounds__(kTfThreads, 1)
     if (threadIdx.x == 0) mark(0);
     if (warp == 0) {
       if (lane == 0) {  // TMA producer: the split state, GR K chunks per A tile
-        bool good = true;
+        // the whole state first, then one proxy fence (a fence between copies would wait for the
+        // ones in flight)
+        bool good = wait_ready((unsigned)G * (unsigned)(i + 1));
+        tf_fence_proxy_global();
         uint32_t it = it0;
-        for (int t = 0; t < nst; ++t, ++it) {
+        for (int t = 0; t < nst && good; ++t, ++it) {
           const int st = it % kTfStages;
           if (!mbar_wait_bounded(&bars[kTEmpty + st], ((it / kTfStages) & 1u) ^ 1u, limit, abort_s)) {
             good = false;
@@ -368,10 +364,16 @@ __global__ void __launch_bounds__(kTfThreads, 1)
         bf16* hl = p.S_hl + ((size_t)(B - rb) + b) * 2 * Hs;  // the other buffer
         put_units<NU>(s, p.states + ((size_t)b * L + i + 1) * Hs + j0 + u0, hl + j0 + u0, hl + Hs + j0 + u0);
       }
+      signal_written();
       if (warp == 4 && lane == 0) mark(5);
     }
     it0 += (uint32_t)nst;
-    ok = grid_sync();
+    // the next update's MMAs overwrite the accumulator the epilogue has just read
+    tmem_fence_before_sync();
+    const bool stop = __syncthreads_or(*abort_s != 0);
+    tmem_fence_after_sync();
+    if (tracer && i + 2 < p.ntrace) p.trace[i + 2] = globaltimer_ns();
+    if (stop) break;
   }
 
   if (warp == 0 && lane == 0) {  // the W_hh copies have landed (a call with no update never waited)
@@ -383,7 +385,7 @@ __global__ void __launch_bounds__(kTfThreads, 1)
   tmem_fence_after_sync();
   if (warp == 1) tmem_dealloc(tbase, kTfTmemCols);
   if (threadIdx.x == 0 && *abort_s) set_status(p.status, DOMINO_STATUS_DEVICE_TIMEOUT);
-  if (tracer && (int)epoch + 1 < p.ntrace) p.trace[epoch + 1] = globaltimer_ns();
+  if (tracer && L + 1 < p.ntrace) p.trace[L + 1] = globaltimer_ns();
 }
 
 int g_tf_fit[64];  // per device: 0 unknown, 1 fits, -1 does not
@@ -424,7 +426,8 @@ bool tf_units_ok(const Shape& s) {
 
 const char* tf_units_plan() {
   return "k_tf_units: one cooperative launch, each CTA owning eight state units with their W_hh rows in shared "
-         "memory, per update a tcgen05 product of the split state and the cell, one bounded grid barrier";
+         "memory, per update a tcgen05 product of the split state and the cell; the next update's loads wait on "
+         "a counter of the CTAs' state writes";
 }
 
 cudaError_t launch_tf_units(const Shape& s, const domino_weights_t& w, const float* S0, const int32_t* tokens,
@@ -448,7 +451,7 @@ cudaError_t launch_tf_units(const Shape& s, const domino_weights_t& w, const flo
   a.b_hh = (const bf16*)w.b_hh;
   a.states = states;
   a.S_hl = ws.S_hl;
-  a.bar = ws.sync;
+  a.ready = ws.sync;
   a.status = status;
   a.B = s.B; a.L = s.L; a.Hs = s.Hs; a.V = s.V;
   a.chunks3d = c3 ? 1 : 0;

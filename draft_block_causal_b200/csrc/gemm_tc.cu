@@ -990,12 +990,9 @@ SkinnyPlan plan_skinny(int M, int N, int K) {
   SkinnyPlan best{16, 1};
   if (sms <= 0) return best;
   double best_cost = 1e300;
-  // 256-column tiles only where N is wider than two 128-column tiles (their split-K receive buffer
-  // leaves room for two stages)
-  const int bns[5] = {16, 32, 64, 128, 256};
+  const int bns[4] = {16, 32, 64, 128};
   for (int bn : bns) {
     if (bn > 16 && (bn / 2) >= N) break;  // wider tiles only add padding
-    if (bn == 256 && N <= 256) break;
     const long long tiles = m_tiles * ((N + bn - 1) / bn);
     for (int ks = 1; ks <= 8; ++ks) {
       double cost;
@@ -1004,11 +1001,9 @@ SkinnyPlan plan_skinny(int M, int N, int K) {
         cost = (double)waves * (kBM + bn) * 2.0 * K;
       } else {
         if (kblocks < 2 * ks || tiles * ks > sms) break;
-        const int fit = bn == 16    ? max_clusters<16, Epi>(ks)
-                        : bn == 32  ? max_clusters<32, Epi>(ks)
-                        : bn == 64  ? max_clusters<64, Epi>(ks)
-                        : bn == 128 ? max_clusters<128, Epi>(ks)
-                                    : max_clusters<256, Epi>(ks);
+        const int fit = bn == 16 ? max_clusters<16, Epi>(ks)
+                                 : bn == 32 ? max_clusters<32, Epi>(ks)
+                                            : bn == 64 ? max_clusters<64, Epi>(ks) : max_clusters<128, Epi>(ks);
         if (tiles > fit) continue;
         cost = (double)(kBM + bn) * 2.0 * ((kblocks + ks - 1) / ks) * kBK + 2.0 * kBM * bn * 4.0;
       }
@@ -1038,9 +1033,6 @@ cudaError_t launch_gemm_skinny(const void* A, const void* Bm, int M, int N, int 
     case 64:
       return launch_gemm<64>(A, Bm, M, N, K, epi, status, limit, st, lda, 0, a_kwrap, nullptr, 0, A2, a_split, lda2,
                              p.ks, a_stream, indep);
-    case 256:
-      return launch_gemm<256>(A, Bm, M, N, K, epi, status, limit, st, lda, 0, a_kwrap, nullptr, 0, A2, a_split,
-                              lda2, p.ks, a_stream, indep);
     default:
       return launch_gemm<128>(A, Bm, M, N, K, epi, status, limit, st, lda, 0, a_kwrap, nullptr, 0, A2, a_split,
                               lda2, p.ks, a_stream, indep);

@@ -47,25 +47,13 @@ def test_forced_plans_match_float64(bn, ks):
 
 
 @pytest.mark.parametrize("M,N,K,trans", [(3072, 128, 4096, True), (3328, 32, 2048, True), (1000, 20, 192, False),
-                                         (1000, 20, 192, True), (128, 1, 64, True), (256, 256, 1024, False),
-                                         (3072, 480, 4096, True), (3328, 300, 2048, True)])
+                                         (1000, 20, 192, True), (128, 1, 64, True), (256, 256, 1024, False)])
 def test_automatic_plan_matches_float64(M, N, K, trans):
-    """Automatic plans, including 256-column tiles with a cluster split over K (N above 256, e.g.
-    the W_ih product over all 480 given tokens of a 32-row teacher-forced call)."""
     A, B = _operands(M, N, K, seed=M + N + K)
     ref = _reference(A, B)
     got = domino.debug_gemm(A, B, trans=trans)
     torch.cuda.synchronize()
     _check(got.T if trans else got, ref, K)
-    if N > 256:  # split partials are added in piece order: repeats are bit-identical
-        again = domino.debug_gemm(A, B, trans=trans)
-        torch.cuda.synchronize()
-        assert torch.equal(got, again)
-
-
-def test_wide_batches_take_256_column_tiles():
-    shape = domino.Shape(480, 16, 4096, 1024, 256, 151936, 1)  # the per-phase path's W_ih product, N = 480
-    assert "tiles 128x256" in domino.greedy_plan(shape)
 
 
 @pytest.mark.parametrize("ks", [1, 4])

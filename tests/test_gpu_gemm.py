@@ -47,7 +47,8 @@ def test_forced_plans_match_float64(bn, ks):
 
 
 @pytest.mark.parametrize("M,N,K,trans", [(3072, 128, 4096, True), (3328, 32, 2048, True), (1000, 20, 192, False),
-                                         (1000, 20, 192, True), (128, 1, 64, True), (256, 256, 1024, False)])
+                                         (1000, 20, 192, True), (128, 1, 64, True), (256, 256, 1024, False),
+                                         (3072, 480, 4096, True)])
 def test_automatic_plan_matches_float64(M, N, K, trans):
     A, B = _operands(M, N, K, seed=M + N + K)
     ref = _reference(A, B)

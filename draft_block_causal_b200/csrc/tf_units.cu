@@ -81,7 +81,7 @@ struct TfArgs {
                               // 1 copies issued, 2 copies landed, 3 MMAs issued, 4 accumulator in the
                               // epilogue, 5 epilogue done).  Entries past ntrace are not written.
 };
-constexpr int kTfTraceMarks = 64;
+constexpr int kTfTraceMarks = 128;  // past CTA 0's stamps (L + 2 <= 66 entries)
 
 __device__ __forceinline__ unsigned tf_ld_acquire(const unsigned* p) {
   unsigned v;
@@ -244,6 +244,7 @@ __global__ void __launch_bounds__(kTfThreads, 1)
   };
   if (warp >= 4) signal_written();
 
+  if (tracer && 1 < p.ntrace) p.trace[1] = globaltimer_ns();
   uint32_t it0 = 0;  // A tiles gone through the ring before this update
   for (int i = 0; i + 1 < L; ++i) {
     const int rb = (i & 1) * B;  // first row of the buffer this update reads

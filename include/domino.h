@@ -301,7 +301,11 @@ DOMINO_API int domino_draft_greedy_noalloc(const domino_shape_t* shape, const do
  * partials done, 7: state barrier passed}.  The persistent batched kernel (5..128 rows) records the
  * globaltimer (ns) of CTA 0: [0] start, [e] when it passed grid barrier e (phases C0, D, E, then per
  * position A, B, C, D, E -- B absent with a projection table -- and A alone at the last position),
- * then its end.  NULL turns it off.  Process-wide. */
+ * then its end.  The teacher-forced recurrence of 5..128 rows (k_tf_units) records the globaltimer
+ * of CTA 0: [0] start, [1] set-up done, [i + 2] update i done, [L + 1] end; and, from entry 128,
+ * per CTA c the milestones k of update 1 at [128 + k * G + c] (G = Hs / 8 CTAs; k: 0 start, 1 copies
+ * issued, 2 copies landed, 3 MMAs issued, 4 accumulator in the epilogue, 5 cell done and counted).
+ * NULL turns it off.  Process-wide. */
 DOMINO_API int domino_debug_set_trace(void* device_buf, int32_t n_entries);
 
 /* Test and tuning hook for the tensor-core GEMM engine behind the batched paths:

@@ -15,7 +15,7 @@
 //   warp 0      streams the split state S_hl = [hi | lo] of every row (bf16, K = 2Hs) by TMA;
 //   warp 1      issues tcgen05.mma: D[row][gate row] += S_hl[row][k] . W_hh[gate row][k mod Hs];
 //   warps 4..7  read the accumulator (TMEM lane = batch row), apply the cell to the CTA's units and
-//               write the new states, the states output and their split for every CTA's next update.
+//               write the states output and the new split state for every CTA's next update.
 // The split state is double-buffered (update i reads buffer i & 1 and writes the other).  Instead of
 // a grid barrier, every CTA counts its writes of the state on one ready counter, and only the
 // producer thread waits (bounded) for the count before loading; the other roles wait on their
@@ -75,11 +75,12 @@ struct TfArgs {
   int B, L, Hs, V;
   int chunks3d;           // the split-state map is tmap_bf16_chunks (one box per A tile), else 2-D
   unsigned long long limit;
-  unsigned long long* trace;  // optional (globaltimer, ns): [0] CTA 0's start, [e] when CTA 0 ended
-  int ntrace;                 // update e - 1 (e = 1: its set-up), then its end; from kTfTraceMarks, per CTA c the
-                              // milestones k of update 1 at [kTfTraceMarks + k * G + c] (k: 0 start,
-                              // 1 copies issued, 2 copies landed, 3 MMAs issued, 4 accumulator in the
-                              // epilogue, 5 epilogue done).  Entries past ntrace are not written.
+  unsigned long long* trace;  // optional (globaltimer, ns): [0] CTA 0's start, [1] its set-up issued,
+  int ntrace;                 // [i + 2] its update i done, [L + 1] its end; from kTfTraceMarks, per
+                              // CTA c the milestones k of update 1 at [kTfTraceMarks + k * G + c]
+                              // (k: 0 start, 1 copies issued, 2 copies landed, 3 MMAs issued, 4
+                              // accumulator in the epilogue, 5 cell done and counted).  Entries past
+                              // ntrace are not written.
 };
 constexpr int kTfTraceMarks = 128;  // past CTA 0's stamps (L + 2 <= 66 entries)
 

@@ -302,7 +302,7 @@ DOMINO_API int domino_draft_greedy_noalloc(const domino_shape_t* shape, const do
  * globaltimer (ns) of CTA 0: [0] start, [e] when it passed grid barrier e (phases C0, D, E, then per
  * position A, B, C, D, E -- B absent with a projection table -- and A alone at the last position),
  * then its end.  The teacher-forced recurrence of 5..128 rows (k_tf_units) records the globaltimer
- * of CTA 0: [0] start, [1] set-up done, [i + 2] update i done, [L + 1] end; and, from entry 128,
+ * of CTA 0: [0] start, [1] set-up issued, [i + 2] update i done, [L + 1] end; and, from entry 128,
  * per CTA c the milestones k of update 1 at [128 + k * G + c] (G = Hs / 8 CTAs; k: 0 start, 1 copies
  * issued, 2 copies landed, 3 MMAs issued, 4 accumulator in the epilogue, 5 cell done and counted).
  * NULL turns it off.  Process-wide. */

@@ -53,3 +53,39 @@ def test_teacher_forcing_bytes():
     assert bench.tf_bytes(_sh(1)) == 214_806_592
     assert bench.tf_bytes(_sh(32)) - bench.tf_bytes(_sh(1)) == 31 * (
         16 * 151936 * 2 + 16 * 4096 * 2 + 15 * 4096 * 2 + 1024 * 4 + 16 * 4 + 16 * 151936 * 4)
+
+
+def test_near_gpu_placement_leaves_the_affinity_as_it_found_it(monkeypatch):
+    """The e2e pinned-buffer placement: with a fake NVML that names half of the allowed CPUs as the
+    GPU's nearest, the block runs on those and the previous affinity comes back afterwards; when the
+    query fails, nothing changes."""
+    import types
+    before = os.sched_getaffinity(0)
+    allowed = sorted(before)
+    near = set(allowed[: max(1, len(allowed) // 2)])
+    mask = [0] * ((max(allowed) // 64) + 1)
+    for c in near:
+        mask[c // 64] |= 1 << (c % 64)
+
+    class Props:
+        pci_domain_id = pci_bus_id = pci_device_id = 0
+
+    fake_torch = types.SimpleNamespace(cuda=types.SimpleNamespace(get_device_properties=lambda i: Props()))
+    fake_nvml = types.SimpleNamespace(nvmlInit=lambda: None, nvmlDeviceGetHandleByPciBusId=lambda bus: "h",
+                                      nvmlDeviceGetHandleByIndex=lambda i: "h",
+                                      nvmlDeviceGetCpuAffinity=lambda h, n: mask[:n] + [0] * max(0, n - len(mask)))
+    monkeypatch.setitem(sys.modules, "pynvml", fake_nvml)
+    monkeypatch.setitem(sys.modules, "torch", fake_torch)
+    with bench.NearGpu(0) as g:
+        inside = os.sched_getaffinity(0)
+    assert os.sched_getaffinity(0) == before
+    if near != before:
+        assert inside == near and "nearest the GPU" in g.describe()
+
+    def broken(*a):
+        raise RuntimeError("no NVML")
+
+    fake_nvml.nvmlInit = broken
+    with bench.NearGpu(0) as g:
+        assert os.sched_getaffinity(0) == before
+    assert g.describe() == "process CPU affinity unchanged"

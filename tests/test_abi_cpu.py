@@ -247,3 +247,5 @@ def test_projection_and_debug_entry_points_check_their_arguments(L):
     # the plan text of an invalid shape, and the CUDA-core kernels of fp32 storage
     assert L.domino_greedy_plan(ctypes.byref(_shape(B=0))) == b"invalid shape"
     assert b"k_w2" in L.domino_greedy_plan(ctypes.byref(_shape(dtype=0)))
+    assert L.domino_teacher_forced_plan(ctypes.byref(_shape(B=0))) == b"invalid shape"
+    assert b"k_gru" in L.domino_teacher_forced_plan(ctypes.byref(_shape(dtype=0)))

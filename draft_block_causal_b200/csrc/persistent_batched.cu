@@ -27,9 +27,10 @@
 // The last position runs phase A only.  Before position 0: C0 (the split of S0), D and E.  With
 // the embedding projection table phases X and B are skipped.
 //
-// Teacher forcing (given tokens) runs the recurrence only: C0, then per update D (W_hh . S, the
-// 3Hs gate rows alone) and C (the cell, with the gate inputs precomputed for every given token or
-// read from the projection table); the caller computes the activations and logits of all positions
+// Teacher forcing (given tokens) runs the recurrence only, for shapes the unit-owned recurrence
+// kernel (tf_units.cu) does not take (Hs above 1024): C0, then per update D (W_hh . S, the 3Hs gate
+// rows alone) and C (the cell, with the gate inputs precomputed for every given token or read from
+// the projection table); the caller computes the activations and logits of all positions
 // afterwards in two tensor-core GEMMs.
 //
 // Roles keep running counters of the stages, tiles and phases they have gone through, so the
